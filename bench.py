@@ -1,0 +1,404 @@
+"""Benchmark of the fused ZeRO-2/3 mixed-precision Adam step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole hot path (in-HBM reduce-scatter of the R
+rank gradients, Adam/AdamW on the fp32 masters and moments, round-to-nearest
+cast into the replicated 16-bit parameters) over one batch of synthetic
+gradients.  The default workload is the flat 16,777,259-parameter vector with
+R = 8 bf16 rank gradients (uneven owner slices), AdamW.  Prints one JSON line.
+
+Several GPUs (torchrun, one process per GPU) run independent replicas of the
+workload: the step has no exchange between GPUs in this configuration, so
+scaling is weak and no collective is on the data path; the only collectives
+are the barrier and the max-over-ranks reduction of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "fused ZeRO step: params updated/sec and HBM GB/s (% of B200 peak), 1 GPU"
+UNIT = "params/s"
+ADAMW = (1e-3, 0.8, 0.999, 1e-8, 3e-7)
+
+# name -> (kind, P or tensor-list builder, R, grad dtype, param dtype, fp16 loss scaling)
+WORKLOADS = {
+    "flat16m": ("flat", 16_777_259, 8, "bf16", "bf16", False),
+    "gpt2m": ("list", "gpt2m", 4, "f16", "f16", True),
+    "flat1p5b": ("flat", 1_500_000_000, 4, "bf16", "bf16", False),
+    "flat1p5b_f32": ("flat", 1_500_000_000, 4, "f32", "bf16", False),
+    "llama3b": ("list", "llama3b", 8, "bf16", "bf16", False),
+    # bandwidth sweep of the flat kernel, R = 8 bf16
+    "sweep1m": ("flat", 1 << 20, 8, "bf16", "bf16", False),
+    "sweep4m": ("flat", 1 << 22, 8, "bf16", "bf16", False),
+    "sweep64m": ("flat", 1 << 26, 8, "bf16", "bf16", False),
+    "sweep256m": ("flat", 1 << 28, 8, "bf16", "bf16", False),
+    "sweep1b": ("flat", 1 << 30, 8, "bf16", "bf16", False),
+    "sweep3p2b": ("flat", 3_212_749_824, 8, "bf16", "bf16", False),
+}
+GRAD_BYTES = {"bf16": 2, "f16": 2, "f32": 4}
+
+
+def bytes_per_param(R: int, gdt: str) -> int:
+    """Algorithmic HBM bytes per parameter: R gradient reads, fp32 master and
+    both moments read and written (24), one 16-bit parameter write (2)."""
+    return GRAD_BYTES[gdt] * R + 24 + 2
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in ("mixed_precision_adam_zero_b200/csrc/zero_adam_kernels.cuh",
+                "mixed_precision_adam_zero_b200/csrc/zero_adam_api.cu"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except OSError:
+        return {}
+
+
+def traffic_for(workload: str):
+    """DRAM bytes per launch of the step kernel from the committed ncu summary,
+    or None if there is none for the current kernel source."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except OSError:
+        return None
+    e = t.get(workload)
+    if not e or e.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = [(0x1, "gpu_idle"), (0x2, "applications_clocks_setting"), (0x4, "sw_power_cap"),
+               (0x8, "hw_slowdown"), (0x10, "sync_boost"), (0x20, "sw_thermal_slowdown"),
+               (0x40, "hw_thermal_slowdown"), (0x80, "hw_power_brake_slowdown"),
+               (0x100, "display_clock_setting")]
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.err = [], 0, None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report why
+            self.nvml, self.err = None, f"nvml unavailable: {e}"
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        n = self.nvml
+        get_reasons = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(n, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.h))
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.nvml is not None:
+            self._t.join()
+
+    def summary(self):
+        if self.nvml is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err or "no samples"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [name for bit, name in self.REASONS if self.reasons & bit and bit != 0x1],
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ workload
+
+def build_workload(name: str, device):
+    import torch
+    import synth
+    from mixed_precision_adam_zero_b200.buffers import FlatZero, ListZero
+    kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
+    wl = synth.WORKLOADS.get(name.split("_")[0], 9)
+    S = 65536.0 if scaled else 1.0
+    if kind == "flat":
+        z = FlatZero(size, R, gdt, pdt, device=device, loss_scale=S, two_set=scaled)
+        gbufs = z.grads
+    else:
+        tensors = synth.gpt2_medium_tensors() if size == "gpt2m" else synth.llama_3b_tensors()
+        numels = [n for _, n in tensors]
+        gt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
+        gbufs = [torch.empty(sum(numels), dtype=gt[gdt], device=device) for _ in range(R)]
+        pbuf = torch.empty(sum(numels), dtype=gt[pdt], device=device)
+        z = ListZero(numels, R, gdt, pdt, device=device, loss_scale=S, two_set=scaled,
+                     params16=list(pbuf.split(numels)), grads=[list(g.split(numels)) for g in gbufs])
+        z.flat_p16 = pbuf
+    z.load_master(synth.normal(z.P, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device))
+    for r, g in enumerate(gbufs):
+        synth.fill_normal_(g, 1e-3, synth.seed_for(wl, synth.KIND_GRAD, r, 1), scale=S)
+    z.gbufs = gbufs
+    z.check = scaled
+    return z
+
+
+def launches_per_step(z) -> int:
+    if not z.check:
+        return 1
+    return 2  # two-set single pass + the restore kernel (a no-op unless skipped)
+
+
+# ------------------------------------------------------------ arms
+
+def run_gpu(args) -> None:
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+
+    z = build_workload(args.workload, device)
+    stream = torch.cuda.current_stream(device)
+    step_args = z.step_args(hp=ADAMW, check=z.check)
+    from mixed_precision_adam_zero_b200 import zero_step_fused, zero_step_fused_list
+    if hasattr(z, "list"):
+        call = lambda: zero_step_fused_list(step_args, z.list, stream)
+    else:
+        call = lambda: zero_step_fused(step_args, stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    with ClockSampler(local) as clocks:
+        for i in range(K):
+            starts[i].record(stream)
+            call()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    per_launch_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
+
+    # end to end: host (pinned) gradients copied in, 16-bit parameters read back, every step
+    K_e2e = min(K, args.e2e_steps)
+    h2d = sum(g.numel() * g.element_size() for g in z.gbufs)
+    if h2d > (8 << 30):
+        K_e2e = 0          # pinned host copies of this workload would not fit comfortably
+    host_grads = [g.cpu().pin_memory() for g in z.gbufs] if K_e2e else []
+    p16 = z.flat_p16 if hasattr(z, "flat_p16") else z.params16
+    host_p16 = torch.empty(p16.shape, dtype=p16.dtype).pin_memory() if K_e2e else None
+    for _ in range(2 if K_e2e else 0):
+        for hg, dg in zip(host_grads, z.gbufs):
+            dg.copy_(hg, non_blocking=True)
+        call()
+        host_p16.copy_(p16, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K_e2e):
+        for hg, dg in zip(host_grads, z.gbufs):
+            dg.copy_(hg, non_blocking=True)
+        call()
+        host_p16.copy_(p16, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    times = torch.tensor([total_ms, per_launch_ms, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, per_launch_ms, e2e_ms = times.tolist()
+    ctrl = z.ctrl()
+
+    if rank == 0:
+        kind, size, R, gdt, pdt, scaled = WORKLOADS[args.workload]
+        P = z.P
+        bpp = bytes_per_param(R, gdt)
+        peaks = measured_peaks()
+        peak = peaks.get("hbm_gbs")
+        peak_src = "measured" if peak else "fallback"
+        peak = peak or 6650.0
+        ms_step = total_ms / K
+        achieved = bpp * P / (per_launch_ms * 1e-3) / 1e9
+        traffic = traffic_for(args.workload)
+        line = {
+            "metric": METRIC,
+            "value": world * P * K / (total_ms * 1e-3),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {
+                "workload": args.workload, "P": P, "R": R, "grad_dtype": gdt, "param_dtype": pdt,
+                "optimizer": "AdamW lr=1e-3 betas=(0.8,0.999) eps=1e-8 wd=3e-7",
+                "loss_scale_check": bool(scaled), "bytes_per_param": bpp,
+                "hbm_gbs_algorithmic": bpp * P / (ms_step * 1e-3) / 1e9,
+                "l2": f"inputs larger than L2 ({bpp * P / 1e6:.0f} MB touched per step vs 126 MB L2), no flush",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                "applied_steps": int(ctrl.step),
+            },
+            "roofline": {
+                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
+                "traffic": traffic,
+                "kernel": "step_kernel (flat)" if kind == "flat" else "step_kernel (list)",
+                "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms,
+            },
+            "e2e": {
+                "value": world * P * K_e2e / (e2e_ms * 1e-3), "unit": UNIT, "steps": K_e2e,
+                "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": p16.numel() * p16.element_size(),
+            } if K_e2e else None,
+            "gpu_launches": K * launches_per_step(z),
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _oracle_sample(workload: str, n: int):
+    """Host inputs for the oracle: the first n parameters of the workload."""
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    kind, size, R, gdt, pdt, scaled = WORKLOADS[workload]
+    wl = synth.WORKLOADS.get(workload.split("_")[0], 9)
+    S = 65536.0 if scaled else 1.0
+    tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt]
+    grads = []
+    for r in range(R):
+        g = synth.normal(n, 1e-3, synth.seed_for(wl, synth.KIND_GRAD, r, 1), dtype=tdt, scale=S)
+        grads.append(g.view(torch.int16).numpy().view(np.uint16) if gdt != "f32" else g.numpy())
+    w0 = synth.normal(n, 0.02, synth.seed_for(wl, synth.KIND_MASTER)).double().numpy()
+    st = oracle.State.create(w0, loss_scale=S)
+    return st, grads, gdt, scaled
+
+
+def cpu_baseline(workload: str, seconds: float) -> dict:
+    """The float64 oracle, as it stands, on this host's cores: steps over a
+    bounded sample of the workload until `seconds` have passed."""
+    import oracle
+    n = min(WORKLOADS[workload][1] if isinstance(WORKLOADS[workload][1], int) else 1 << 24, 1 << 24)
+    st, grads, gdt, scaled = _oracle_sample(workload, n)
+    hp = oracle.HP(*ADAMW)
+    steps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.step(st, grads, gdt, hp, check=scaled)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": n * steps / el, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"first {n} parameters of {workload}, {WORKLOADS[workload][2]} ranks, {steps} steps, "
+                      f"{el:.1f} s (float64 C loops, OpenMP)"}
+
+
+def run_reference(args) -> None:
+    """Reference arm: the float64 CPU oracle on the same workload, each step a
+    bounded sample of it; rank 0 alone runs it under torchrun."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+    n = 1 << 20
+    st, grads, gdt, scaled = _oracle_sample(args.workload, n)
+    hp = oracle.HP(*ADAMW)
+    for _ in range(args.warmup):
+        oracle.step(st, grads, gdt, hp, check=scaled)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.step(st, grads, gdt, hp, check=scaled)
+    el = time.perf_counter() - t0
+    value = n * args.steps / el
+    kind, size, R, g, p, sc = WORKLOADS[args.workload]
+    P = size if isinstance(size, int) else None
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "P": P, "R": R, "grad_dtype": g, "param_dtype": p,
+                   "optimizer": "AdamW lr=1e-3 betas=(0.8,0.999) eps=1e-8 wd=3e-7"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+                         "sample": f"first {n} parameters of {args.workload} per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="flat16m", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,285 @@
+/*
+ * zero_adam.h -- C ABI of the B200 (sm_100a) ZeRO-2/3 mixed-precision Adam
+ * step, run on one GPU with R logical data-parallel ranks held as R gradient
+ * buffers in that GPU's memory.
+ *
+ * The method (sources, cited by page title and section):
+ *   "Deep dive: DeepSpeed" lesson --
+ *     "Count state before choosing a stage": the 16-byte recipe (2-byte
+ *        weight, 2-byte gradient, fp32 master and both Adam moments) and the
+ *        per-rank state of each ZeRO stage;
+ *     "Reduce first, then update the owned slice": contiguous ownership
+ *        [floor(P*r/R), floor(P*(r+1)/R)), reduce the gradient across ranks
+ *        first, then apply Adam once per owned element to the reduced
+ *        gradient; the token-weighted mean for unequal token counts;
+ *     "Communication volume isn't elapsed time": ZeRO-2 is a gradient
+ *        reduce-scatter followed by an all-gather of the updated parameters.
+ *   DeepSpeed documentation page "ZeRO" (zero3.rst) -- stages 1-3 and the
+ *        AdamW optimizer configuration (lr, betas, eps, weight_decay) with
+ *        fp16 enabled.
+ *
+ * One fused pass per element does, for each owned index i:
+ *   g   = (sum_r c_r * grad_r[i]) / S       c_r = w_r / sum(w), S = loss scale
+ *   m   = b1*m + (1-b1)*g ;  v = b2*v + (1-b2)*g^2
+ *   w   = w - lr*( (m/(1-b1^t)) / (sqrt(v/(1-b2^t)) + eps) + wd*w )
+ *   p16 = round-to-nearest-even(w)          (written into the replicated
+ *                                             16-bit parameter buffer)
+ * with t the 1-based count of applied steps.  With the overflow check on, a
+ * step whose gradients hold any inf or NaN changes no weight or moment, keeps
+ * t, and halves S.
+ *
+ * Conventions for every entry point:
+ *   - Return 0 (ZERO_OK) or a negative ZERO_E* code; arguments are checked on
+ *     the host before anything is launched, and a rejected call launches
+ *     nothing.  No error is signalled from the device by trapping.
+ *   - Device-side calls are asynchronous on the given stream (a NULL stream is
+ *     the legacy default stream) unless stated otherwise.
+ *   - The caller owns and allocates every buffer; the library allocates no
+ *     device memory and keeps no state between calls apart from per-device
+ *     launch-shape caches.
+ *   - "device pointer" means memory of the current CUDA device; sizes are in
+ *     elements unless named *_bytes.
+ */
+#ifndef ZERO_ADAM_H
+#define ZERO_ADAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------ status codes */
+#define ZERO_OK 0
+#define ZERO_EINVAL (-1)    /* NULL pointer, unknown dtype, bad count or hyperparameter */
+#define ZERO_EALIGN (-2)    /* a device pointer is not 16-byte aligned */
+#define ZERO_EOVERFLOW (-3) /* a byte size does not fit in 64 bits */
+#define ZERO_ERANGE (-4)    /* a count beyond a documented limit */
+#define ZERO_ECUDA (-5)     /* a CUDA runtime call or launch failed (zero_last_cuda_error) */
+
+/* ------------------------------------------------------------------ dtypes */
+#define ZERO_F32 0  /* IEEE binary32 */
+#define ZERO_BF16 1 /* bfloat16 */
+#define ZERO_F16 2  /* IEEE binary16 */
+
+/* Largest number of logical ranks one step call accepts. */
+#define ZERO_MAX_RANKS 256
+
+/* Bytes of the scratch workspace every step call needs (see zero_step_args). */
+#define ZERO_WORKSPACE_BYTES 256
+
+/* Adam/AdamW hyperparameters ("ZeRO" documentation page, optimizer config:
+ * lr, betas, eps, weight_decay).  weight_decay = 0 is plain Adam, as in the
+ * scalar update of "Reduce first, then update the owned slice".
+ * Valid: lr >= 0, 0 <= beta1 < 1, 0 <= beta2 < 1, eps >= 0, weight_decay >= 0,
+ * all finite.  They are rounded to float32 for the per-element arithmetic;
+ * the bias corrections 1 - beta^t are formed in float64 on the device. */
+typedef struct zero_adam_hparams {
+    double lr;
+    double beta1;
+    double beta2;
+    double eps;
+    double weight_decay;
+} zero_adam_hparams;
+
+/* Control block: the persistent scalar state of one optimizer, in DEVICE
+ * memory (caller-allocated, zero_ctrl_bytes() bytes, 8-byte aligned).  Set it
+ * with zero_ctrl_init / zero_ctrl_set; step calls read and update it in
+ * stream order, so no host synchronisation is needed between steps.  Together
+ * with master, exp_avg and exp_avg_sq it is everything a resumed run needs
+ * ("Resume training and export weights separately"). */
+typedef struct zero_ctrl {
+    uint64_t step;            /* t: applied updates so far */
+    uint64_t skipped;         /* steps skipped because of inf/NaN gradients */
+    float loss_scale;         /* S: gradients are stored multiplied by S */
+    uint32_t growth_tracker;  /* applied steps since S last changed (check on) */
+    uint32_t parity;          /* two-set mode: index of the set holding the state */
+    uint32_t last_skipped;    /* 1 if the most recent step call skipped */
+    uint32_t reserved[2];     /* zero */
+} zero_ctrl;
+
+/* Arguments of one step over a FLAT parameter vector of P elements.
+ *
+ * Layout: every array is indexed by the flat parameter index i in [0, P);
+ * owner r's slice is [floor(P*r/R), floor(P*(r+1)/R)).  All device pointers
+ * must be 16-byte aligned (ZERO_EALIGN).
+ *
+ * State sets: master/exp_avg/exp_avg_sq[0] hold the fp32 master weights and
+ * moments.  If all three [1] pointers are NULL the step updates set 0 in
+ * place.  If all three are given ("two-set mode"), the step reads set
+ * ctrl.parity and writes set 1-ctrl.parity, and flips ctrl.parity only when
+ * the step is applied; with the overflow check on, this lets the whole step
+ * run as one pass over memory, because a skipped step leaves the old set
+ * untouched.  Mixing NULL and non-NULL [1] pointers is ZERO_EINVAL. */
+typedef struct zero_step_args {
+    uint64_t P;                   /* parameters (elements); 0 is allowed */
+    uint32_t R;                   /* logical ranks, 1..ZERO_MAX_RANKS */
+    int32_t owner;                /* -1: every owner's slice (all of [0,P)) in
+                                     this one call; 0..R-1: only that owner's
+                                     slice, with that owner's own ctrl */
+    int32_t grad_dtype;           /* ZERO_F32, ZERO_BF16 or ZERO_F16 */
+    int32_t param_dtype;          /* ZERO_BF16 or ZERO_F16 */
+    const void *const *grads;     /* HOST array of R device pointers, rank r's
+                                     gradient [P] of grad_dtype (flat call);
+                                     NULL for the list call */
+    const double *rank_weights;   /* HOST array of R weights w_r (token counts:
+                                     finite, >= 0, sum > 0), or NULL for the
+                                     equal-weight mean w_r = 1; used in
+                                     float64 as given */
+    float *master[2];             /* device [P] fp32 master weights */
+    float *exp_avg[2];            /* device [P] fp32 first moment m */
+    float *exp_avg_sq[2];         /* device [P] fp32 second moment v */
+    void *params16;               /* device [P] param_dtype: the replicated
+                                     16-bit parameters (flat call); NULL for
+                                     the list call */
+    float *reduced_out;           /* optional device [P] fp32: receives the
+                                     reduced, unscaled gradient g of every
+                                     updated element (the ZeRO-2 retained
+                                     gradient slice); NULL: not written */
+    zero_adam_hparams hp;
+    int32_t check_nonfinite;      /* 1: skip the step on any inf/NaN gradient */
+    uint32_t growth_interval;     /* check on: S doubles after this many
+                                     consecutive applied steps; 0: never */
+    void *ctrl;                   /* device zero_ctrl */
+    void *workspace;              /* device scratch of ZERO_WORKSPACE_BYTES,
+                                     16-byte aligned, all zero before its
+                                     first use (zero_workspace_init); every
+                                     call leaves it all zero again.  Calls
+                                     that may overlap on the GPU need separate
+                                     workspaces. */
+} zero_step_args;
+
+/* Device-resident description of a TENSOR LIST: T parameter tensors whose
+ * concatenation, in list order and without padding, is the flat vector the
+ * master weights and moments are laid out over.  Built once by
+ * zero_list_table_build (the per-step call then only passes this handle).
+ * All fields are filled by the build call; do not modify them. */
+typedef struct zero_tensor_list {
+    void *table;              /* caller-owned device memory holding the table */
+    uint64_t P;               /* sum of the tensors' element counts */
+    uint32_t T;               /* tensors */
+    uint32_t R;               /* ranks */
+    int32_t grad_dtype;
+    int32_t param_dtype;
+    uint64_t table_bytes;
+} zero_tensor_list;
+
+/* ---------------------------------------------------------------- host-only */
+
+/* Ownership bounds ("Reduce first, then update the owned slice"):
+ * lo[r] = floor(P*r/R), hi[r] = floor(P*(r+1)/R) for r in [0,R), computed
+ * exactly (128-bit intermediates).  Slices may be uneven, and empty when
+ * R > P.  lo, hi: caller HOST arrays of R entries.  ZERO_EINVAL for R == 0 or
+ * NULL arrays.  Pure host function; needs no GPU. */
+int zero_partition_bounds(uint64_t P, uint32_t R, uint64_t *lo, uint64_t *hi);
+
+/* Per-rank persistent state bytes ("Count state before choosing a stage"):
+ * with param_b, grad_b, opt_b the bytes per parameter of the 16-bit weight,
+ * the gradient and the optimizer state (master + moments), and S = P/R,
+ *   DP     = P*(param_b + grad_b + opt_b)
+ *   ZeRO-1 = P*(param_b + grad_b) + S*opt_b
+ *   ZeRO-2 = P*param_b + S*(grad_b + opt_b)
+ *   ZeRO-3 = S*(param_b + grad_b + opt_b).
+ * The values can be fractional, so out_times_R[k] receives R times the bytes
+ * of stage k (k = 0: DP, 1..3: ZeRO-1..3), exactly.  ZERO_EINVAL if any count
+ * or width is 0 or out is NULL, ZERO_EOVERFLOW if a product exceeds 64 bits.
+ * Pure host function. */
+int zero_state_bytes(uint64_t P, uint32_t R, uint32_t param_b, uint32_t grad_b,
+                     uint32_t opt_b, uint64_t out_times_R[4]);
+
+/* Human-readable text of a status code (static storage). */
+const char *zero_status_string(int status);
+
+/* Text of the last CUDA error this thread saw inside the library
+ * ("no error" if none); static storage, valid until the next call. */
+const char *zero_last_cuda_error(void);
+
+/* Sizes of the caller-allocated device blocks. */
+size_t zero_ctrl_bytes(void);      /* sizeof(zero_ctrl) */
+size_t zero_workspace_bytes(void); /* ZERO_WORKSPACE_BYTES */
+
+/* Bytes of device memory a tensor-list table for T tensors and R ranks needs. */
+size_t zero_list_table_bytes(uint32_t T, uint32_t R);
+
+/* ---------------------------------------------------------- control block */
+
+/* ctrl = {step 0, skipped 0, loss_scale, growth 0, parity 0, last_skipped 0}.
+ * loss_scale must be finite and > 0 (1 when no loss scaling is used). */
+int zero_ctrl_init(void *ctrl, float loss_scale, void *stream);
+
+/* ctrl = *value (e.g. restoring a checkpoint); value is a HOST struct passed
+ * by value to the device, so it may be freed as soon as the call returns. */
+int zero_ctrl_set(void *ctrl, const zero_ctrl *value, void *stream);
+
+/* Copy the device ctrl into *out (HOST) and wait for it: synchronises the
+ * stream. */
+int zero_ctrl_read(const void *ctrl, zero_ctrl *out, void *stream);
+
+/* Zero a workspace of ZERO_WORKSPACE_BYTES (cudaMemsetAsync). */
+int zero_workspace_init(void *workspace, void *stream);
+
+/* ------------------------------------------------------------- the step */
+
+/* One fused ZeRO-2/3 optimizer step over a flat parameter vector:
+ * in-HBM reduce-scatter of the R rank gradients into the owner slices, the
+ * optional loss-scale undo and inf/NaN skip, Adam/AdamW with bias correction
+ * on the fp32 masters and moments, and the round-to-nearest-even cast of the
+ * updated masters written into the replicated 16-bit parameters (the
+ * updated-parameter all-gather).  The reduction runs over ranks 0..R-1 in
+ * that order as float64 fused multiply-adds of w_r times the gradient (both
+ * exact in float64), is scaled by 1/(sum(w)*S) and rounded once to float32;
+ * results are bitwise reproducible run to run.  Sources: "Reduce first, then update the owned
+ * slice" and "Communication volume isn't elapsed time" ("Deep dive:
+ * DeepSpeed"); the AdamW/fp16 configuration of the "ZeRO" documentation page.
+ *
+ * Launches: one kernel, except (a) check on, in place, or check on with
+ * owner >= 0: a scan kernel over all R gradients first (the skip decision
+ * covers every rank's whole gradient, as a flag combined across ranks would);
+ * (b) check on in two-set mode with owner == -1: one pass plus a restore
+ * kernel that, only if the step was skipped, re-casts the 16-bit parameters
+ * from the untouched master set.
+ * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ERANGE (R > ZERO_MAX_RANKS),
+ * ZERO_EOVERFLOW (P*4 bytes overflow), ZERO_ECUDA. */
+int zero_step_fused(const zero_step_args *args, void *stream);
+
+/* The same step over a tensor list: args->grads and args->params16 must be
+ * NULL (the list supplies them), args->P / R / grad_dtype / param_dtype must
+ * equal the list's.  master/exp_avg/exp_avg_sq are flat [P] over the list's
+ * concatenation.  Tensors whose flat start is not a multiple of 8, or whose
+ * buffers are not 16-byte aligned, take a scalar path (correct, slower). */
+int zero_step_fused_list(const zero_step_args *args, const zero_tensor_list *list,
+                         void *stream);
+
+/* Build a tensor-list table in caller-owned device memory `table`
+ * (>= zero_list_table_bytes(T, R) bytes, 16-byte aligned) and fill *out.
+ *   numel:    HOST array of T element counts (0 allowed)
+ *   params16: HOST array of T device pointers (param_dtype; NULL if numel 0)
+ *   grads:    HOST array of R*T device pointers, RANK-MAJOR: grads[r*T + j]
+ *             is rank r's gradient of tensor j (grad_dtype; NULL if numel 0)
+ * SYNCHRONOUS: copies the table to the device and waits for the stream.
+ * Rebuild it whenever a buffer moves. */
+int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t *numel,
+                          void *const *params16, const void *const *grads,
+                          int32_t grad_dtype, int32_t param_dtype, void *table,
+                          size_t table_bytes, zero_tensor_list *out, void *stream);
+
+/* --------------------------------------------------------------- gathers */
+
+/* params16[i] = round-to-nearest-even(master[i]) for i in [0,P): the cast of
+ * the fp32 masters into the replicated 16-bit buffer on its own (the
+ * updated-parameter all-gather of "Communication volume isn't elapsed time",
+ * on one GPU).  Also used to initialise params16 from fresh masters.
+ * master, params16: device, 16-byte aligned. */
+int zero_gather_params(const float *master, void *params16, int32_t param_dtype,
+                       uint64_t P, void *stream);
+
+/* The same over a tensor list's parameter tensors. */
+int zero_gather_params_list(const float *master, const zero_tensor_list *list,
+                            void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZERO_ADAM_H */

@@ -1,0 +1,261 @@
+"""Python binding of libzero_adam.so, the B200 (sm_100a) fused ZeRO-2/3
+mixed-precision Adam step.
+
+Argument marshalling only: every function forwards to the C entry point of
+the same name (declared in include/zero_adam.h) and raises ZeroError on a
+non-zero status.  All arithmetic of the step runs in the library's CUDA
+kernels; there is no fallback of any kind, and importing this package fails
+loudly when the library has not been built.
+
+Pointers are accepted as ints or as objects with ``data_ptr()`` (torch
+tensors).  Streams are accepted as ints (``cudaStream_t`` values), as objects
+with ``cuda_stream`` (torch streams), or None for the legacy default stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzero_adam.so")
+
+ZERO_OK = 0
+ZERO_EINVAL = -1
+ZERO_EALIGN = -2
+ZERO_EOVERFLOW = -3
+ZERO_ERANGE = -4
+ZERO_ECUDA = -5
+
+ZERO_F32 = 0
+ZERO_BF16 = 1
+ZERO_F16 = 2
+
+ZERO_MAX_RANKS = 256
+ZERO_WORKSPACE_BYTES = 256
+
+EXPORTED = [
+    "zero_partition_bounds", "zero_state_bytes", "zero_status_string", "zero_last_cuda_error",
+    "zero_ctrl_bytes", "zero_workspace_bytes", "zero_list_table_bytes", "zero_ctrl_init",
+    "zero_ctrl_set", "zero_ctrl_read", "zero_workspace_init", "zero_step_fused",
+    "zero_step_fused_list", "zero_list_table_build", "zero_gather_params",
+    "zero_gather_params_list",
+]
+
+
+class ZeroError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        text = _lib().zero_status_string(status).decode()
+        if status == ZERO_ECUDA:
+            text += ": " + _lib().zero_last_cuda_error().decode()
+        super().__init__(f"{where}: status {status} ({text})")
+        self.status = status
+
+
+class zero_adam_hparams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
+                ("eps", ctypes.c_double), ("weight_decay", ctypes.c_double)]
+
+
+class zero_ctrl(ctypes.Structure):
+    _fields_ = [("step", ctypes.c_uint64), ("skipped", ctypes.c_uint64),
+                ("loss_scale", ctypes.c_float), ("growth_tracker", ctypes.c_uint32),
+                ("parity", ctypes.c_uint32), ("last_skipped", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32 * 2)]
+
+
+class zero_step_args(ctypes.Structure):
+    _fields_ = [("P", ctypes.c_uint64), ("R", ctypes.c_uint32), ("owner", ctypes.c_int32),
+                ("grad_dtype", ctypes.c_int32), ("param_dtype", ctypes.c_int32),
+                ("grads", ctypes.POINTER(ctypes.c_void_p)),
+                ("rank_weights", ctypes.POINTER(ctypes.c_double)),
+                ("master", ctypes.c_void_p * 2), ("exp_avg", ctypes.c_void_p * 2),
+                ("exp_avg_sq", ctypes.c_void_p * 2), ("params16", ctypes.c_void_p),
+                ("reduced_out", ctypes.c_void_p), ("hp", zero_adam_hparams),
+                ("check_nonfinite", ctypes.c_int32), ("growth_interval", ctypes.c_uint32),
+                ("ctrl", ctypes.c_void_p), ("workspace", ctypes.c_void_p)]
+
+
+class zero_tensor_list(ctypes.Structure):
+    _fields_ = [("table", ctypes.c_void_p), ("P", ctypes.c_uint64), ("T", ctypes.c_uint32),
+                ("R", ctypes.c_uint32), ("grad_dtype", ctypes.c_int32),
+                ("param_dtype", ctypes.c_int32), ("table_bytes", ctypes.c_uint64)]
+
+
+_handle = None
+
+
+def _lib() -> ctypes.CDLL:
+    global _handle
+    if _handle is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: the CUDA library has not been built "
+                "(run `python -c 'import __graft_entry__ as g; g.build()'` at the repository root)")
+        L = ctypes.CDLL(LIB_PATH)
+        u64, u32, i32, vp, sz = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+        u64p = ctypes.POINTER(ctypes.c_uint64)
+        L.zero_partition_bounds.argtypes = [u64, u32, u64p, u64p]
+        L.zero_state_bytes.argtypes = [u64, u32, u32, u32, u32, u64p]
+        L.zero_status_string.argtypes = [ctypes.c_int]
+        L.zero_status_string.restype = ctypes.c_char_p
+        L.zero_last_cuda_error.restype = ctypes.c_char_p
+        L.zero_ctrl_bytes.restype = sz
+        L.zero_workspace_bytes.restype = sz
+        L.zero_list_table_bytes.argtypes = [u32, u32]
+        L.zero_list_table_bytes.restype = sz
+        L.zero_ctrl_init.argtypes = [vp, ctypes.c_float, vp]
+        L.zero_ctrl_set.argtypes = [vp, ctypes.POINTER(zero_ctrl), vp]
+        L.zero_ctrl_read.argtypes = [vp, ctypes.POINTER(zero_ctrl), vp]
+        L.zero_workspace_init.argtypes = [vp, vp]
+        L.zero_step_fused.argtypes = [ctypes.POINTER(zero_step_args), vp]
+        L.zero_step_fused_list.argtypes = [ctypes.POINTER(zero_step_args), ctypes.POINTER(zero_tensor_list), vp]
+        L.zero_list_table_build.argtypes = [u32, u32, u64p, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32,
+                                            vp, sz, ctypes.POINTER(zero_tensor_list), vp]
+        L.zero_gather_params.argtypes = [vp, vp, i32, u64, vp]
+        L.zero_gather_params_list.argtypes = [vp, ctypes.POINTER(zero_tensor_list), vp]
+        _handle = L
+    return _handle
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if hasattr(x, "data_ptr"):
+        return int(x.data_ptr())
+    return int(x)
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        return None
+    if hasattr(s, "cuda_stream"):
+        return int(s.cuda_stream)
+    return int(s)
+
+
+def _check(status: int, where: str) -> None:
+    if status != ZERO_OK:
+        raise ZeroError(status, where)
+
+
+# ------------------------------------------------------------ host-only calls
+
+def zero_partition_bounds(P: int, R: int) -> Tuple[List[int], List[int]]:
+    lo = (ctypes.c_uint64 * max(R, 1))()
+    hi = (ctypes.c_uint64 * max(R, 1))()
+    _check(_lib().zero_partition_bounds(P, R, lo, hi), "zero_partition_bounds")
+    return list(lo)[:R], list(hi)[:R]
+
+
+def zero_state_bytes(P: int, R: int, param_b: int = 2, grad_b: int = 2, opt_b: int = 12) -> List[int]:
+    """R times the per-rank bytes of DP, ZeRO-1, ZeRO-2, ZeRO-3 (exact ints)."""
+    out = (ctypes.c_uint64 * 4)()
+    _check(_lib().zero_state_bytes(P, R, param_b, grad_b, opt_b, out), "zero_state_bytes")
+    return list(out)
+
+
+def zero_status_string(status: int) -> str:
+    return _lib().zero_status_string(status).decode()
+
+
+def zero_last_cuda_error() -> str:
+    return _lib().zero_last_cuda_error().decode()
+
+
+def zero_ctrl_bytes() -> int:
+    return int(_lib().zero_ctrl_bytes())
+
+
+def zero_workspace_bytes() -> int:
+    return int(_lib().zero_workspace_bytes())
+
+
+def zero_list_table_bytes(T: int, R: int) -> int:
+    return int(_lib().zero_list_table_bytes(T, R))
+
+
+# ------------------------------------------------------------ device calls
+
+def zero_ctrl_init(ctrl, loss_scale: float = 1.0, stream=None) -> None:
+    _check(_lib().zero_ctrl_init(_ptr(ctrl), loss_scale, _stream(stream)), "zero_ctrl_init")
+
+
+def zero_ctrl_set(ctrl, value: zero_ctrl, stream=None) -> None:
+    _check(_lib().zero_ctrl_set(_ptr(ctrl), ctypes.byref(value), _stream(stream)), "zero_ctrl_set")
+
+
+def zero_ctrl_read(ctrl, stream=None) -> zero_ctrl:
+    out = zero_ctrl()
+    _check(_lib().zero_ctrl_read(_ptr(ctrl), ctypes.byref(out), _stream(stream)), "zero_ctrl_read")
+    return out
+
+
+def zero_workspace_init(workspace, stream=None) -> None:
+    _check(_lib().zero_workspace_init(_ptr(workspace), _stream(stream)), "zero_workspace_init")
+
+
+def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master, exp_avg, exp_avg_sq,
+                   ctrl, workspace, grads: Optional[Sequence] = None, params16=None,
+                   rank_weights: Optional[Sequence[float]] = None, owner: int = -1,
+                   hp: Tuple[float, float, float, float, float] = (1e-3, 0.9, 0.999, 1e-8, 0.0),
+                   check_nonfinite: bool = False, growth_interval: int = 0, reduced_out=None,
+                   master2=None, exp_avg2=None, exp_avg_sq2=None) -> zero_step_args:
+    """Fill a zero_step_args (the returned struct keeps its host arrays alive)."""
+    a = zero_step_args()
+    a.P, a.R, a.owner = P, R, owner
+    a.grad_dtype, a.param_dtype = grad_dtype, param_dtype
+    if grads is not None:
+        arr = (ctypes.c_void_p * len(grads))(*[_ptr(g) for g in grads])
+        a._grads_keep = arr
+        a.grads = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    if rank_weights is not None:
+        w = (ctypes.c_double * len(rank_weights))(*[float(x) for x in rank_weights])
+        a._weights_keep = w
+        a.rank_weights = ctypes.cast(w, ctypes.POINTER(ctypes.c_double))
+    a.master[0], a.exp_avg[0], a.exp_avg_sq[0] = _ptr(master), _ptr(exp_avg), _ptr(exp_avg_sq)
+    a.master[1], a.exp_avg[1], a.exp_avg_sq[1] = _ptr(master2), _ptr(exp_avg2), _ptr(exp_avg_sq2)
+    a.params16 = _ptr(params16)
+    a.reduced_out = _ptr(reduced_out)
+    a.hp = zero_adam_hparams(*[float(x) for x in hp])
+    a.check_nonfinite = int(bool(check_nonfinite))
+    a.growth_interval = growth_interval
+    a.ctrl, a.workspace = _ptr(ctrl), _ptr(workspace)
+    return a
+
+
+def zero_step_fused(args: zero_step_args, stream=None) -> None:
+    _check(_lib().zero_step_fused(ctypes.byref(args), _stream(stream)), "zero_step_fused")
+
+
+def zero_step_fused_list(args: zero_step_args, lst: zero_tensor_list, stream=None) -> None:
+    _check(_lib().zero_step_fused_list(ctypes.byref(args), ctypes.byref(lst), _stream(stream)),
+           "zero_step_fused_list")
+
+
+def zero_list_table_build(numel: Sequence[int], params16: Sequence, grads: Sequence[Sequence],
+                          grad_dtype: int, param_dtype: int, table, table_bytes: int,
+                          stream=None) -> zero_tensor_list:
+    """grads[r][j]: rank r's gradient of tensor j (rank-major, as the C call)."""
+    T, R = len(numel), len(grads)
+    n = (ctypes.c_uint64 * T)(*numel)
+    p = (ctypes.c_void_p * T)(*[_ptr(x) for x in params16])
+    g = (ctypes.c_void_p * (R * T))(*[_ptr(grads[r][j]) for r in range(R) for j in range(T)])
+    out = zero_tensor_list()
+    _check(_lib().zero_list_table_build(T, R, n, p, g, grad_dtype, param_dtype, _ptr(table), table_bytes,
+                                        ctypes.byref(out), _stream(stream)), "zero_list_table_build")
+    return out
+
+
+def zero_gather_params(master, params16, param_dtype: int, P: int, stream=None) -> None:
+    _check(_lib().zero_gather_params(_ptr(master), _ptr(params16), param_dtype, P, _stream(stream)),
+           "zero_gather_params")
+
+
+def zero_gather_params_list(master, lst: zero_tensor_list, stream=None) -> None:
+    _check(_lib().zero_gather_params_list(_ptr(master), ctypes.byref(lst), _stream(stream)),
+           "zero_gather_params_list")

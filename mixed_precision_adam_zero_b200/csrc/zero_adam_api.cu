@@ -1,0 +1,472 @@
+// zero_adam_api.cu -- the exported C ABI around the sm_100a kernels:
+// argument checks, launch shapes and kernel selection.  Declarations and
+// the contract of every entry point: include/zero_adam.h.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "zero_adam.h"
+#include "zero_adam_kernels.cuh"
+
+using namespace zadam;
+
+namespace {
+
+thread_local char g_cuda_error[256] = "no error";
+
+// Remember the text of a failed CUDA call for zero_last_cuda_error().
+int zadam_record_cuda(cudaError_t e) {
+    std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return ZERO_ECUDA;
+}
+
+// ------------------------------------------------------------ launch shapes
+
+struct OccEntry {
+    const void* fn;
+    int device;
+    int ctas;  // max CTAs resident on the whole device
+};
+
+std::mutex g_occ_mu;
+std::vector<OccEntry> g_occ;
+
+// Resident CTAs of `fn` on the current device (SMs x CTAs per SM), cached.
+int resident_ctas(const void* fn, int* err) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) { *err = zadam_record_cuda(e); return 0; }
+    {
+        std::lock_guard<std::mutex> lk(g_occ_mu);
+        for (const OccEntry& o : g_occ)
+            if (o.fn == fn && o.device == dev) return o.ctas;
+    }
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
+    if (e != cudaSuccess) { *err = zadam_record_cuda(e); return 0; }
+    if (per_sm < 1) per_sm = 1;
+    const int ctas = sms * per_sm;
+    std::lock_guard<std::mutex> lk(g_occ_mu);
+    g_occ.push_back({fn, dev, ctas});
+    return ctas;
+}
+
+struct Shape {
+    uint64_t base, chunk;
+    unsigned grid;
+};
+
+// Split [lo, hi) into at most max_ctas contiguous CTA ranges whose inner
+// boundaries are multiples of 8 (absolute index), each at least one vector
+// per thread long.
+Shape make_shape(uint64_t lo, uint64_t hi, int max_ctas) {
+    Shape s;
+    s.base = lo & ~7ull;
+    if (hi <= lo) { s.chunk = kVec; s.grid = 1; return s; }
+    const uint64_t n = hi - s.base;
+    const uint64_t min_chunk = (uint64_t)kThreads * kVec;
+    uint64_t g = (n + min_chunk - 1) / min_chunk;
+    if (g > (uint64_t)max_ctas) g = (uint64_t)max_ctas;
+    if (g < 1) g = 1;
+    uint64_t ch = (n + g - 1) / g;
+    ch = (ch + kVec - 1) & ~(uint64_t)(kVec - 1);
+    s.chunk = ch;
+    s.grid = (unsigned)((n + ch - 1) / ch);
+    return s;
+}
+
+int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st) {
+    void* args[] = {params};
+    const cudaError_t e = cudaLaunchKernel(fn, dim3(sh.grid), dim3(kThreads), args, 0, st);
+    if (e != cudaSuccess) return zadam_record_cuda(e);
+    return ZERO_OK;
+}
+
+// ------------------------------------------------------------ kernel tables
+
+template <class G, class Pm, bool LIST>
+const void* step_fn_rc(uint32_t R) {
+    switch (R) {
+        case 1: return (const void*)step_kernel<G, Pm, 1, LIST>;
+        case 2: return (const void*)step_kernel<G, Pm, 2, LIST>;
+        case 4: return (const void*)step_kernel<G, Pm, 4, LIST>;
+        case 8: return (const void*)step_kernel<G, Pm, 8, LIST>;
+        default: return (const void*)step_kernel<G, Pm, 0, LIST>;
+    }
+}
+
+template <class G, bool LIST>
+const void* step_fn_pm(int32_t param_dtype, uint32_t R) {
+    return param_dtype == ZERO_BF16 ? step_fn_rc<G, __nv_bfloat16, LIST>(R) : step_fn_rc<G, __half, LIST>(R);
+}
+
+template <bool LIST>
+const void* step_fn(int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
+    switch (grad_dtype) {
+        case ZERO_F32: return step_fn_pm<float, LIST>(param_dtype, R);
+        case ZERO_BF16: return step_fn_pm<__nv_bfloat16, LIST>(param_dtype, R);
+        default: return step_fn_pm<__half, LIST>(param_dtype, R);
+    }
+}
+
+template <bool LIST>
+const void* scan_fn(int32_t grad_dtype) {
+    switch (grad_dtype) {
+        case ZERO_F32: return (const void*)scan_kernel<float, LIST>;
+        case ZERO_BF16: return (const void*)scan_kernel<__nv_bfloat16, LIST>;
+        default: return (const void*)scan_kernel<__half, LIST>;
+    }
+}
+
+template <bool LIST>
+const void* gather_fn(int32_t param_dtype) {
+    return param_dtype == ZERO_BF16 ? (const void*)gather_kernel<__nv_bfloat16, LIST>
+                                    : (const void*)gather_kernel<__half, LIST>;
+}
+
+// ------------------------------------------------------------ argument checks
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool finite_nonneg(double x) { return std::isfinite(x) && x >= 0.0; }
+
+int check_hparams(const zero_adam_hparams& h) {
+    if (!finite_nonneg(h.lr) || !finite_nonneg(h.eps) || !finite_nonneg(h.weight_decay)) return ZERO_EINVAL;
+    if (!(h.beta1 >= 0.0 && h.beta1 < 1.0) || !(h.beta2 >= 0.0 && h.beta2 < 1.0)) return ZERO_EINVAL;
+    return ZERO_OK;
+}
+
+bool is_grad_dtype(int32_t d) { return d == ZERO_F32 || d == ZERO_BF16 || d == ZERO_F16; }
+bool is_param_dtype(int32_t d) { return d == ZERO_BF16 || d == ZERO_F16; }
+
+// Checks shared by the flat and the list step; fills the rank weights, the
+// hyperparameters and the state pointers of `kp`.
+int check_common(const zero_step_args* a, StepParams* kp) {
+    if (a == nullptr) return ZERO_EINVAL;
+    if (a->R == 0) return ZERO_EINVAL;
+    if (a->R > ZERO_MAX_RANKS) return ZERO_ERANGE;
+    if (a->owner < -1 || a->owner >= (int64_t)a->R) return ZERO_EINVAL;
+    if (!is_grad_dtype(a->grad_dtype) || !is_param_dtype(a->param_dtype)) return ZERO_EINVAL;
+    if (a->check_nonfinite != 0 && a->check_nonfinite != 1) return ZERO_EINVAL;
+    if (a->P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
+    int rc = check_hparams(a->hp);
+    if (rc) return rc;
+    if (a->ctrl == nullptr || a->workspace == nullptr) return ZERO_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(a->ctrl) & 7u) != 0 || !aligned16(a->workspace)) return ZERO_EALIGN;
+    const bool two = a->master[1] != nullptr || a->exp_avg[1] != nullptr || a->exp_avg_sq[1] != nullptr;
+    if (two && (a->master[1] == nullptr || a->exp_avg[1] == nullptr || a->exp_avg_sq[1] == nullptr))
+        return ZERO_EINVAL;
+    const int sets = two ? 2 : 1;
+    for (int k = 0; k < sets; ++k) {
+        if (a->P > 0 && (a->master[k] == nullptr || a->exp_avg[k] == nullptr || a->exp_avg_sq[k] == nullptr))
+            return ZERO_EINVAL;
+        if (!aligned16(a->master[k]) || !aligned16(a->exp_avg[k]) || !aligned16(a->exp_avg_sq[k])) return ZERO_EALIGN;
+    }
+    if (!aligned16(a->reduced_out)) return ZERO_EALIGN;
+
+    // Rank weights as given (float64) and their sum, in rank order.
+    double wsum = 0.0;
+    for (uint32_t r = 0; r < a->R; ++r) {
+        const double wr = a->rank_weights ? a->rank_weights[r] : 1.0;
+        if (!finite_nonneg(wr)) return ZERO_EINVAL;
+        wsum += wr;
+    }
+    if (!(wsum > 0.0) || !std::isfinite(wsum)) return ZERO_EINVAL;
+    std::memset(kp, 0, sizeof(*kp));
+    for (uint32_t r = 0; r < a->R; ++r) kp->wt[r] = a->rank_weights ? a->rank_weights[r] : 1.0;
+    kp->wsum = wsum;
+
+    for (int k = 0; k < 2; ++k) {
+        const int src = two ? k : 0;
+        kp->w[k] = a->master[src];
+        kp->m[k] = a->exp_avg[src];
+        kp->v[k] = a->exp_avg_sq[src];
+    }
+    kp->reduced = a->reduced_out;
+    const zero_adam_hparams& h = a->hp;
+    kp->h.b1 = (float)h.beta1;
+    kp->h.b2 = (float)h.beta2;
+    kp->h.omb1 = (float)(1.0 - h.beta1);
+    kp->h.omb2 = (float)(1.0 - h.beta2);
+    kp->h.eps = (float)h.eps;
+    kp->h.lr_wd = (float)(h.lr * h.weight_decay);
+    kp->h.lr = h.lr;
+    kp->h.b1d = h.beta1;
+    kp->h.b2d = h.beta2;
+    kp->ctrl = static_cast<zero_ctrl*>(a->ctrl);
+    kp->ws = static_cast<Workspace*>(a->workspace);
+    kp->R = a->R;
+    kp->growth_interval = a->growth_interval;
+    kp->two_set = two ? 1 : 0;
+    return ZERO_OK;
+}
+
+// Range of the launch: every slice, or one owner's.
+void owner_range(const zero_step_args* a, uint64_t* lo, uint64_t* hi) {
+    if (a->owner < 0) { *lo = 0; *hi = a->P; return; }
+    const unsigned __int128 P = a->P;
+    *lo = (uint64_t)((P * (uint32_t)a->owner) / a->R);
+    *hi = (uint64_t)((P * ((uint32_t)a->owner + 1u)) / a->R);
+}
+
+// The launch sequence shared by the flat and list calls.
+template <bool LIST>
+int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
+    uint64_t lo, hi;
+    owner_range(a, &lo, &hi);
+    kp->lo = lo;
+    kp->hi = hi;
+    int err = ZERO_OK;
+    const bool check = a->check_nonfinite != 0;
+    const bool single_pass = check && kp->two_set && a->owner < 0;
+    if (check && !single_pass) {
+        // Scan every rank's whole gradient first; the step then reads the flag.
+        StepParams sp = *kp;
+        const void* sfn = scan_fn<LIST>(a->grad_dtype);
+        const int ctas = resident_ctas(sfn, &err);
+        if (err) return err;
+        const Shape sh = make_shape(0, a->P, ctas);
+        sp.lo = 0;
+        sp.hi = a->P;
+        sp.base = sh.base;
+        sp.chunk = sh.chunk;
+        if ((err = launch(sfn, sh, &sp, st))) return err;
+        kp->check = 2;
+    } else {
+        kp->check = check ? 1 : 0;
+    }
+    const void* fn = step_fn<LIST>(a->grad_dtype, a->param_dtype, a->R);
+    const int ctas = resident_ctas(fn, &err);
+    if (err) return err;
+    const Shape sh = make_shape(lo, hi, ctas);
+    kp->base = sh.base;
+    kp->chunk = sh.chunk;
+    if ((err = launch(fn, sh, kp, st))) return err;
+    if (single_pass) {
+        // Only if the step was skipped: re-cast the 16-bit parameters from
+        // the master set that stayed current.
+        GatherParams gp;
+        std::memset(&gp, 0, sizeof gp);
+        gp.w[0] = kp->w[0];
+        gp.w[1] = kp->w[1];
+        gp.params16 = kp->params16;
+        gp.tab = kp->tab;
+        gp.lo = lo;
+        gp.hi = hi;
+        gp.ctrl = kp->ctrl;
+        gp.only_if_skipped = 1;
+        const void* gfn = gather_fn<LIST>(a->param_dtype);
+        const int gctas = resident_ctas(gfn, &err);
+        if (err) return err;
+        const Shape gsh = make_shape(lo, hi, gctas);
+        gp.base = gsh.base;
+        gp.chunk = gsh.chunk;
+        if ((err = launch(gfn, gsh, &gp, st))) return err;
+    }
+    return ZERO_OK;
+}
+
+// Host copy of a list's table layout: byte offsets of each array.
+struct TableLayout {
+    size_t offs, params, grads, flags, total;
+};
+
+TableLayout table_layout(uint32_t T, uint32_t R) {
+    TableLayout L;
+    L.offs = 0;
+    L.params = L.offs + 8ull * ((size_t)T + 1);
+    L.grads = L.params + 8ull * T;
+    L.flags = L.grads + 8ull * (size_t)T * R;
+    L.total = L.flags + ((4ull * T + 15) & ~15ull);
+    return L;
+}
+
+Table device_table(const zero_tensor_list* l) {
+    const TableLayout L = table_layout(l->T, l->R);
+    const char* base = static_cast<const char*>(l->table);
+    Table t;
+    t.offs = reinterpret_cast<const uint64_t*>(base + L.offs);
+    t.params = reinterpret_cast<void* const*>(base + L.params);
+    t.grads = reinterpret_cast<const void* const*>(base + L.grads);
+    t.flags = reinterpret_cast<const uint32_t*>(base + L.flags);
+    t.T = l->T;
+    return t;
+}
+
+int check_list(const zero_tensor_list* l) {
+    if (l == nullptr || l->table == nullptr || l->T == 0 || l->R == 0) return ZERO_EINVAL;
+    if (l->R > ZERO_MAX_RANKS) return ZERO_ERANGE;
+    if (!aligned16(l->table)) return ZERO_EALIGN;
+    if (l->table_bytes < table_layout(l->T, l->R).total) return ZERO_EINVAL;
+    if (!is_grad_dtype(l->grad_dtype) || !is_param_dtype(l->param_dtype)) return ZERO_EINVAL;
+    return ZERO_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+
+extern "C" {
+
+const char* zero_last_cuda_error(void) { return g_cuda_error; }
+
+size_t zero_ctrl_bytes(void) { return sizeof(zero_ctrl); }
+size_t zero_workspace_bytes(void) { return ZERO_WORKSPACE_BYTES; }
+
+size_t zero_list_table_bytes(uint32_t T, uint32_t R) { return table_layout(T, R).total; }
+
+int zero_ctrl_init(void* ctrl, float loss_scale, void* stream) {
+    if (!(std::isfinite(loss_scale) && loss_scale > 0.0f)) return ZERO_EINVAL;
+    zero_ctrl v;
+    std::memset(&v, 0, sizeof v);
+    v.loss_scale = loss_scale;
+    return zero_ctrl_set(ctrl, &v, stream);
+}
+
+int zero_ctrl_set(void* ctrl, const zero_ctrl* value, void* stream) {
+    if (ctrl == nullptr || value == nullptr) return ZERO_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(ctrl) & 7u) != 0) return ZERO_EALIGN;
+    if (!(std::isfinite(value->loss_scale) && value->loss_scale > 0.0f) || value->parity > 1u) return ZERO_EINVAL;
+    ctrl_set_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<zero_ctrl*>(ctrl), *value);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ZERO_OK : zadam_record_cuda(e);
+}
+
+int zero_ctrl_read(const void* ctrl, zero_ctrl* out, void* stream) {
+    if (ctrl == nullptr || out == nullptr) return ZERO_EINVAL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(out, ctrl, sizeof(zero_ctrl), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return e == cudaSuccess ? ZERO_OK : zadam_record_cuda(e);
+}
+
+int zero_workspace_init(void* workspace, void* stream) {
+    if (workspace == nullptr) return ZERO_EINVAL;
+    if (!aligned16(workspace)) return ZERO_EALIGN;
+    const cudaError_t e = cudaMemsetAsync(workspace, 0, ZERO_WORKSPACE_BYTES, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ZERO_OK : zadam_record_cuda(e);
+}
+
+int zero_step_fused(const zero_step_args* a, void* stream) {
+    StepParams kp;
+    int rc = check_common(a, &kp);
+    if (rc) return rc;
+    if (a->grads == nullptr) return ZERO_EINVAL;
+    if (a->P > 0 && a->params16 == nullptr) return ZERO_EINVAL;
+    if (!aligned16(a->params16)) return ZERO_EALIGN;
+    for (uint32_t r = 0; r < a->R; ++r) {
+        if (a->P > 0 && a->grads[r] == nullptr) return ZERO_EINVAL;
+        if (!aligned16(a->grads[r])) return ZERO_EALIGN;
+        kp.grads[r] = a->grads[r];
+    }
+    kp.params16 = a->params16;
+    return run_step<false>(a, &kp, static_cast<cudaStream_t>(stream));
+}
+
+int zero_step_fused_list(const zero_step_args* a, const zero_tensor_list* l, void* stream) {
+    StepParams kp;
+    int rc = check_common(a, &kp);
+    if (rc) return rc;
+    if ((rc = check_list(l))) return rc;
+    if (a->grads != nullptr || a->params16 != nullptr) return ZERO_EINVAL;
+    if (a->P != l->P || a->R != l->R || a->grad_dtype != l->grad_dtype || a->param_dtype != l->param_dtype)
+        return ZERO_EINVAL;
+    kp.tab = device_table(l);
+    return run_step<true>(a, &kp, static_cast<cudaStream_t>(stream));
+}
+
+int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t* numel, void* const* params16,
+                          const void* const* grads, int32_t grad_dtype, int32_t param_dtype, void* table,
+                          size_t table_bytes, zero_tensor_list* out, void* stream) {
+    if (T == 0 || R == 0 || numel == nullptr || params16 == nullptr || grads == nullptr || table == nullptr ||
+        out == nullptr)
+        return ZERO_EINVAL;
+    if (R > ZERO_MAX_RANKS) return ZERO_ERANGE;
+    if (!is_grad_dtype(grad_dtype) || !is_param_dtype(param_dtype)) return ZERO_EINVAL;
+    if (!aligned16(table)) return ZERO_EALIGN;
+    const TableLayout L = table_layout(T, R);
+    if (table_bytes < L.total) return ZERO_EINVAL;
+    std::vector<unsigned char> buf(L.total, 0);
+    uint64_t* offs = reinterpret_cast<uint64_t*>(buf.data() + L.offs);
+    void** prm = reinterpret_cast<void**>(buf.data() + L.params);
+    const void** grd = reinterpret_cast<const void**>(buf.data() + L.grads);
+    uint32_t* flags = reinterpret_cast<uint32_t*>(buf.data() + L.flags);
+    uint64_t P = 0;
+    for (uint32_t j = 0; j < T; ++j) {
+        offs[j] = P;
+        if (numel[j] > (UINT64_MAX >> 3) - P) return ZERO_EOVERFLOW;
+        P += numel[j];
+        bool vec_ok = (offs[j] & 7u) == 0;
+        if (numel[j] > 0 && params16[j] == nullptr) return ZERO_EINVAL;
+        vec_ok = vec_ok && aligned16(params16[j]);
+        prm[j] = params16[j];
+        for (uint32_t r = 0; r < R; ++r) {
+            const void* g = grads[(size_t)r * T + j];
+            if (numel[j] > 0 && g == nullptr) return ZERO_EINVAL;
+            vec_ok = vec_ok && aligned16(g);
+            grd[(size_t)j * R + r] = g;
+        }
+        flags[j] = vec_ok ? 1u : 0u;
+    }
+    offs[T] = P;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(table, buf.data(), L.total, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return zadam_record_cuda(e);
+    out->table = table;
+    out->P = P;
+    out->T = T;
+    out->R = R;
+    out->grad_dtype = grad_dtype;
+    out->param_dtype = param_dtype;
+    out->table_bytes = L.total;
+    return ZERO_OK;
+}
+
+int zero_gather_params(const float* master, void* params16, int32_t param_dtype, uint64_t P, void* stream) {
+    if (!is_param_dtype(param_dtype)) return ZERO_EINVAL;
+    if (P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
+    if (P > 0 && (master == nullptr || params16 == nullptr)) return ZERO_EINVAL;
+    if (!aligned16(master) || !aligned16(params16)) return ZERO_EALIGN;
+    if (P == 0) return ZERO_OK;
+    GatherParams gp;
+    std::memset(&gp, 0, sizeof gp);
+    gp.w[0] = gp.w[1] = master;
+    gp.params16 = params16;
+    gp.lo = 0;
+    gp.hi = P;
+    int err = ZERO_OK;
+    const void* fn = gather_fn<false>(param_dtype);
+    const int ctas = resident_ctas(fn, &err);
+    if (err) return err;
+    const Shape sh = make_shape(0, P, ctas);
+    gp.base = sh.base;
+    gp.chunk = sh.chunk;
+    return launch(fn, sh, &gp, static_cast<cudaStream_t>(stream));
+}
+
+int zero_gather_params_list(const float* master, const zero_tensor_list* l, void* stream) {
+    int rc = check_list(l);
+    if (rc) return rc;
+    if (l->P > 0 && master == nullptr) return ZERO_EINVAL;
+    if (!aligned16(master)) return ZERO_EALIGN;
+    if (l->P == 0) return ZERO_OK;
+    GatherParams gp;
+    std::memset(&gp, 0, sizeof gp);
+    gp.w[0] = gp.w[1] = master;
+    gp.tab = device_table(l);
+    gp.lo = 0;
+    gp.hi = l->P;
+    int err = ZERO_OK;
+    const void* fn = gather_fn<true>(l->param_dtype);
+    const int ctas = resident_ctas(fn, &err);
+    if (err) return err;
+    const Shape sh = make_shape(0, l->P, ctas);
+    gp.base = sh.base;
+    gp.chunk = sh.chunk;
+    return launch(fn, sh, &gp, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// zero_adam_host.cpp -- the pure host functions of the C ABI (no CUDA):
+// ownership bounds, per-rank state accounting and status texts.
+#include <cstdint>
+
+#include "zero_adam.h"
+
+extern "C" {
+
+// "Deep dive: DeepSpeed", "Reduce first, then update the owned slice":
+// owner r keeps [floor(P*r/R), floor(P*(r+1)/R)); 128-bit products so that
+// P*r never wraps.
+int zero_partition_bounds(uint64_t P, uint32_t R, uint64_t* lo, uint64_t* hi) {
+    if (R == 0 || lo == nullptr || hi == nullptr) return ZERO_EINVAL;
+    const unsigned __int128 p = P;
+    for (uint32_t r = 0; r < R; ++r) {
+        lo[r] = (uint64_t)((p * r) / R);
+        hi[r] = (uint64_t)((p * (r + 1u)) / R);
+    }
+    return ZERO_OK;
+}
+
+// "Deep dive: DeepSpeed", "Count state before choosing a stage": each stage
+// keeps a 1/R share of one more kind of state (optimizer, then gradient,
+// then weight).  Returned multiplied by R so the values stay integers.
+int zero_state_bytes(uint64_t P, uint32_t R, uint32_t param_b, uint32_t grad_b, uint32_t opt_b,
+                     uint64_t out_times_R[4]) {
+    if (P == 0 || R == 0 || param_b == 0 || grad_b == 0 || opt_b == 0 || out_times_R == nullptr)
+        return ZERO_EINVAL;
+    const uint32_t width[3] = {opt_b, grad_b, param_b};  // the order the stages shard them
+    for (int stage = 0; stage < 4; ++stage) {
+        unsigned __int128 total = 0;
+        for (int k = 0; k < 3; ++k) {
+            // replicated: P*width bytes (R*P*width after scaling by R);
+            // sharded: P*width/R bytes (P*width after scaling by R)
+            unsigned __int128 term = (unsigned __int128)P * width[k];
+            if (k >= stage) term *= R;
+            total += term;
+        }
+        if (total > (unsigned __int128)UINT64_MAX) return ZERO_EOVERFLOW;
+        out_times_R[stage] = (uint64_t)total;
+    }
+    return ZERO_OK;
+}
+
+const char* zero_status_string(int status) {
+    switch (status) {
+        case ZERO_OK: return "ok";
+        case ZERO_EINVAL: return "invalid argument (NULL pointer, unknown dtype, bad count or hyperparameter)";
+        case ZERO_EALIGN: return "device pointer not 16-byte aligned";
+        case ZERO_EOVERFLOW: return "byte size overflows 64 bits";
+        case ZERO_ERANGE: return "count beyond a documented limit";
+        case ZERO_ECUDA: return "CUDA runtime error (see zero_last_cuda_error)";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

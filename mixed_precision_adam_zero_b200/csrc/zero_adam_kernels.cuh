@@ -1,0 +1,584 @@
+// zero_adam_kernels.cuh -- sm_100a kernels of the fused ZeRO-2/3 Adam step.
+//
+// The step is HBM-bound (about 25 flops against 2R+26 bytes per parameter),
+// so it is written as streaming kernels, not as tensor-core work:
+//   * one CTA per slot of a persistent grid (SMs x resident CTAs), each CTA
+//     owning one contiguous range of the flat index space, so every CTA
+//     streams sequential addresses and the ranges balance to within 8
+//     elements;
+//   * 128-bit loads and stores with the streaming (evict-first) cache hint;
+//     one vector is 8 elements: one 16-byte load per 16-bit gradient, two per
+//     fp32 array;
+//   * the rank reduction is a fixed-order float64 FMA chain over r = 0..R-1
+//     of the raw rank weights times the gradients (both exact in float64),
+//     scaled once by 1/(sum(w)*S) and rounded once to float32.  A float32
+//     chain is not enough: at small step counts Adam moves w by about
+//     lr*g/(|g|+eps), whose sensitivity to an absolute error in g reaches
+//     lr/eps, so the reduced gradient must be accurate relative to itself
+//     even where the ranks' gradients nearly cancel.  The chain is the same
+//     in the vector and the scalar path, so results are bitwise reproducible;
+//   * grid-level results (the inf/NaN flag, the step counter) use a
+//     last-block-done epilogue: each CTA fences and bumps an arrival counter
+//     in the workspace, and the CTA that arrives last updates the control
+//     block and re-zeroes the workspace.  Nothing spins or waits.
+//
+// Sources of the arithmetic ("Deep dive: DeepSpeed", "Reduce first, then
+// update the owned slice"; AdamW of the "ZeRO" documentation page): see
+// include/zero_adam.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zero_adam.h"
+
+namespace zadam {
+
+constexpr int kThreads = 256;  // threads per CTA
+constexpr int kVec = 8;        // elements per vector
+
+// Scratch of one step call (ZERO_WORKSPACE_BYTES).  All zero between calls.
+struct Workspace {
+    unsigned int arrive;  // CTAs of the running launch that have finished
+    unsigned int found;   // nonzero: some gradient was inf or NaN
+    unsigned int pad[62];
+};
+static_assert(sizeof(Workspace) == ZERO_WORKSPACE_BYTES, "workspace size");
+
+struct Hyper {
+    float b1, b2, omb1, omb2, eps, lr_wd;  // float32 per-element constants
+    double lr, b1d, b2d;                   // float64, for the bias corrections
+};
+
+// Device view of a tensor-list table.
+struct Table {
+    const uint64_t* offs;       // [T+1] flat start of each tensor, offs[T] = P
+    void* const* params;        // [T] 16-bit parameter tensors
+    const void* const* grads;   // [T*R] gradients, tensor-major: grads[j*R + r]
+    const uint32_t* flags;      // [T] bit 0: vector path allowed
+    uint32_t T;
+};
+
+struct StepParams {
+    const void* grads[ZERO_MAX_RANKS];  // flat call: rank r's gradient [P]
+    double wt[ZERO_MAX_RANKS];          // rank weights w_r (1 for the equal mean)
+    double wsum;                        // sum of the w_r
+    float* w[2];                        // master sets
+    float* m[2];
+    float* v[2];
+    void* params16;                     // flat call: 16-bit parameters [P]
+    float* reduced;                     // optional reduced-gradient output
+    Table tab;                          // list call
+    uint64_t lo, hi;                    // elements this launch updates
+    uint64_t base, chunk;               // CTA b: [base + b*chunk, base + (b+1)*chunk) within [lo, hi)
+    Hyper h;
+    zero_ctrl* ctrl;
+    Workspace* ws;
+    uint32_t R;
+    uint32_t growth_interval;
+    int32_t two_set;  // 1: read set ctrl.parity, write the other set
+    int32_t check;    // 0: none; 1: detect inf/NaN in this pass; 2: a scan decided
+};
+
+struct GatherParams {
+    const float* w[2];
+    void* params16;
+    Table tab;
+    uint64_t lo, hi, base, chunk;
+    const zero_ctrl* ctrl;     // non-NULL: read the set at ctrl.parity
+    int32_t only_if_skipped;   // 1: do nothing unless ctrl.last_skipped
+};
+
+// Per-call scalars derived from the control block.
+struct Scal {
+    float b1, b2, omb1, omb2, eps, lr_wd;
+    float step;          // lr / (1 - b1^t)
+    float inv_sqrt_bc2;  // 1 / sqrt(1 - b2^t)
+    double inv_ws;       // 1 / (sum(w) * S)
+};
+
+// b^e by binary exponentiation (float64).
+__device__ __forceinline__ double pow_u64(double b, uint64_t e) {
+    double r = 1.0;
+    while (e) {
+        if (e & 1ull) r *= b;
+        b *= b;
+        e >>= 1;
+    }
+    return r;
+}
+
+__device__ __forceinline__ Scal make_scal(const Hyper& h, uint64_t t, float S, double wsum) {
+    Scal s;
+    s.b1 = h.b1;
+    s.b2 = h.b2;
+    s.omb1 = h.omb1;
+    s.omb2 = h.omb2;
+    s.eps = h.eps;
+    s.lr_wd = h.lr_wd;
+    const double bc1 = 1.0 - pow_u64(h.b1d, t);
+    const double bc2 = 1.0 - pow_u64(h.b2d, t);
+    s.step = (float)(h.lr / bc1);
+    s.inv_sqrt_bc2 = (float)(1.0 / sqrt(bc2));
+    s.inv_ws = 1.0 / (wsum * (double)S);
+    return s;
+}
+
+// One element of Adam/AdamW on the reduced, unscaled gradient g.
+__device__ __forceinline__ void adam1(float g, float& w, float& m, float& v, const Scal& s) {
+    m = fmaf(s.b1, m, s.omb1 * g);
+    v = fmaf(s.b2, v, s.omb2 * (g * g));
+    const float denom = fmaf(sqrtf(v), s.inv_sqrt_bc2, s.eps);
+    w = w - fmaf(s.step, m / denom, s.lr_wd * w);
+}
+
+// ------------------------------------------------------------ gradient I/O
+
+template <class G> struct Raw8;
+template <> struct Raw8<float> { uint4 a, b; };
+template <> struct Raw8<__nv_bfloat16> { uint4 a; };
+template <> struct Raw8<__half> { uint4 a; };
+
+template <class G> __device__ __forceinline__ Raw8<G> load8(const G* p, uint64_t i);
+template <> __device__ __forceinline__ Raw8<float> load8<float>(const float* p, uint64_t i) {
+    Raw8<float> r;
+    r.a = __ldcs(reinterpret_cast<const uint4*>(p + i));
+    r.b = __ldcs(reinterpret_cast<const uint4*>(p + i + 4));
+    return r;
+}
+template <> __device__ __forceinline__ Raw8<__nv_bfloat16> load8<__nv_bfloat16>(const __nv_bfloat16* p, uint64_t i) {
+    Raw8<__nv_bfloat16> r;
+    r.a = __ldcs(reinterpret_cast<const uint4*>(p + i));
+    return r;
+}
+template <> __device__ __forceinline__ Raw8<__half> load8<__half>(const __half* p, uint64_t i) {
+    Raw8<__half> r;
+    r.a = __ldcs(reinterpret_cast<const uint4*>(p + i));
+    return r;
+}
+
+__device__ __forceinline__ void bf16x2(uint32_t u, float& lo, float& hi) {
+    lo = __uint_as_float(u << 16);
+    hi = __uint_as_float(u & 0xFFFF0000u);
+}
+__device__ __forceinline__ void f16x2(uint32_t u, float& lo, float& hi) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&u));
+    lo = f.x;
+    hi = f.y;
+}
+
+__device__ __forceinline__ void unpack8(const Raw8<float>& r, float (&f)[8]) {
+    f[0] = __uint_as_float(r.a.x); f[1] = __uint_as_float(r.a.y);
+    f[2] = __uint_as_float(r.a.z); f[3] = __uint_as_float(r.a.w);
+    f[4] = __uint_as_float(r.b.x); f[5] = __uint_as_float(r.b.y);
+    f[6] = __uint_as_float(r.b.z); f[7] = __uint_as_float(r.b.w);
+}
+__device__ __forceinline__ void unpack8(const Raw8<__nv_bfloat16>& r, float (&f)[8]) {
+    bf16x2(r.a.x, f[0], f[1]); bf16x2(r.a.y, f[2], f[3]);
+    bf16x2(r.a.z, f[4], f[5]); bf16x2(r.a.w, f[6], f[7]);
+}
+__device__ __forceinline__ void unpack8(const Raw8<__half>& r, float (&f)[8]) {
+    f16x2(r.a.x, f[0], f[1]); f16x2(r.a.y, f[2], f[3]);
+    f16x2(r.a.z, f[4], f[5]); f16x2(r.a.w, f[6], f[7]);
+}
+
+// Non-finite test on raw bits: exponent field all ones.
+__device__ __forceinline__ bool exp_all_ones32(uint32_t u) { return (u & 0x7F800000u) == 0x7F800000u; }
+__device__ __forceinline__ bool exp_all_ones2(uint32_t u, uint32_t mask) {
+    return __vcmpeq2(u & mask, mask) != 0u;
+}
+__device__ __forceinline__ bool bad8(const Raw8<float>& r) {
+    return exp_all_ones32(r.a.x) | exp_all_ones32(r.a.y) | exp_all_ones32(r.a.z) | exp_all_ones32(r.a.w) |
+           exp_all_ones32(r.b.x) | exp_all_ones32(r.b.y) | exp_all_ones32(r.b.z) | exp_all_ones32(r.b.w);
+}
+__device__ __forceinline__ bool bad8(const Raw8<__nv_bfloat16>& r) {
+    const uint32_t k = 0x7F807F80u;
+    return exp_all_ones2(r.a.x, k) | exp_all_ones2(r.a.y, k) | exp_all_ones2(r.a.z, k) | exp_all_ones2(r.a.w, k);
+}
+__device__ __forceinline__ bool bad8(const Raw8<__half>& r) {
+    const uint32_t k = 0x7C007C00u;
+    return exp_all_ones2(r.a.x, k) | exp_all_ones2(r.a.y, k) | exp_all_ones2(r.a.z, k) | exp_all_ones2(r.a.w, k);
+}
+
+template <class G> __device__ __forceinline__ float load1(const G* p, uint64_t i, bool& bad);
+template <> __device__ __forceinline__ float load1<float>(const float* p, uint64_t i, bool& bad) {
+    const uint32_t u = __ldcs(reinterpret_cast<const unsigned int*>(p + i));
+    bad |= exp_all_ones32(u);
+    return __uint_as_float(u);
+}
+template <> __device__ __forceinline__ float load1<__nv_bfloat16>(const __nv_bfloat16* p, uint64_t i, bool& bad) {
+    const uint32_t u = __ldcs(reinterpret_cast<const unsigned short*>(p + i));
+    bad |= (u & 0x7F80u) == 0x7F80u;
+    return __uint_as_float(u << 16);
+}
+template <> __device__ __forceinline__ float load1<__half>(const __half* p, uint64_t i, bool& bad) {
+    const unsigned short u = __ldcs(reinterpret_cast<const unsigned short*>(p + i));
+    bad |= (u & 0x7C00u) == 0x7C00u;
+    return __half2float(__ushort_as_half(u));
+}
+
+// ------------------------------------------------------------ parameter I/O
+
+template <class Pm> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+template <> __device__ __forceinline__ uint32_t pack2<__half>(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+template <class Pm> __device__ __forceinline__ unsigned short cvt1(float x);
+template <> __device__ __forceinline__ unsigned short cvt1<__nv_bfloat16>(float x) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
+template <> __device__ __forceinline__ unsigned short cvt1<__half>(float x) {
+    return __half_as_ushort(__float2half_rn(x));
+}
+
+// Gradient base pointers of one tensor: registers for a compile-time rank
+// count, or read through from parameter/shared memory for any R.
+template <class G, int RC> struct GradPtrs {
+    const G* p[RC];
+    __device__ __forceinline__ explicit GradPtrs(const void* const* src) {
+#pragma unroll
+        for (int r = 0; r < RC; ++r) p[r] = static_cast<const G*>(src[r]);
+    }
+    __device__ __forceinline__ const G* operator[](int r) const { return p[r]; }
+};
+template <class G> struct GradPtrs<G, 0> {
+    const void* const* src;
+    __device__ __forceinline__ explicit GradPtrs(const void* const* s) : src(s) {}
+    __device__ __forceinline__ const G* operator[](int r) const { return static_cast<const G*>(src[r]); }
+};
+
+struct StateIO {
+    const float* wi;
+    const float* mi;
+    const float* vi;
+    float* wo;
+    float* mo;
+    float* vo;
+};
+
+// ------------------------------------------------------------ step bodies
+
+// One 8-element vector at flat index e (multiple of 8); le = e - tensor start.
+template <class G, class Pm, int RC>
+__device__ __forceinline__ void vec_step(const StepParams& p, const Scal& s, const GradPtrs<G, RC>& gp,
+                                         Pm* pp, uint64_t e, uint64_t le, const StateIO& io, bool& bad) {
+    double acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.0;
+
+    float4 w0, w1, m0, m1, v0, v1;
+    if constexpr (RC > 0) {
+        Raw8<G> raw[RC];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) raw[r] = load8<G>(gp[r], le);
+        w0 = __ldcs(reinterpret_cast<const float4*>(io.wi + e));
+        w1 = __ldcs(reinterpret_cast<const float4*>(io.wi + e + 4));
+        m0 = __ldcs(reinterpret_cast<const float4*>(io.mi + e));
+        m1 = __ldcs(reinterpret_cast<const float4*>(io.mi + e + 4));
+        v0 = __ldcs(reinterpret_cast<const float4*>(io.vi + e));
+        v1 = __ldcs(reinterpret_cast<const float4*>(io.vi + e + 4));
+#pragma unroll
+        for (int r = 0; r < RC; ++r) {
+            if (p.check == 1) bad |= bad8(raw[r]);
+            float f[8];
+            unpack8(raw[r], f);
+            const double c = p.wt[r];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = fma(c, (double)f[k], acc[k]);
+        }
+    } else {
+        w0 = __ldcs(reinterpret_cast<const float4*>(io.wi + e));
+        w1 = __ldcs(reinterpret_cast<const float4*>(io.wi + e + 4));
+        m0 = __ldcs(reinterpret_cast<const float4*>(io.mi + e));
+        m1 = __ldcs(reinterpret_cast<const float4*>(io.mi + e + 4));
+        v0 = __ldcs(reinterpret_cast<const float4*>(io.vi + e));
+        v1 = __ldcs(reinterpret_cast<const float4*>(io.vi + e + 4));
+        const int R = (int)p.R;
+        for (int r0 = 0; r0 < R; r0 += 8) {
+            Raw8<G> raw[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                if (r0 + q < R) raw[q] = load8<G>(gp[r0 + q], le);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (r0 + q < R) {
+                    if (p.check == 1) bad |= bad8(raw[q]);
+                    float f[8];
+                    unpack8(raw[q], f);
+                    const double c = p.wt[r0 + q];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) acc[k] = fma(c, (double)f[k], acc[k]);
+                }
+            }
+        }
+    }
+
+    float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+    float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float g[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        g[k] = (float)(acc[k] * s.inv_ws);
+        adam1(g[k], w[k], m[k], v[k], s);
+    }
+    __stcs(reinterpret_cast<float4*>(io.wo + e), make_float4(w[0], w[1], w[2], w[3]));
+    __stcs(reinterpret_cast<float4*>(io.wo + e + 4), make_float4(w[4], w[5], w[6], w[7]));
+    __stcs(reinterpret_cast<float4*>(io.mo + e), make_float4(m[0], m[1], m[2], m[3]));
+    __stcs(reinterpret_cast<float4*>(io.mo + e + 4), make_float4(m[4], m[5], m[6], m[7]));
+    __stcs(reinterpret_cast<float4*>(io.vo + e), make_float4(v[0], v[1], v[2], v[3]));
+    __stcs(reinterpret_cast<float4*>(io.vo + e + 4), make_float4(v[4], v[5], v[6], v[7]));
+    uint4 o;
+    o.x = pack2<Pm>(w[0], w[1]);
+    o.y = pack2<Pm>(w[2], w[3]);
+    o.z = pack2<Pm>(w[4], w[5]);
+    o.w = pack2<Pm>(w[6], w[7]);
+    __stcs(reinterpret_cast<uint4*>(pp + le), o);
+    if (p.reduced != nullptr) {
+        __stcs(reinterpret_cast<float4*>(p.reduced + e), make_float4(g[0], g[1], g[2], g[3]));
+        __stcs(reinterpret_cast<float4*>(p.reduced + e + 4), make_float4(g[4], g[5], g[6], g[7]));
+    }
+}
+
+// One element (heads, tails and tensors that cannot take the vector path).
+template <class G, class Pm, int RC>
+__device__ __forceinline__ void elem_step(const StepParams& p, const Scal& s, const GradPtrs<G, RC>& gp,
+                                          Pm* pp, uint64_t e, uint64_t le, const StateIO& io, bool& bad) {
+    double acc = 0.0;
+    const int R = RC > 0 ? RC : (int)p.R;
+    for (int r = 0; r < R; ++r) {
+        bool b = false;
+        const float x = load1<G>(gp[r], le, b);
+        if (p.check == 1) bad |= b;
+        acc = fma(p.wt[r], (double)x, acc);
+    }
+    const float g = (float)(acc * s.inv_ws);
+    float w = io.wi[e], m = io.mi[e], v = io.vi[e];
+    adam1(g, w, m, v, s);
+    io.wo[e] = w;
+    io.mo[e] = m;
+    io.vo[e] = v;
+    reinterpret_cast<unsigned short*>(pp)[le] = cvt1<Pm>(w);
+    if (p.reduced != nullptr) p.reduced[e] = g;
+}
+
+// Flat range [a, b) of one tensor that starts at flat index toff.
+template <class G, class Pm, int RC>
+__device__ __forceinline__ void run_segment(const StepParams& p, const Scal& s, const GradPtrs<G, RC>& gp,
+                                            Pm* pp, uint64_t toff, uint64_t a, uint64_t b, bool vec_ok,
+                                            const StateIO& io, bool& bad) {
+    uint64_t va = b, vb = b;
+    if (vec_ok) {
+        va = (a + 7) & ~7ull;
+        if (va > b) va = b;
+        vb = b & ~7ull;
+        if (vb < va) vb = va;
+    }
+    for (uint64_t e = a + threadIdx.x; e < va; e += kThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e - toff, io, bad);
+    for (uint64_t e = va + (uint64_t)threadIdx.x * kVec; e < vb; e += (uint64_t)kThreads * kVec)
+        vec_step<G, Pm, RC>(p, s, gp, pp, e, e - toff, io, bad);
+    for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e - toff, io, bad);
+}
+
+// Index of the tensor holding flat element x (offs[j] <= x < offs[j+1]).
+__device__ __forceinline__ uint32_t find_tensor(const Table& t, uint64_t x) {
+    uint32_t lo = 0, hi = t.T;
+    while (hi - lo > 1) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (t.offs[mid] <= x) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// Grid-level epilogue: the last CTA to finish updates the control block.
+__device__ __forceinline__ void finish_step(const StepParams& p, bool bad) {
+    const int any = __syncthreads_or(bad ? 1 : 0);
+    if (threadIdx.x == 0) {
+        Workspace* ws = p.ws;
+        if (any) atomicOr(&ws->found, 1u);
+        __threadfence();
+        const unsigned prev = atomicAdd(&ws->arrive, 1u);
+        if (prev == gridDim.x - 1) {
+            __threadfence();
+            const unsigned found = p.check ? atomicOr(&ws->found, 0u) : 0u;
+            zero_ctrl* c = p.ctrl;
+            if (found) {
+                c->loss_scale *= 0.5f;
+                c->growth_tracker = 0u;
+                c->skipped += 1ull;
+                c->last_skipped = 1u;
+            } else {
+                c->step += 1ull;
+                c->last_skipped = 0u;
+                if (p.two_set) c->parity ^= 1u;
+                if (p.check) {
+                    uint32_t gt = c->growth_tracker + 1u;
+                    if (p.growth_interval != 0u && gt >= p.growth_interval) {
+                        c->loss_scale *= 2.0f;
+                        gt = 0u;
+                    }
+                    c->growth_tracker = gt;
+                }
+            }
+            ws->found = 0u;
+            ws->arrive = 0u;
+            __threadfence();
+        }
+    }
+}
+
+template <class G, class Pm, int RC, bool LIST>
+__global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ StepParams p) {
+    __shared__ const void* s_gp[LIST ? ZERO_MAX_RANKS : 1];
+    const zero_ctrl* c = p.ctrl;
+    const uint32_t par = p.two_set ? c->parity : 0u;
+    const uint32_t out = par ^ (uint32_t)p.two_set;
+    const StateIO io{p.w[par], p.m[par], p.v[par], p.w[out], p.m[out], p.v[out]};
+    bool skip = false;
+    if (p.check == 2) skip = *reinterpret_cast<volatile const unsigned*>(&p.ws->found) != 0u;
+    const Scal s = make_scal(p.h, c->step + 1ull, c->loss_scale, p.wsum);
+
+    uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
+    uint64_t b = a + p.chunk;
+    if (a < p.lo) a = p.lo;
+    if (b > p.hi) b = p.hi;
+    bool bad = false;
+    if (!skip && a < b) {
+        if constexpr (!LIST) {
+            const GradPtrs<G, RC> gp(&p.grads[0]);
+            run_segment<G, Pm, RC>(p, s, gp, static_cast<Pm*>(p.params16), 0ull, a, b, true, io, bad);
+        } else {
+            uint32_t j = find_tensor(p.tab, a);
+            uint64_t x = a;
+            while (x < b) {
+                const uint64_t t0 = p.tab.offs[j], t1 = p.tab.offs[j + 1];
+                const uint64_t sb = t1 < b ? t1 : b;
+                if (x < sb) {
+                    __syncthreads();
+                    for (uint32_t r = threadIdx.x; r < p.R; r += kThreads)
+                        s_gp[r] = p.tab.grads[(uint64_t)j * p.R + r];
+                    __syncthreads();
+                    const GradPtrs<G, RC> gp(s_gp);
+                    run_segment<G, Pm, RC>(p, s, gp, static_cast<Pm*>(p.tab.params[j]), t0, x, sb,
+                                           (p.tab.flags[j] & 1u) != 0u, io, bad);
+                }
+                x = sb;
+                ++j;
+            }
+        }
+    }
+    finish_step(p, bad);
+}
+
+// ------------------------------------------------------------ overflow scan
+
+template <class G>
+__device__ __forceinline__ void scan_range(const G* g, uint64_t a, uint64_t b, bool vec_ok, bool& bad) {
+    uint64_t va = b, vb = b;
+    if (vec_ok) {
+        va = (a + 7) & ~7ull;
+        if (va > b) va = b;
+        vb = b & ~7ull;
+        if (vb < va) vb = va;
+    }
+    for (uint64_t e = a + threadIdx.x; e < va; e += kThreads) (void)load1<G>(g, e, bad);
+    for (uint64_t e = va + (uint64_t)threadIdx.x * kVec; e < vb; e += (uint64_t)kThreads * kVec)
+        bad |= bad8(load8<G>(g, e));
+    for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads) (void)load1<G>(g, e, bad);
+}
+
+// Sets ws.found if any gradient of any rank in [lo, hi) is inf or NaN.
+template <class G, bool LIST>
+__global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ StepParams p) {
+    uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
+    uint64_t b = a + p.chunk;
+    if (a < p.lo) a = p.lo;
+    if (b > p.hi) b = p.hi;
+    bool bad = false;
+    if (a < b) {
+        if constexpr (!LIST) {
+            for (uint32_t r = 0; r < p.R; ++r) scan_range<G>(static_cast<const G*>(p.grads[r]), a, b, true, bad);
+        } else {
+            uint32_t j = find_tensor(p.tab, a);
+            uint64_t x = a;
+            while (x < b) {
+                const uint64_t t0 = p.tab.offs[j], t1 = p.tab.offs[j + 1];
+                const uint64_t sb = t1 < b ? t1 : b;
+                if (x < sb) {
+                    const bool vec_ok = (p.tab.flags[j] & 1u) != 0u;
+                    for (uint32_t r = 0; r < p.R; ++r)
+                        scan_range<G>(static_cast<const G*>(p.tab.grads[(uint64_t)j * p.R + r]), x - t0, sb - t0,
+                                      vec_ok, bad);
+                }
+                x = sb;
+                ++j;
+            }
+        }
+    }
+    if (__syncthreads_or(bad ? 1 : 0) && threadIdx.x == 0) atomicOr(&p.ws->found, 1u);
+}
+
+// ------------------------------------------------------------ 16-bit cast
+
+template <class Pm>
+__device__ __forceinline__ void cast_range(const float* w, Pm* pp, uint64_t toff, uint64_t a, uint64_t b,
+                                           bool vec_ok) {
+    uint64_t va = b, vb = b;
+    if (vec_ok) {
+        va = (a + 7) & ~7ull;
+        if (va > b) va = b;
+        vb = b & ~7ull;
+        if (vb < va) vb = va;
+    }
+    unsigned short* po = reinterpret_cast<unsigned short*>(pp);
+    for (uint64_t e = a + threadIdx.x; e < va; e += kThreads) po[e - toff] = cvt1<Pm>(w[e]);
+    for (uint64_t e = va + (uint64_t)threadIdx.x * kVec; e < vb; e += (uint64_t)kThreads * kVec) {
+        const float4 x = __ldcs(reinterpret_cast<const float4*>(w + e));
+        const float4 y = __ldcs(reinterpret_cast<const float4*>(w + e + 4));
+        uint4 o;
+        o.x = pack2<Pm>(x.x, x.y);
+        o.y = pack2<Pm>(x.z, x.w);
+        o.z = pack2<Pm>(y.x, y.y);
+        o.w = pack2<Pm>(y.z, y.w);
+        __stcs(reinterpret_cast<uint4*>(po + (e - toff)), o);
+    }
+    for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads) po[e - toff] = cvt1<Pm>(w[e]);
+}
+
+template <class Pm, bool LIST>
+__global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ GatherParams p) {
+    if (p.only_if_skipped && p.ctrl->last_skipped == 0u) return;
+    const float* w = p.ctrl != nullptr ? p.w[p.ctrl->parity & 1u] : p.w[0];
+    uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
+    uint64_t b = a + p.chunk;
+    if (a < p.lo) a = p.lo;
+    if (b > p.hi) b = p.hi;
+    if (a >= b) return;
+    if constexpr (!LIST) {
+        cast_range<Pm>(w, static_cast<Pm*>(p.params16), 0ull, a, b, true);
+    } else {
+        uint32_t j = find_tensor(p.tab, a);
+        uint64_t x = a;
+        while (x < b) {
+            const uint64_t t0 = p.tab.offs[j], t1 = p.tab.offs[j + 1];
+            const uint64_t sb = t1 < b ? t1 : b;
+            if (x < sb)
+                cast_range<Pm>(w, static_cast<Pm*>(p.tab.params[j]), t0, x, sb, (p.tab.flags[j] & 1u) != 0u);
+            x = sb;
+            ++j;
+        }
+    }
+}
+
+// ------------------------------------------------------------ control block
+
+__global__ void ctrl_set_kernel(zero_ctrl* c, zero_ctrl value) { *c = value; }
+
+}  // namespace zadam
