@@ -264,6 +264,33 @@ int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t *numel,
                           int32_t grad_dtype, int32_t param_dtype, void *table,
                           size_t table_bytes, zero_tensor_list *out, void *stream);
 
+/* Bytes of the library-owned scratch array behind zero_step_fused_noalloc. */
+#define ZERO_NOALLOC_SCRATCH_BYTES 256
+
+/* The same flat step as zero_step_fused, for callers that cannot allocate
+ * device memory: a plugin running inside another framework whose memory pool
+ * already holds the device's memory and that hands it only the parameter,
+ * gradient and optimizer-state buffers; a runtime that forbids allocation
+ * after start-up; or a latency-critical loop that must not take the device
+ * synchronisation cudaMalloc and cudaFree can imply.  The pages describe no
+ * counterpart of this entry point: it exists only for such callers.
+ *
+ * args->workspace must be NULL.  Instead of a caller workspace the step uses
+ * one library-owned array of ZERO_NOALLOC_SCRATCH_BYTES in device memory,
+ * which every GPU that loads the library keeps until the process exits.  The
+ * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine.  The first call on a device looks up that device's copy of the
+ * array (cudaGetSymbolAddress, with the device current); make that first
+ * call before any stream capture.  Each call clears the array on `stream`
+ * before the step, and the array keeps the last call's contents afterwards.
+ * All calls share the one array: calls that may overlap on the GPU (other
+ * streams, other host threads) race on it and must be ordered by the caller.
+ * The step needs ZERO_WORKSPACE_BYTES of scratch whatever P and R are; a
+ * build whose step needed more than the array holds would be refused with
+ * ZERO_ERANGE.  All other arguments, limits and errors are those of
+ * zero_step_fused. */
+int zero_step_fused_noalloc(const zero_step_args *args, void *stream);
+
 /* --------------------------------------------------------------- gathers */
 
 /* params16[i] = round-to-nearest-even(master[i]) for i in [0,P): the cast of

@@ -33,13 +33,14 @@ ZERO_F16 = 2
 
 ZERO_MAX_RANKS = 256
 ZERO_WORKSPACE_BYTES = 256
+ZERO_NOALLOC_SCRATCH_BYTES = 256
 
 EXPORTED = [
     "zero_partition_bounds", "zero_state_bytes", "zero_status_string", "zero_last_cuda_error",
     "zero_ctrl_bytes", "zero_workspace_bytes", "zero_list_table_bytes", "zero_ctrl_init",
     "zero_ctrl_set", "zero_ctrl_read", "zero_workspace_init", "zero_step_fused",
     "zero_step_fused_list", "zero_list_table_build", "zero_gather_params",
-    "zero_gather_params_list",
+    "zero_gather_params_list", "zero_step_fused_noalloc",
 ]
 
 
@@ -109,6 +110,7 @@ def _lib() -> ctypes.CDLL:
         L.zero_ctrl_read.argtypes = [vp, ctypes.POINTER(zero_ctrl), vp]
         L.zero_workspace_init.argtypes = [vp, vp]
         L.zero_step_fused.argtypes = [ctypes.POINTER(zero_step_args), vp]
+        L.zero_step_fused_noalloc.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_step_fused_list.argtypes = [ctypes.POINTER(zero_step_args), ctypes.POINTER(zero_tensor_list), vp]
         L.zero_list_table_build.argtypes = [u32, u32, u64p, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32,
                                             vp, sz, ctypes.POINTER(zero_tensor_list), vp]
@@ -230,6 +232,12 @@ def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master,
 
 def zero_step_fused(args: zero_step_args, stream=None) -> None:
     _check(_lib().zero_step_fused(ctypes.byref(args), _stream(stream)), "zero_step_fused")
+
+
+def zero_step_fused_noalloc(args: zero_step_args, stream=None) -> None:
+    """The flat step with the library's own scratch (args.workspace must be
+    NULL); for callers that cannot allocate device memory."""
+    _check(_lib().zero_step_fused_noalloc(ctypes.byref(args), _stream(stream)), "zero_step_fused_noalloc")
 
 
 def zero_step_fused_list(args: zero_step_args, lst: zero_tensor_list, stream=None) -> None:

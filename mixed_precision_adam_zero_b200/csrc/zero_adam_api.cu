@@ -304,6 +304,34 @@ int check_list(const zero_tensor_list* l) {
     return ZERO_OK;
 }
 
+// ------------------------------------------------------------ no-alloc scratch
+
+// Library-owned scratch of zero_step_fused_noalloc: one workspace per device,
+// alive until the process exits.  Host code sees only a stand-in symbol; the
+// device address comes from cudaGetSymbolAddress with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ZERO_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of this device's scratch array (looked up on first use).
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return zadam_record_cuda(e);
+    if (dev < 0 || dev >= kMaxDevices) return ZERO_ERANGE;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return zadam_record_cuda(e);
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return ZERO_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI
@@ -375,6 +403,20 @@ int zero_step_fused_list(const zero_step_args* a, const zero_tensor_list* l, voi
         return ZERO_EINVAL;
     kp.tab = device_table(l);
     return run_step<true>(a, &kp, static_cast<cudaStream_t>(stream));
+}
+
+int zero_step_fused_noalloc(const zero_step_args* a, void* stream) {
+    if (a == nullptr || a->workspace != nullptr) return ZERO_EINVAL;
+    if (ZERO_WORKSPACE_BYTES > ZERO_NOALLOC_SCRATCH_BYTES) return ZERO_ERANGE;
+    void* ws = nullptr;
+    int rc = noalloc_scratch(&ws);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = cudaMemsetAsync(ws, 0, ZERO_WORKSPACE_BYTES, st);
+    if (e != cudaSuccess) return zadam_record_cuda(e);
+    zero_step_args b = *a;
+    b.workspace = ws;
+    return zero_step_fused(&b, stream);
 }
 
 int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t* numel, void* const* params16,

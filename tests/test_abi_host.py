@@ -168,3 +168,10 @@ def test_gather_and_ctrl_argument_errors():
 def test_list_table_bytes():
     T, R = 292, 4
     assert za.zero_list_table_bytes(T, R) == 8 * (T + 1) + 8 * T + 8 * T * R + ((4 * T + 15) // 16) * 16
+
+
+def test_noalloc_step_refuses_a_caller_workspace():
+    a = _args()                                    # carries a workspace pointer
+    with pytest.raises(za.ZeroError) as e:
+        za.zero_step_fused_noalloc(a)
+    assert e.value.status == za.ZERO_EINVAL
