@@ -59,6 +59,7 @@ def bytes_per_param(R: int, gdt: str) -> int:
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
     for rel in ("mixed_precision_adam_zero_b200/csrc/zero_adam_kernels.cuh",
+                "mixed_precision_adam_zero_b200/csrc/zero_adam_bulk.cuh",
                 "mixed_precision_adam_zero_b200/csrc/zero_adam_api.cu"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())

@@ -96,7 +96,11 @@ typedef struct zero_ctrl {
     uint32_t growth_tracker;  /* applied steps since S last changed (check on) */
     uint32_t parity;          /* two-set mode: index of the set holding the state */
     uint32_t last_skipped;    /* 1 if the most recent step call skipped */
-    uint32_t reserved[2];     /* zero */
+    uint32_t device_error;    /* nonzero: a bounded device-side wait of some
+                                 step gave up (sticky until reset with
+                                 zero_ctrl_set); that step's results are
+                                 undefined.  Never expected in normal use. */
+    uint32_t reserved;        /* zero */
 } zero_ctrl;
 
 /* Arguments of one step over a FLAT parameter vector of P elements.

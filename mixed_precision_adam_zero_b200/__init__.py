@@ -62,7 +62,7 @@ class zero_ctrl(ctypes.Structure):
     _fields_ = [("step", ctypes.c_uint64), ("skipped", ctypes.c_uint64),
                 ("loss_scale", ctypes.c_float), ("growth_tracker", ctypes.c_uint32),
                 ("parity", ctypes.c_uint32), ("last_skipped", ctypes.c_uint32),
-                ("reserved", ctypes.c_uint32 * 2)]
+                ("device_error", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
 
 
 class zero_step_args(ctypes.Structure):

@@ -9,6 +9,7 @@
 
 #include "zero_adam.h"
 #include "zero_adam_kernels.cuh"
+#include "zero_adam_bulk.cuh"
 
 using namespace zadam;
 
@@ -30,11 +31,18 @@ struct OccEntry {
     int ctas;  // max CTAs resident on the whole device
 };
 
+// A kernel and the dynamic shared memory it is launched with.
+struct Kern {
+    const void* fn;
+    unsigned smem;
+};
+
 std::mutex g_occ_mu;
 std::vector<OccEntry> g_occ;
 
 // Resident CTAs of `fn` on the current device (SMs x CTAs per SM), cached.
-int resident_ctas(const void* fn, int* err) {
+// A kernel with dynamic shared memory gets its opt-in limit raised first.
+int resident_ctas(const void* fn, int* err, unsigned smem = 0) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) { *err = zadam_record_cuda(e); return 0; }
@@ -45,7 +53,9 @@ int resident_ctas(const void* fn, int* err) {
     }
     int sms = 0, per_sm = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, 0);
+    if (e == cudaSuccess && smem > 0)
+        e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
     if (e != cudaSuccess) { *err = zadam_record_cuda(e); return 0; }
     if (per_sm < 1) per_sm = 1;
     const int ctas = sms * per_sm;
@@ -78,14 +88,42 @@ Shape make_shape(uint64_t lo, uint64_t hi, int max_ctas) {
     return s;
 }
 
-int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st) {
+int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st, unsigned smem = 0) {
     void* args[] = {params};
-    const cudaError_t e = cudaLaunchKernel(fn, dim3(sh.grid), dim3(kThreads), args, 0, st);
+    const cudaError_t e = cudaLaunchKernel(fn, dim3(sh.grid), dim3(kThreads), args, smem, st);
     if (e != cudaSuccess) return zadam_record_cuda(e);
     return ZERO_OK;
 }
 
 // ------------------------------------------------------------ kernel tables
+
+// Flat calls with a compile-time rank count stage their tiles through shared
+// memory with bulk copies; other rank counts and lists use the register path.
+template <class G, class Pm, int RC>
+Kern bulk_kern() {
+    return Kern{(const void*)step_bulk_kernel<G, Pm, RC>, BulkShape<G, RC>::kSmem};
+}
+
+template <class G, class Pm>
+Kern step_kern_flat(uint32_t R) {
+#ifndef ZADAM_REGISTER_PATH_ONLY
+    switch (R) {
+        case 1: return bulk_kern<G, Pm, 1>();
+        case 2: return bulk_kern<G, Pm, 2>();
+        case 4: return bulk_kern<G, Pm, 4>();
+        case 8: return bulk_kern<G, Pm, 8>();
+        default: break;
+    }
+#endif
+    return Kern{(const void*)step_kernel<G, Pm, 0, false>, 0u};
+}
+
+template <class G>
+Kern step_kern_flat_pm(int32_t param_dtype, uint32_t R) {
+    return param_dtype == ZERO_BF16 ? step_kern_flat<G, __nv_bfloat16>(R) : step_kern_flat<G, __half>(R);
+}
+
+Kern step_kern(bool list, int32_t grad_dtype, int32_t param_dtype, uint32_t R);
 
 template <class G, class Pm, bool LIST>
 const void* step_fn_rc(uint32_t R) {
@@ -110,6 +148,19 @@ const void* step_fn(int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
         case ZERO_BF16: return step_fn_pm<__nv_bfloat16, LIST>(param_dtype, R);
         default: return step_fn_pm<__half, LIST>(param_dtype, R);
     }
+}
+
+Kern step_kern(bool list, int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
+    if (list) return Kern{step_fn<true>(grad_dtype, param_dtype, R), 0u};
+#ifdef ZADAM_REGISTER_PATH_ONLY
+    return Kern{step_fn<false>(grad_dtype, param_dtype, R), 0u};
+#else
+    switch (grad_dtype) {
+        case ZERO_F32: return step_kern_flat_pm<float>(param_dtype, R);
+        case ZERO_BF16: return step_kern_flat_pm<__nv_bfloat16>(param_dtype, R);
+        default: return step_kern_flat_pm<__half>(param_dtype, R);
+    }
+#endif
 }
 
 template <bool LIST>
@@ -237,13 +288,13 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
     } else {
         kp->check = check ? 1 : 0;
     }
-    const void* fn = step_fn<LIST>(a->grad_dtype, a->param_dtype, a->R);
-    const int ctas = resident_ctas(fn, &err);
+    const Kern k = step_kern(LIST, a->grad_dtype, a->param_dtype, a->R);
+    const int ctas = resident_ctas(k.fn, &err, k.smem);
     if (err) return err;
     const Shape sh = make_shape(lo, hi, ctas);
     kp->base = sh.base;
     kp->chunk = sh.chunk;
-    if ((err = launch(fn, sh, kp, st))) return err;
+    if ((err = launch(k.fn, sh, kp, st, k.smem))) return err;
     if (single_pass) {
         // Only if the step was skipped: re-cast the 16-bit parameters from
         // the master set that stayed current.

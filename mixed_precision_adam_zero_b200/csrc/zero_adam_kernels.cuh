@@ -43,7 +43,8 @@ constexpr int kVec = 8;        // elements per vector
 struct Workspace {
     unsigned int arrive;  // CTAs of the running launch that have finished
     unsigned int found;   // nonzero: some gradient was inf or NaN
-    unsigned int pad[62];
+    unsigned int error;   // nonzero: a bounded device-side wait gave up
+    unsigned int pad[61];
 };
 static_assert(sizeof(Workspace) == ZERO_WORKSPACE_BYTES, "workspace size");
 
@@ -427,7 +428,10 @@ __device__ __forceinline__ void finish_step(const StepParams& p, bool bad) {
                     c->growth_tracker = gt;
                 }
             }
+            const unsigned err = atomicOr(&ws->error, 0u);
+            if (err) c->device_error = err;
             ws->found = 0u;
+            ws->error = 0u;
             ws->arrive = 0u;
             __threadfence();
         }
