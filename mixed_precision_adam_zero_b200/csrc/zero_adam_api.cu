@@ -31,10 +31,11 @@ struct OccEntry {
     int ctas;  // max CTAs resident on the whole device
 };
 
-// A kernel and the dynamic shared memory it is launched with.
+// A kernel, its block size and the dynamic shared memory it is launched with.
 struct Kern {
     const void* fn;
     unsigned smem;
+    int threads;
 };
 
 std::mutex g_occ_mu;
@@ -42,7 +43,7 @@ std::vector<OccEntry> g_occ;
 
 // Resident CTAs of `fn` on the current device (SMs x CTAs per SM), cached.
 // A kernel with dynamic shared memory gets its opt-in limit raised first.
-int resident_ctas(const void* fn, int* err, unsigned smem = 0) {
+int resident_ctas(const void* fn, int* err, unsigned smem = 0, int threads = kThreads) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) { *err = zadam_record_cuda(e); return 0; }
@@ -55,7 +56,7 @@ int resident_ctas(const void* fn, int* err, unsigned smem = 0) {
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess && smem > 0)
         e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
     if (e != cudaSuccess) { *err = zadam_record_cuda(e); return 0; }
     if (per_sm < 1) per_sm = 1;
     const int ctas = sms * per_sm;
@@ -70,57 +71,60 @@ struct Shape {
 };
 
 // Split [lo, hi) into at most max_ctas contiguous CTA ranges whose inner
-// boundaries are multiples of 8 (absolute index), each at least one vector
-// per thread long.
+// boundaries are multiples of 64 elements (absolute index: 128-byte aligned
+// for 16-bit arrays), each at least one vector per thread long.
+constexpr uint64_t kChunkAlign = 64;
+
 Shape make_shape(uint64_t lo, uint64_t hi, int max_ctas) {
     Shape s;
-    s.base = lo & ~7ull;
-    if (hi <= lo) { s.chunk = kVec; s.grid = 1; return s; }
+    s.base = lo & ~(kChunkAlign - 1);
+    if (hi <= lo) { s.chunk = kChunkAlign; s.grid = 1; return s; }
     const uint64_t n = hi - s.base;
     const uint64_t min_chunk = (uint64_t)kThreads * kVec;
     uint64_t g = (n + min_chunk - 1) / min_chunk;
     if (g > (uint64_t)max_ctas) g = (uint64_t)max_ctas;
     if (g < 1) g = 1;
     uint64_t ch = (n + g - 1) / g;
-    ch = (ch + kVec - 1) & ~(uint64_t)(kVec - 1);
+    ch = (ch + kChunkAlign - 1) & ~(kChunkAlign - 1);
     s.chunk = ch;
     s.grid = (unsigned)((n + ch - 1) / ch);
     return s;
 }
 
-int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st, unsigned smem = 0) {
+int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st, unsigned smem = 0,
+           int threads = kThreads) {
     void* args[] = {params};
-    const cudaError_t e = cudaLaunchKernel(fn, dim3(sh.grid), dim3(kThreads), args, smem, st);
+    const cudaError_t e = cudaLaunchKernel(fn, dim3(sh.grid), dim3(threads), args, smem, st);
     if (e != cudaSuccess) return zadam_record_cuda(e);
     return ZERO_OK;
 }
 
 // ------------------------------------------------------------ kernel tables
 
-// Flat calls with a compile-time rank count stage their tiles through shared
-// memory with bulk copies; other rank counts and lists use the register path.
-template <class G, class Pm, int RC>
+// Calls with a compile-time rank count stage their tiles through shared
+// memory with bulk copies; other rank counts use the register path.
+template <class G, class Pm, int RC, bool LIST>
 Kern bulk_kern() {
-    return Kern{(const void*)step_bulk_kernel<G, Pm, RC>, BulkShape<G, RC>::kSmem};
+    return Kern{(const void*)step_bulk_kernel<G, Pm, RC, LIST>, BulkShape<G, RC>::kSmem, kBulkThreads};
 }
 
-template <class G, class Pm>
-Kern step_kern_flat(uint32_t R) {
+template <class G, class Pm, bool LIST>
+Kern step_kern_rc(uint32_t R) {
 #ifndef ZADAM_REGISTER_PATH_ONLY
     switch (R) {
-        case 1: return bulk_kern<G, Pm, 1>();
-        case 2: return bulk_kern<G, Pm, 2>();
-        case 4: return bulk_kern<G, Pm, 4>();
-        case 8: return bulk_kern<G, Pm, 8>();
+        case 1: return bulk_kern<G, Pm, 1, LIST>();
+        case 2: return bulk_kern<G, Pm, 2, LIST>();
+        case 4: return bulk_kern<G, Pm, 4, LIST>();
+        case 8: return bulk_kern<G, Pm, 8, LIST>();
         default: break;
     }
 #endif
-    return Kern{(const void*)step_kernel<G, Pm, 0, false>, 0u};
+    return Kern{(const void*)step_kernel<G, Pm, 0, LIST>, 0u, kThreads};
 }
 
-template <class G>
-Kern step_kern_flat_pm(int32_t param_dtype, uint32_t R) {
-    return param_dtype == ZERO_BF16 ? step_kern_flat<G, __nv_bfloat16>(R) : step_kern_flat<G, __half>(R);
+template <class G, bool LIST>
+Kern step_kern_pm(int32_t param_dtype, uint32_t R) {
+    return param_dtype == ZERO_BF16 ? step_kern_rc<G, __nv_bfloat16, LIST>(R) : step_kern_rc<G, __half, LIST>(R);
 }
 
 Kern step_kern(bool list, int32_t grad_dtype, int32_t param_dtype, uint32_t R);
@@ -150,16 +154,21 @@ const void* step_fn(int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
     }
 }
 
-Kern step_kern(bool list, int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
-    if (list) return Kern{step_fn<true>(grad_dtype, param_dtype, R), 0u};
-#ifdef ZADAM_REGISTER_PATH_ONLY
-    return Kern{step_fn<false>(grad_dtype, param_dtype, R), 0u};
-#else
+template <bool LIST>
+Kern step_kern_gd(int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
     switch (grad_dtype) {
-        case ZERO_F32: return step_kern_flat_pm<float>(param_dtype, R);
-        case ZERO_BF16: return step_kern_flat_pm<__nv_bfloat16>(param_dtype, R);
-        default: return step_kern_flat_pm<__half>(param_dtype, R);
+        case ZERO_F32: return step_kern_pm<float, LIST>(param_dtype, R);
+        case ZERO_BF16: return step_kern_pm<__nv_bfloat16, LIST>(param_dtype, R);
+        default: return step_kern_pm<__half, LIST>(param_dtype, R);
     }
+}
+
+Kern step_kern(bool list, int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
+#ifdef ZADAM_REGISTER_PATH_ONLY
+    return Kern{list ? step_fn<true>(grad_dtype, param_dtype, R) : step_fn<false>(grad_dtype, param_dtype, R), 0u,
+                kThreads};
+#else
+    return list ? step_kern_gd<true>(grad_dtype, param_dtype, R) : step_kern_gd<false>(grad_dtype, param_dtype, R);
 #endif
 }
 
@@ -289,12 +298,12 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
         kp->check = check ? 1 : 0;
     }
     const Kern k = step_kern(LIST, a->grad_dtype, a->param_dtype, a->R);
-    const int ctas = resident_ctas(k.fn, &err, k.smem);
+    const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;
     const Shape sh = make_shape(lo, hi, ctas);
     kp->base = sh.base;
     kp->chunk = sh.chunk;
-    if ((err = launch(k.fn, sh, kp, st, k.smem))) return err;
+    if ((err = launch(k.fn, sh, kp, st, k.smem, k.threads))) return err;
     if (single_pass) {
         // Only if the step was skipped: re-cast the 16-bit parameters from
         // the master set that stayed current.

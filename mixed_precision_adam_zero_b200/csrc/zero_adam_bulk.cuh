@@ -1,6 +1,6 @@
-// zero_adam_bulk.cuh -- the flat step with shared-memory staging by 1-D bulk
-// asynchronous copies (the TMA engine's cp.async.bulk, no tensor map, no
-// multicast).
+// zero_adam_bulk.cuh -- the step (flat buffer or tensor list) with
+// shared-memory staging by 1-D bulk asynchronous copies (the TMA engine's
+// cp.async.bulk, no tensor map, no multicast).
 //
 // Why: the register-staged kernel holds each thread's loads in registers, so
 // the bytes a SM keeps in flight are bounded by registers x resident warps.
@@ -11,9 +11,11 @@
 //
 // Per tile of n <= kTile elements (n a multiple of 8, every source 16-byte
 // aligned): stage = [R gradient slices][w][m][v], each slice contiguous.
-// Thread t consumes two groups of 4 elements, [4t, 4t+4) and
-// [n/2 + 4t, n/2 + 4t + 4), so every shared-memory read is conflict-free and
-// every global store is coalesced.  The arithmetic per element is exactly
+// Thread t of the 512 consumes the 4 elements [4t, 4t+4), so every
+// shared-memory read is conflict-free and every global store is coalesced.
+// Sixteen consumer warps per SM keep the per-tile arithmetic (a float64
+// reduction, an IEEE divide and square root per element) well below the
+// tile's DRAM time; with eight the two were close and the kernel lost ~10 %.  The arithmetic per element is exactly
 // that of step_kernel (adam1 and the float64 rank reduction), so the two
 // kernels give bitwise identical results.
 //
@@ -26,9 +28,16 @@
 
 namespace zadam {
 
-constexpr int kTile = 2048;                     // elements per stage (256 threads x 8)
+#ifndef ZADAM_BULK_CONSUMERS
+#define ZADAM_BULK_CONSUMERS 256
+#endif
+constexpr int kConsumers = ZADAM_BULK_CONSUMERS;  // consumer threads per CTA
+constexpr int kBulkThreads = kConsumers + 32;     // plus one producer warp
+constexpr int kTile = 2048;                     // elements per stage
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-constexpr int kBarBytes = 128;                  // barrier block at the start of shared memory
+constexpr int kBarBytes = 384;                  // full and empty stage barriers (at most 2 x 8 x 8 B), padded
+constexpr int kGpBytes = 640;                   // gradient bases of a tensor (scalar pass of a list);
+                                                // pads the header so the stage ring starts 1024-B aligned
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -45,6 +54,10 @@ __device__ __forceinline__ void fence_mbar_init() {
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Global -> shared bulk copy completing on `bar` (16-byte aligned, size % 16 == 0).
@@ -127,17 +140,20 @@ struct BulkShape {
     static constexpr uint32_t kGradSlice = kTile * sizeof(G);
     static constexpr uint32_t kStage = RC * kGradSlice + 3u * kTile * 4u;
     static constexpr int kBudget = 200 * 1024;
-    static constexpr int kStages = (kBudget / kStage) > 6 ? 6 : (kBudget / kStage);
-    static constexpr uint32_t kSmem = kBarBytes + kStages * kStage;
+    static constexpr int kStages = (kBudget / kStage) > 8 ? 8 : (kBudget / kStage);
+    static constexpr uint32_t kSmem = kBarBytes + kGpBytes + kStages * kStage;
     static_assert(kStages >= 2, "stage too large for the ring");
+    static_assert((kBarBytes + kGpBytes) % 1024 == 0, "stage ring must start 1024-byte aligned");
+    static_assert(kStage % 1024 == 0, "stages must stay 1024-byte aligned");
 };
 
 // Four consecutive elements at flat index e (tile-relative offset q in the
-// stage), reduced, updated and stored.
+// stage, index le within the tensor's 16-bit parameters), reduced, updated
+// and stored.
 template <class G, class Pm, int RC>
 __device__ __forceinline__ void bulk_group(const StepParams& p, const Scal& s, const unsigned char* stage,
-                                           uint32_t q, uint64_t e, float* wo, float* mo, float* vo, Pm* pp,
-                                           bool& bad) {
+                                           uint32_t q, uint64_t e, uint64_t le, float* wo, float* mo, float* vo,
+                                           Pm* pp, bool& bad) {
     using Sh = BulkShape<G, RC>;
     Raw4<G> raw[RC];
 #pragma unroll
@@ -171,104 +187,314 @@ __device__ __forceinline__ void bulk_group(const StepParams& p, const Scal& s, c
     uint2 o;
     o.x = pack2<Pm>(w[0], w[1]);
     o.y = pack2<Pm>(w[2], w[3]);
-    __stcs(reinterpret_cast<uint2*>(pp + e), o);
+    __stcs(reinterpret_cast<uint2*>(pp + le), o);
     if (p.reduced != nullptr) __stcs(reinterpret_cast<float4*>(p.reduced + e), make_float4(g[0], g[1], g[2], g[3]));
 }
 
-// Issue the copies of tile k (flat elements [e0, e0+n)) into `stage`.
+// Issue the copies of one tile into `stage` (gradient bases already offset
+// to the tile's tensor; `le0` = tile start within the tensor).
 template <class G, int RC>
-__device__ __forceinline__ void bulk_issue(const StepParams& p, const StateIO& io, unsigned char* stage,
-                                           uint64_t* bar, uint64_t e0, uint32_t n) {
+__device__ __forceinline__ void bulk_issue(const StateIO& io, const G* const (&gb)[RC], unsigned char* stage,
+                                           uint64_t* bar, uint64_t e0, uint64_t le0, uint32_t n) {
     using Sh = BulkShape<G, RC>;
-    const uint32_t gb = n * (uint32_t)sizeof(G), sb = n * 4u;
-    mbar_expect_tx(bar, RC * gb + 3u * sb);
+    const uint32_t gbytes = n * (uint32_t)sizeof(G), sbytes = n * 4u;
+    mbar_expect_tx(bar, RC * gbytes + 3u * sbytes);
 #pragma unroll
-    for (int r = 0; r < RC; ++r)
-        bulk_g2s(stage + r * Sh::kGradSlice, static_cast<const G*>(p.grads[r]) + e0, gb, bar);
+    for (int r = 0; r < RC; ++r) bulk_g2s(stage + r * Sh::kGradSlice, gb[r] + le0, gbytes, bar);
     unsigned char* st = stage + RC * Sh::kGradSlice;
-    bulk_g2s(st, io.wi + e0, sb, bar);
-    bulk_g2s(st + kTile * 4u, io.mi + e0, sb, bar);
-    bulk_g2s(st + 2u * kTile * 4u, io.vi + e0, sb, bar);
+    bulk_g2s(st, io.wi + e0, sbytes, bar);
+    bulk_g2s(st + kTile * 4u, io.mi + e0, sbytes, bar);
+    bulk_g2s(st + 2u * kTile * 4u, io.vi + e0, sbytes, bar);
 }
 
+// The walk over a CTA's vector tiles.  Flat: one tensor [0, P).  List:
+// tensors in order; a tensor's vector body is its part of [a, b) rounded
+// inward to multiples of 8, and only tensors flagged for the vector path
+// have one.  Everything outside the bodies is left to the scalar pass, which
+// walks the same segments.  Every thread runs the walk in registers (the
+// tile sequence is a pure function of the range and the table); the issuing
+// thread runs a second copy D tiles ahead that also loads each tensor's
+// gradient bases.
+template <class G, int RC, bool LIST, bool GRADS>
+struct TileWalk {
+    uint64_t x, bb;  // next tile start and end of the current vector body
+    uint64_t segx;   // list: flat start of the next segment to examine
+    uint64_t b;      // end of the CTA's range
+    uint32_t j;      // list: next tensor to examine
+    const G* gb[GRADS ? RC : 1];
+    void* params;
+    uint64_t toff;
+
+    __device__ __forceinline__ void start(const StepParams& p, uint64_t a, uint64_t b_) {
+        b = b_;
+        toff = 0;
+        params = p.params16;
+        if constexpr (!LIST) {
+            x = (a + 7) & ~7ull;
+            bb = b & ~7ull;
+            if constexpr (GRADS) {
+#pragma unroll
+                for (int r = 0; r < RC; ++r) gb[r] = static_cast<const G*>(p.grads[r]);
+            }
+        } else {
+            x = bb = 0;
+            segx = a;
+            j = find_tensor(p.tab, a);
+        }
+    }
+
+    // List: move to the next segment that has a vector body; the table is
+    // read only here, once per tensor.
+    __device__ __forceinline__ bool next_body(const StepParams& p) {
+        while (segx < b) {
+            const uint64_t t0 = p.tab.offs[j], t1 = p.tab.offs[j + 1];
+            const uint64_t sb = t1 < b ? t1 : b;
+            const uint32_t jt = j++;
+            if (segx >= sb) continue;            // empty tensor
+            const uint64_t ba = (segx + 7) & ~7ull, be = sb & ~7ull;
+            segx = sb;
+            if ((p.tab.flags[jt] & 1u) == 0u || ba >= be) continue;  // scalar pass only
+            x = ba;
+            bb = be;
+            toff = t0;
+            params = p.tab.params[jt];
+            if constexpr (GRADS) {
+#pragma unroll
+                for (int r = 0; r < RC; ++r) gb[r] = static_cast<const G*>(p.tab.grads[(uint64_t)jt * RC + r]);
+            }
+            return true;
+        }
+        return false;
+    }
+
+    // Next tile: flat start e0 and length n (a multiple of 8); false at the end.
+    __device__ __forceinline__ bool next(const StepParams& p, uint64_t& e0, uint32_t& n) {
+        if (x >= bb) {
+            if constexpr (!LIST) return false;
+            else if (!next_body(p)) return false;
+        }
+        e0 = x;
+        n = (uint32_t)((bb - x) < (uint64_t)kTile ? (bb - x) : (uint64_t)kTile);
+        x += n;
+        return true;
+    }
+};
+
+// Scalar pass over everything the tile walk leaves out.
+template <class G, class Pm, int RC, bool LIST>
+__device__ __forceinline__ void bulk_scalar_pass(const StepParams& p, const Scal& s, uint64_t a, uint64_t b,
+                                                 const StateIO& io, bool& bad, const void** s_gp) {
+    if constexpr (!LIST) {
+        const GradPtrs<G, RC> gp(&p.grads[0]);
+        Pm* pp = static_cast<Pm*>(p.params16);
+        uint64_t va = (a + 7) & ~7ull, vb = b & ~7ull;
+        if (va > b) va = b;
+        if (vb < va) vb = va;
+        for (uint64_t e = a + threadIdx.x; e < va; e += kBulkThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e, io, bad);
+        for (uint64_t e = vb + threadIdx.x; e < b; e += kBulkThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e, io, bad);
+    } else {
+        uint32_t j = find_tensor(p.tab, a);
+        uint64_t x = a;
+        while (x < b) {
+            const uint64_t t0 = p.tab.offs[j], t1 = p.tab.offs[j + 1];
+            const uint64_t sb = t1 < b ? t1 : b;
+            if (x < sb) {
+                const bool vec = (p.tab.flags[j] & 1u) != 0u;
+                uint64_t ba = sb, bb = sb;
+                if (vec) {
+                    ba = (x + 7) & ~7ull;
+                    bb = sb & ~7ull;
+                    if (ba > sb) ba = sb;
+                    if (bb < ba) bb = ba;
+                }
+                if (ba > x || bb < sb) {
+                    __syncthreads();
+                    for (uint32_t r = threadIdx.x; r < RC; r += kBulkThreads) s_gp[r] = p.tab.grads[(uint64_t)j * RC + r];
+                    __syncthreads();
+                    const GradPtrs<G, RC> gp(s_gp);
+                    Pm* pp = static_cast<Pm*>(p.tab.params[j]);
+                    for (uint64_t e = x + threadIdx.x; e < ba; e += kBulkThreads)
+                        elem_step<G, Pm, RC>(p, s, gp, pp, e, e - t0, io, bad);
+                    for (uint64_t e = bb + threadIdx.x; e < sb; e += kBulkThreads)
+                        elem_step<G, Pm, RC>(p, s, gp, pp, e, e - t0, io, bad);
+                }
+            }
+            x = sb;
+            ++j;
+        }
+    }
+}
+
+
+// Input and output state arrays of this step (set ctrl.parity in two-set mode).
+__device__ __forceinline__ StateIO state_io(const StepParams& p) {
+    const uint32_t par = p.two_set ? p.ctrl->parity : 0u;
+    const uint32_t out = par ^ (uint32_t)p.two_set;
+    return StateIO{p.w[par], p.m[par], p.v[par], p.w[out], p.m[out], p.v[out]};
+}
+
+// Flat call: tiles are handed out dynamically.  The launch's vector body
+// [round_up(lo, 8), round_down(hi, 8)) is cut into kTile-element tiles, and
+// each CTA's producer claims the next one from a counter in the workspace,
+// one claim ahead of use so the atomic's latency overlaps the copies.  All
+// CTAs then finish within about one tile of each other, whatever the speed
+// of their SM.  The tile id travels to the consumers in a per-stage slot,
+// written before the stage's barrier is armed; kEndTile marks the end.
+constexpr uint32_t kEndTile = 0xFFFFFFFFu;
+
 template <class G, class Pm, int RC>
-__global__ void __launch_bounds__(kThreads, 1) step_bulk_kernel(const __grid_constant__ StepParams p) {
+__device__ __forceinline__ void flat_dynamic(const StepParams& p, uint64_t* full, uint64_t* empty,
+                                             uint32_t* slot, unsigned char* ring, bool& bad) {
     using Sh = BulkShape<G, RC>;
     constexpr int D = Sh::kStages;
-    extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    unsigned char* ring = smem + kBarBytes;
+    const uint64_t va = (p.lo + 7) & ~7ull;
+    const uint64_t vb = p.hi & ~7ull;
+    const uint32_t ntiles = va < vb ? (uint32_t)((vb - va + kTile - 1) / kTile) : 0u;
+    if (threadIdx.x == kConsumers) {
+        const StateIO io = state_io(p);
+        const G* gb[RC];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) gb[r] = static_cast<const G*>(p.grads[r]);
+        uint32_t next = atomicAdd(&p.ws->next_tile, 1u);
+        uint32_t k = 0;
+        bool ok = true;
+        for (;; ++k) {
+            const int st = (int)(k % D);
+            if (k >= (uint32_t)D && !mbar_wait_bounded(&empty[st], ((k / D) - 1u) & 1u)) {
+                ok = false;
+                break;
+            }
+            const uint32_t tile = next;
+            if (tile >= ntiles) {
+                slot[st] = kEndTile;
+                mbar_arrive(&full[st]);
+                break;
+            }
+            next = atomicAdd(&p.ws->next_tile, 1u);
+            slot[st] = tile;
+            const uint64_t e0 = va + (uint64_t)tile * kTile;
+            const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
+            bulk_issue<G, RC>(io, gb, ring + st * Sh::kStage, &full[st], e0, e0, n);
+        }
+        if (!ok) {
+            atomicOr(&p.ws->error, 1u);
+            for (uint32_t j = k > (uint32_t)D ? k - D : 0u; j < k; ++j)
+                (void)mbar_wait_bounded(&full[j % D], (j / D) & 1u);
+        }
+    } else if (threadIdx.x < kConsumers) {
+        const StateIO io = state_io(p);
+        const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
+        Pm* pp = static_cast<Pm*>(p.params16);
+        for (uint32_t k = 0;; ++k) {
+            const int st = (int)(k % D);
+            if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
+                atomicOr(&p.ws->error, 1u);
+                break;
+            }
+            const uint32_t tile = slot[st];
+            if (tile == kEndTile) break;
+            const uint64_t e0 = va + (uint64_t)tile * kTile;
+            const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
+            const unsigned char* stage = ring + st * Sh::kStage;
+            for (uint32_t q = 4u * threadIdx.x; q < n; q += 4u * kConsumers)
+                bulk_group<G, Pm, RC>(p, s, stage, q, e0 + q, e0 + q, io.wo, io.mo, io.vo, pp, bad);
+            __syncwarp();
+            if ((threadIdx.x & 31u) == 0u) mbar_arrive(&empty[st]);
+        }
+    }
+}
 
-    const zero_ctrl* c = p.ctrl;
-    const uint32_t par = p.two_set ? c->parity : 0u;
-    const uint32_t out = par ^ (uint32_t)p.two_set;
-    const StateIO io{p.w[par], p.m[par], p.v[par], p.w[out], p.m[out], p.v[out]};
-    bool skip = false;
-    if (p.check == 2) skip = *reinterpret_cast<volatile const unsigned*>(&p.ws->found) != 0u;
-    const Scal s = make_scal(p.h, c->step + 1ull, c->loss_scale, p.wsum);
+// List call: each CTA walks its own contiguous range of the concatenation.
+template <class G, class Pm, int RC>
+__device__ __forceinline__ void list_static(const StepParams& p, uint64_t a, uint64_t b, uint64_t* full,
+                                            uint64_t* empty, unsigned char* ring, bool& bad) {
+    using Sh = BulkShape<G, RC>;
+    constexpr int D = Sh::kStages;
+    if (threadIdx.x == kConsumers) {
+        const StateIO io = state_io(p);
+        TileWalk<G, RC, true, true> pw;
+        pw.start(p, a, b);
+        uint64_t e0;
+        uint32_t n;
+        uint32_t k = 0;
+        bool ok = true;
+        for (; pw.next(p, e0, n); ++k) {
+            const int st = (int)(k % D);
+            if (k >= (uint32_t)D && !mbar_wait_bounded(&empty[st], ((k / D) - 1u) & 1u)) {
+                ok = false;
+                break;
+            }
+            bulk_issue<G, RC>(io, pw.gb, ring + st * Sh::kStage, &full[st], e0, e0 - pw.toff, n);
+        }
+        if (!ok) {
+            // Do not leave while copies of this CTA may still land in its
+            // shared memory: wait (bounded) for the last tile of every stage.
+            atomicOr(&p.ws->error, 1u);
+            for (uint32_t j = k > (uint32_t)D ? k - D : 0u; j < k; ++j)
+                (void)mbar_wait_bounded(&full[j % D], (j / D) & 1u);
+        }
+    } else if (threadIdx.x < kConsumers) {
+        const StateIO io = state_io(p);
+        const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
+        TileWalk<G, RC, true, false> cw;
+        cw.start(p, a, b);
+        uint64_t e0;
+        uint32_t n;
+        for (uint32_t k = 0; cw.next(p, e0, n); ++k) {
+            const int st = (int)(k % D);
+            if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
+                atomicOr(&p.ws->error, 1u);
+                break;
+            }
+            const unsigned char* stage = ring + st * Sh::kStage;
+            Pm* pp = static_cast<Pm*>(cw.params);
+            const uint64_t le0 = e0 - cw.toff;
+            for (uint32_t q = 4u * threadIdx.x; q < n; q += 4u * kConsumers)
+                bulk_group<G, Pm, RC>(p, s, stage, q, e0 + q, le0 + q, io.wo, io.mo, io.vo, pp, bad);
+            __syncwarp();
+            if ((threadIdx.x & 31u) == 0u) mbar_arrive(&empty[st]);
+        }
+    }
+}
+
+template <class G, class Pm, int RC, bool LIST>
+__global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid_constant__ StepParams p) {
+    using Sh = BulkShape<G, RC>;
+    constexpr int D = Sh::kStages;
+    constexpr uint32_t kConsumerWarps = kConsumers / 32;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);        // data of stage s has landed
+    uint64_t* empty = reinterpret_cast<uint64_t*>(smem + 64);  // every consumer warp is done with stage s
+    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + 128);  // flat: tile id of stage s
+    const void** s_gp = reinterpret_cast<const void**>(smem + kBarBytes);
+    unsigned char* ring = smem + kBarBytes + kGpBytes;
 
     uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
     uint64_t b = a + p.chunk;
     if (a < p.lo) a = p.lo;
     if (b > p.hi) b = p.hi;
+    bool skip = false;
+    if (p.check == 2) skip = *reinterpret_cast<volatile const unsigned*>(&p.ws->found) != 0u;
     bool bad = false;
-    bool failed = false;
-    if (!skip && a < b) {
-        const GradPtrs<G, RC> gp(&p.grads[0]);
-        Pm* pp = static_cast<Pm*>(p.params16);
-        // ragged head and tail: the register path, same arithmetic
-        uint64_t va = (a + 7) & ~7ull, vb = b & ~7ull;
-        if (va > b) va = b;
-        if (vb < va) vb = va;
-        for (uint64_t e = a + threadIdx.x; e < va; e += kThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e, io, bad);
-        for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e, io, bad);
-
-        const uint64_t nt = (vb - va + kTile - 1) / kTile;
+    const bool work = LIST ? a < b : p.lo < p.hi;
+    if (!skip && work) {
         if (threadIdx.x == 0) {
-            for (int i = 0; i < D; ++i) mbar_init(&bars[i], 1u);
+            for (int i = 0; i < D; ++i) {
+                mbar_init(&full[i], 1u);
+                mbar_init(&empty[i], kConsumerWarps);
+            }
             fence_mbar_init();
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
-            for (uint64_t k = 0; k < nt && k < (uint64_t)D; ++k) {
-                const uint64_t e0 = va + k * kTile;
-                const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
-                bulk_issue<G, RC>(p, io, ring + k * Sh::kStage, &bars[k], e0, n);
-            }
-        }
-        uint64_t k = 0;
-        for (; k < nt; ++k) {
-            const int st = (int)(k % D);
-            const uint32_t phase = (uint32_t)((k / D) & 1u);
-            const bool ok = mbar_wait_bounded(&bars[st], phase);
-            const uint64_t e0 = va + k * kTile;
-            const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
-            const uint32_t half = n >> 1;  // a multiple of 4
-            const uint32_t q = 4u * threadIdx.x;
-            if (ok && q < half) {
-                const unsigned char* stage = ring + st * Sh::kStage;
-                bulk_group<G, Pm, RC>(p, s, stage, q, e0 + q, io.wo, io.mo, io.vo, pp, bad);
-                bulk_group<G, Pm, RC>(p, s, stage, half + q, e0 + half + q, io.wo, io.mo, io.vo, pp, bad);
-            }
-            if (!__syncthreads_and(ok ? 1 : 0)) {
-                failed = true;
-                break;
-            }
-            if (threadIdx.x == 0 && k + D < nt) {
-                const uint64_t e1 = va + (k + D) * kTile;
-                const uint32_t n1 = (uint32_t)((vb - e1) < (uint64_t)kTile ? (vb - e1) : (uint64_t)kTile);
-                bulk_issue<G, RC>(p, io, ring + st * Sh::kStage, &bars[st], e1, n1);
-            }
-        }
-        if (failed && threadIdx.x == 0) {
-            // Do not leave while copies this CTA issued may still land in its
-            // shared memory: wait (bounded) for every issued, unconsumed tile.
-            atomicOr(&p.ws->error, 1u);
-            const uint64_t issued = nt < k + D ? nt : k + D;
-            for (uint64_t j = k; j < issued; ++j)
-                (void)mbar_wait_bounded(&bars[j % D], (uint32_t)((j / D) & 1u));
-        }
+        if constexpr (LIST) list_static<G, Pm, RC>(p, a, b, full, empty, ring, bad);
+        else flat_dynamic<G, Pm, RC>(p, full, empty, slot, ring, bad);
         __syncthreads();
+        // Ragged heads and tails, and tensors that cannot take the vector path
+        // (flat: the launch's ragged ends, on the first CTA only).
+        const StateIO io = state_io(p);
+        const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
+        if constexpr (LIST) bulk_scalar_pass<G, Pm, RC, true>(p, s, a, b, io, bad, s_gp);
+        else if (blockIdx.x == 0) bulk_scalar_pass<G, Pm, RC, false>(p, s, p.lo, p.hi, io, bad, s_gp);
     }
     finish_step(p, bad);
 }

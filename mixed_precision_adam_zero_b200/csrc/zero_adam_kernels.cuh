@@ -41,10 +41,11 @@ constexpr int kVec = 8;        // elements per vector
 
 // Scratch of one step call (ZERO_WORKSPACE_BYTES).  All zero between calls.
 struct Workspace {
-    unsigned int arrive;  // CTAs of the running launch that have finished
-    unsigned int found;   // nonzero: some gradient was inf or NaN
-    unsigned int error;   // nonzero: a bounded device-side wait gave up
-    unsigned int pad[61];
+    unsigned int arrive;     // CTAs of the running launch that have finished
+    unsigned int found;      // nonzero: some gradient was inf or NaN
+    unsigned int error;      // nonzero: a bounded device-side wait gave up
+    unsigned int next_tile;  // flat bulk step: the next tile to hand out
+    unsigned int pad[60];
 };
 static_assert(sizeof(Workspace) == ZERO_WORKSPACE_BYTES, "workspace size");
 
@@ -432,6 +433,7 @@ __device__ __forceinline__ void finish_step(const StepParams& p, bool bad) {
             if (err) c->device_error = err;
             ws->found = 0u;
             ws->error = 0u;
+            ws->next_tile = 0u;
             ws->arrive = 0u;
             __threadfence();
         }
