@@ -330,7 +330,7 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
 
 // Host copy of a list's table layout: byte offsets of each array.
 struct TableLayout {
-    size_t offs, params, grads, flags, total;
+    size_t offs, params, grads, flags, tiles, total;
 };
 
 TableLayout table_layout(uint32_t T, uint32_t R) {
@@ -339,7 +339,8 @@ TableLayout table_layout(uint32_t T, uint32_t R) {
     L.params = L.offs + 8ull * ((size_t)T + 1);
     L.grads = L.params + 8ull * T;
     L.flags = L.grads + 8ull * (size_t)T * R;
-    L.total = L.flags + ((4ull * T + 15) & ~15ull);
+    L.tiles = L.flags + ((4ull * T + 15) & ~15ull);
+    L.total = L.tiles + 8ull * ((size_t)T + 1);
     return L;
 }
 
@@ -351,6 +352,7 @@ Table device_table(const zero_tensor_list* l) {
     t.params = reinterpret_cast<void* const*>(base + L.params);
     t.grads = reinterpret_cast<const void* const*>(base + L.grads);
     t.flags = reinterpret_cast<const uint32_t*>(base + L.flags);
+    t.tiles = reinterpret_cast<const uint64_t*>(base + L.tiles);
     t.T = l->T;
     return t;
 }
@@ -462,6 +464,7 @@ int zero_step_fused_list(const zero_step_args* a, const zero_tensor_list* l, voi
     if (a->P != l->P || a->R != l->R || a->grad_dtype != l->grad_dtype || a->param_dtype != l->param_dtype)
         return ZERO_EINVAL;
     kp.tab = device_table(l);
+    kp.whole = a->owner < 0 ? 1 : 0;
     return run_step<true>(a, &kp, static_cast<cudaStream_t>(stream));
 }
 
@@ -495,6 +498,7 @@ int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t* numel, void* c
     void** prm = reinterpret_cast<void**>(buf.data() + L.params);
     const void** grd = reinterpret_cast<const void**>(buf.data() + L.grads);
     uint32_t* flags = reinterpret_cast<uint32_t*>(buf.data() + L.flags);
+    uint64_t* tiles = reinterpret_cast<uint64_t*>(buf.data() + L.tiles);
     uint64_t P = 0;
     for (uint32_t j = 0; j < T; ++j) {
         offs[j] = P;
@@ -513,6 +517,14 @@ int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t* numel, void* c
         flags[j] = vec_ok ? 1u : 0u;
     }
     offs[T] = P;
+    // Vector tiles of each tensor's body [offs[j], round_down(offs[j+1], 8)),
+    // as running counts (used when a step covers the whole vector).
+    tiles[0] = 0;
+    for (uint32_t j = 0; j < T; ++j) {
+        const uint64_t body_end = offs[j + 1] & ~7ull;
+        const uint64_t nt = (flags[j] && body_end > offs[j]) ? (body_end - offs[j] + kTile - 1) / kTile : 0;
+        tiles[j + 1] = tiles[j] + nt;
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemcpyAsync(table, buf.data(), L.total, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);

@@ -404,6 +404,124 @@ __device__ __forceinline__ void flat_dynamic(const StepParams& p, uint64_t* full
     }
 }
 
+// Tile descriptor handed from the producer to the consumers through shared
+// memory (list calls): written before the stage's barrier is armed.
+struct TileDesc {
+    uint64_t e0;    // flat index of the tile's first element
+    uint64_t toff;  // flat index of the tensor's first element
+    void* params;   // the tensor's 16-bit parameters
+    uint32_t n;     // elements (a multiple of 8); 0: no more tiles
+    uint32_t pad;
+};
+
+// List call over the whole vector: the vector body of tensor j (if it may
+// take the vector path) is [offs[j], round_down(offs[j+1], 8)); the bodies
+// are cut into kTile tiles, numbered across tensors (tab.tiles holds the
+// running count), and handed out dynamically like the flat call's tiles.
+// Tile ids a producer claims only grow, so it finds each tile's tensor by
+// scanning forward from the previous one.
+template <class G, class Pm, int RC>
+__device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full, uint64_t* empty,
+                                             TileDesc* desc, unsigned char* ring, bool& bad) {
+    using Sh = BulkShape<G, RC>;
+    constexpr int D = Sh::kStages;
+    const Table& t = p.tab;
+    const uint64_t ntiles = t.tiles[t.T];
+    if (threadIdx.x == kConsumers) {
+        const StateIO io = state_io(p);
+        const G* gb[RC];
+        uint32_t j = 0xFFFFFFFFu;  // tensor whose pointers are loaded
+        uint32_t jn = 0;           // scan position
+        uint64_t t0 = 0, bb = 0, tfirst = 0;
+        void* params = nullptr;
+        uint64_t next = atomicAdd(&p.ws->next_tile, 1u);
+        if (next < ntiles) jn = find_tensor_by_tile(t, next);
+        uint32_t k = 0;
+        bool ok = true;
+        for (;; ++k) {
+            const int st = (int)(k % D);
+            if (k >= (uint32_t)D && !mbar_wait_bounded(&empty[st], ((k / D) - 1u) & 1u)) {
+                ok = false;
+                break;
+            }
+            const uint64_t tile = next;
+            if (tile >= ntiles) {
+                desc[st] = TileDesc{0ull, 0ull, nullptr, 0u, 0u};
+                mbar_arrive(&full[st]);
+                break;
+            }
+            next = atomicAdd(&p.ws->next_tile, 1u);
+            while (t.tiles[jn + 1] <= tile) ++jn;
+            if (jn != j) {
+                j = jn;
+#pragma unroll
+                for (int r = 0; r < RC; ++r) gb[r] = static_cast<const G*>(t.grads[(uint64_t)j * RC + r]);
+                params = t.params[j];
+                t0 = t.offs[j];
+                bb = t.offs[j + 1] & ~7ull;
+                tfirst = t.tiles[j];
+            }
+            const uint64_t e0 = t0 + (tile - tfirst) * kTile;
+            const uint32_t n = (uint32_t)((bb - e0) < (uint64_t)kTile ? (bb - e0) : (uint64_t)kTile);
+            desc[st] = TileDesc{e0, t0, params, n, 0u};
+            bulk_issue<G, RC>(io, gb, ring + st * Sh::kStage, &full[st], e0, e0 - t0, n);
+        }
+        if (!ok) {
+            atomicOr(&p.ws->error, 1u);
+            for (uint32_t i = k > (uint32_t)D ? k - D : 0u; i < k; ++i)
+                (void)mbar_wait_bounded(&full[i % D], (i / D) & 1u);
+        }
+    } else if (threadIdx.x < kConsumers) {
+        const StateIO io = state_io(p);
+        const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
+        for (uint32_t k = 0;; ++k) {
+            const int st = (int)(k % D);
+            if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
+                atomicOr(&p.ws->error, 1u);
+                break;
+            }
+            const TileDesc d = desc[st];
+            if (d.n == 0u) break;
+            const unsigned char* stage = ring + st * Sh::kStage;
+            Pm* pp = static_cast<Pm*>(d.params);
+            const uint64_t le0 = d.e0 - d.toff;
+            for (uint32_t q = 4u * threadIdx.x; q < d.n; q += 4u * kConsumers)
+                bulk_group<G, Pm, RC>(p, s, stage, q, d.e0 + q, le0 + q, io.wo, io.mo, io.vo, pp, bad);
+            __syncwarp();
+            if ((threadIdx.x & 31u) == 0u) mbar_arrive(&empty[st]);
+        }
+    }
+}
+
+// Scalar part of [a, b) for list_dynamic: everything outside the tensors'
+// vector bodies.
+template <class G, class Pm, int RC>
+__device__ __forceinline__ void list_scalar_whole(const StepParams& p, const Scal& s, uint64_t a, uint64_t b,
+                                                  const StateIO& io, bool& bad, const void** s_gp) {
+    uint32_t j = find_tensor(p.tab, a);
+    uint64_t x = a;
+    while (x < b) {
+        const uint64_t t0 = p.tab.offs[j], t1 = p.tab.offs[j + 1];
+        const uint64_t sb = t1 < b ? t1 : b;
+        if (x < sb) {
+            const bool vec = (p.tab.flags[j] & 1u) != 0u;
+            const uint64_t be = vec ? (t1 & ~7ull) : t0;  // body [t0, be)
+            const uint64_t from = be > x ? be : x;
+            if (from < sb) {
+                __syncthreads();
+                for (uint32_t r = threadIdx.x; r < RC; r += kBulkThreads) s_gp[r] = p.tab.grads[(uint64_t)j * RC + r];
+                __syncthreads();
+                const GradPtrs<G, RC> gp(s_gp);
+                Pm* pp = static_cast<Pm*>(p.tab.params[j]);
+                for (uint64_t e = from + threadIdx.x; e < sb; e += kBulkThreads)
+                    elem_step<G, Pm, RC>(p, s, gp, pp, e, e - t0, io, bad);
+            }
+        }
+        x = sb;
+        ++j;
+    }
+}
+
 // List call: each CTA walks its own contiguous range of the concatenation.
 template <class G, class Pm, int RC>
 __device__ __forceinline__ void list_static(const StepParams& p, uint64_t a, uint64_t b, uint64_t* full,
@@ -465,7 +583,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);        // data of stage s has landed
     uint64_t* empty = reinterpret_cast<uint64_t*>(smem + 64);  // every consumer warp is done with stage s
-    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + 128);  // flat: tile id of stage s
+    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + 128);  // tile id (flat) or TileDesc (list) of stage s
     const void** s_gp = reinterpret_cast<const void**>(smem + kBarBytes);
     unsigned char* ring = smem + kBarBytes + kGpBytes;
 
@@ -476,7 +594,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
     bool skip = false;
     if (p.check == 2) skip = *reinterpret_cast<volatile const unsigned*>(&p.ws->found) != 0u;
     bool bad = false;
-    const bool work = LIST ? a < b : p.lo < p.hi;
+    const bool work = (LIST && !p.whole) ? a < b : p.lo < p.hi;
     if (!skip && work) {
         if (threadIdx.x == 0) {
             for (int i = 0; i < D; ++i) {
@@ -486,15 +604,26 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
             fence_mbar_init();
         }
         __syncthreads();
-        if constexpr (LIST) list_static<G, Pm, RC>(p, a, b, full, empty, ring, bad);
-        else flat_dynamic<G, Pm, RC>(p, full, empty, slot, ring, bad);
+        if constexpr (LIST) {
+            if (p.whole) list_dynamic<G, Pm, RC>(p, full, empty, reinterpret_cast<TileDesc*>(slot), ring, bad);
+            else list_static<G, Pm, RC>(p, a, b, full, empty, ring, bad);
+        } else {
+            flat_dynamic<G, Pm, RC>(p, full, empty, slot, ring, bad);
+        }
         __syncthreads();
         // Ragged heads and tails, and tensors that cannot take the vector path
         // (flat: the launch's ragged ends, on the first CTA only).
         const StateIO io = state_io(p);
         const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
-        if constexpr (LIST) bulk_scalar_pass<G, Pm, RC, true>(p, s, a, b, io, bad, s_gp);
-        else if (blockIdx.x == 0) bulk_scalar_pass<G, Pm, RC, false>(p, s, p.lo, p.hi, io, bad, s_gp);
+        if constexpr (LIST) {
+            if (p.whole) {
+                if (a < b) list_scalar_whole<G, Pm, RC>(p, s, a, b, io, bad, s_gp);
+            } else {
+                if (a < b) bulk_scalar_pass<G, Pm, RC, true>(p, s, a, b, io, bad, s_gp);
+            }
+        } else if (blockIdx.x == 0) {
+            bulk_scalar_pass<G, Pm, RC, false>(p, s, p.lo, p.hi, io, bad, s_gp);
+        }
     }
     finish_step(p, bad);
 }

@@ -60,6 +60,7 @@ struct Table {
     void* const* params;        // [T] 16-bit parameter tensors
     const void* const* grads;   // [T*R] gradients, tensor-major: grads[j*R + r]
     const uint32_t* flags;      // [T] bit 0: vector path allowed
+    const uint64_t* tiles;      // [T+1] vector tiles of tensors 0..j-1 (whole-vector calls)
     uint32_t T;
 };
 
@@ -82,6 +83,7 @@ struct StepParams {
     uint32_t growth_interval;
     int32_t two_set;  // 1: read set ctrl.parity, write the other set
     int32_t check;    // 0: none; 1: detect inf/NaN in this pass; 2: a scan decided
+    int32_t whole;    // 1: the launch covers every owner's slice ([0, P))
 };
 
 struct GatherParams {
@@ -395,6 +397,16 @@ __device__ __forceinline__ uint32_t find_tensor(const Table& t, uint64_t x) {
     while (hi - lo > 1) {
         const uint32_t mid = (lo + hi) >> 1;
         if (t.offs[mid] <= x) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+// Index of the tensor holding vector tile `tile` (tiles[j] <= tile < tiles[j+1]).
+__device__ __forceinline__ uint32_t find_tensor_by_tile(const Table& t, uint64_t tile) {
+    uint32_t lo = 0, hi = t.T;
+    while (hi - lo > 1) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (t.tiles[mid] <= tile) lo = mid; else hi = mid;
     }
     return lo;
 }

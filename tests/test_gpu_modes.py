@@ -56,6 +56,49 @@ def test_per_owner_calls_equal_one_all_owner_call_bitwise(P, R):
         assert za.zero_ctrl_read(c).step == 3
 
 
+@pytest.mark.parametrize("misalign", [False, True])
+def test_list_per_owner_calls_equal_one_whole_call_bitwise(misalign):
+    """The same comparison for a tensor list: the whole-vector call hands out
+    tiles dynamically, per-owner calls walk their slice statically; both must
+    give bitwise the same state."""
+    numels = [1000, 37, 4096 * 3 + 5, 0, 2048, 9, 50_000]
+    R = 4
+    def make():
+        if not misalign:
+            return ListZero(numels, R, "bf16", "bf16")
+        def carve(dtype):
+            buf = torch.zeros(sum(numels) + 3 * len(numels) + 8, dtype=dtype, device="cuda")
+            out, off = [], 1
+            for n in numels:
+                out.append(buf[off:off + n])
+                off += n + 3
+            return out
+        return ListZero(numels, R, "bf16", "bf16", params16=carve(torch.bfloat16),
+                        grads=[carve(torch.bfloat16) for _ in range(R)])
+    whole, shard = make(), make()
+    P = whole.P
+    w0 = synth.normal(P, 0.02, 15, device="cuda")
+    whole.load_master(w0)
+    shard.load_master(w0)
+    ctrls = [torch.zeros(64, dtype=torch.uint8, device="cuda") for _ in range(R)]
+    for c in ctrls:
+        za.zero_ctrl_init(c, 1.0)
+    for k in range(1, 3):
+        grads_for_step(15, k, whole.grads, 1e-3)
+        for r in range(R):
+            for j in range(len(numels)):
+                shard.grads[r][j].copy_(whole.grads[r][j])
+        whole.step(hp=ADAMW_HP)
+        for r in range(R):
+            a = shard.step_args(hp=ADAMW_HP, owner=r)
+            a.ctrl = ctrls[r].data_ptr()
+            za.zero_step_fused_list(a, shard.list)
+    torch.cuda.synchronize()
+    for x, y in zip(whole.current(), shard.current()):
+        assert torch.equal(x, y)
+    assert torch.equal(whole.flat_params16(), shard.flat_params16())
+
+
 # ------------------------------------------------------------ fp16 skip
 
 def _run_fp16(two_set, P=60_013, R=4, steps=9, bad_steps=(3, 7), bad=math.inf, growth_interval=0,
