@@ -294,7 +294,8 @@ def run_gpu(args) -> None:
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
                 "traffic": traffic,
-                "kernel": "step_kernel (flat)" if kind == "flat" else "step_kernel (list)",
+                "kernel": ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") +
+                          (" (flat)" if kind == "flat" else " (list)"),
                 "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms,
             },
             "e2e": {
