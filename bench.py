@@ -177,6 +177,31 @@ def launches_per_step(z) -> int:
     return 2  # two-set single pass + the restore kernel (a no-op unless skipped)
 
 
+# ------------------------------------------------------------ ranks
+
+def rank_env():
+    """(world, rank, local rank) from the launcher's environment."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(values, world: int, device):
+    """Element-wise maximum of per-rank timings (float64) over all ranks."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(world: int, units_per_rank: int, steps: int, max_ms: float) -> float:
+    """Whole-job units per second: every rank runs a replica of the workload,
+    so the job processes world * units_per_rank per step, in the slowest
+    rank's time."""
+    return world * units_per_rank * steps / (max_ms * 1e-3)
+
+
 # ------------------------------------------------------------ arms
 
 def run_gpu(args) -> None:
@@ -184,9 +209,7 @@ def run_gpu(args) -> None:
     import torch.distributed as dist
     from datetime import timedelta
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
     if world > 1:
@@ -251,10 +274,7 @@ def run_gpu(args) -> None:
     barrier()
     e2e_ms = e0.elapsed_time(e1)
 
-    times = torch.tensor([total_ms, per_launch_ms, e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, per_launch_ms, e2e_ms = times.tolist()
+    total_ms, per_launch_ms, e2e_ms = max_over_ranks([total_ms, per_launch_ms, e2e_ms], world, device)
     ctrl = z.ctrl()
 
     if rank == 0:
@@ -270,7 +290,7 @@ def run_gpu(args) -> None:
         traffic = traffic_for(args.workload)
         line = {
             "metric": METRIC,
-            "value": world * P * K / (total_ms * 1e-3),
+            "value": job_throughput(world, P, K, total_ms),
             "unit": UNIT,
             "n_gpus": world,
             "steps": K,
@@ -299,7 +319,7 @@ def run_gpu(args) -> None:
                 "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms,
             },
             "e2e": {
-                "value": world * P * K_e2e / (e2e_ms * 1e-3), "unit": UNIT, "steps": K_e2e,
+                "value": job_throughput(world, P, K_e2e, e2e_ms), "unit": UNIT, "steps": K_e2e,
                 "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": p16.numel() * p16.element_size(),
             } if K_e2e else None,
@@ -354,7 +374,7 @@ def cpu_baseline(workload: str, seconds: float) -> dict:
 def run_reference(args) -> None:
     """Reference arm: the float64 CPU oracle on the same workload, each step a
     bounded sample of it; rank 0 alone runs it under torchrun."""
-    if int(os.environ.get("RANK", "0")) != 0:
+    if rank_env()[1] != 0:
         return
     import oracle
     n = 1 << 20
