@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
         L.zo_step_sharded.argtypes = [u64, u64, u64p, u32, i32, pp, dp, i32, ctypes.POINTER(Hparams),
                                       ctypes.POINTER(Ctrl), dp, dp, dp, u64p, u64p]
         L.zo_reduced_grads.argtypes = [u64, u32, i32, pp, dp, ctypes.c_double, dp]
+        L.zo_accumulate.argtypes = [u64, u32, i32, pp, dp, ctypes.c_double, i32,
+                                    ctypes.POINTER(ctypes.c_float)]
         L.zo_max_threads.restype = ctypes.c_int
         _lib_handle = L
     return _lib_handle
@@ -331,3 +333,20 @@ def any_nonfinite(grads: Sequence[np.ndarray], gdtype: str) -> bool:
 def cast_params(w: np.ndarray, dtype: str) -> np.ndarray:
     """16-bit parameters (uint16 bit patterns) of the float64 masters."""
     return rne16(w, dtype)
+
+
+def accumulate(acc: np.ndarray, grads: Sequence[np.ndarray], gdtype: str, scale: float,
+               first: bool, weights: Optional[Sequence[float]] = None) -> np.ndarray:
+    """Micro-step accumulation into a float32 array, in place:
+    acc = (first ? 0 : acc) + scale * reduced gradient, rounded once to float32."""
+    if acc.dtype != np.float32 or not acc.flags.c_contiguous:
+        raise ValueError("acc must be a contiguous float32 array")
+    n = acc.size
+    keep, arr = _grad_ptrs(grads, gdtype, n)
+    wts = None if weights is None else np.array(weights, dtype=np.float64)
+    rc = lib().zo_accumulate(n, len(grads), DTYPES[gdtype], arr, _dp(wts) if wts is not None else None,
+                             float(scale), int(bool(first)), acc.ctypes.data_as(ctypes.POINTER(ctypes.c_float)))
+    del keep
+    if rc != 0:
+        raise ValueError("bad arguments")
+    return acc

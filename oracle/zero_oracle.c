@@ -332,6 +332,30 @@ int zo_reduced_grads(uint64_t n, uint32_t R, int gdtype, const void *const *grad
     return ZO_OK;
 }
 
+/* Micro-step gradient accumulation ("Deep dive: DeepSpeed", "Let the engine
+ * own the microstep" and "Communication volume isn't elapsed time": ZeRO-2/3
+ * reduce and partition the gradient on every backward call, and the owner
+ * keeps only its slice between calls; "Count state before choosing a stage":
+ * a 4-byte (fp32) accumulation array).  For each element:
+ *   acc = (first ? 0 : acc) + scale * reduced gradient of this micro-batch
+ * computed in float64 and stored rounded to the nearest float32 (the
+ * accumulation dtype), so every micro-step rounds once.  The loss scale is
+ * not undone here: the optimizer step does that on the accumulated sum. */
+int zo_accumulate(uint64_t n, uint32_t R, int gdtype, const void *const *grads,
+                  const double *weights, double scale, int first, float *acc)
+{
+    if (R == 0 || grads == NULL || (n > 0 && acc == NULL)) return ZO_EINVAL;
+    if (gdtype < ZO_F64 || gdtype > ZO_F16) return ZO_EINVAL;
+    double wsum = zo_weight_sum(R, weights);
+#pragma omp parallel for
+    for (uint64_t k = 0; k < n; ++k) {
+        double g = zo_reduce(R, gdtype, grads, weights, wsum, 1.0, k);
+        double prev = first ? 0.0 : (double)acc[k];
+        acc[k] = (float)(prev + scale * g);
+    }
+    return ZO_OK;
+}
+
 int zo_max_threads(void)
 {
 #ifdef _OPENMP

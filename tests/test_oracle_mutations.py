@@ -36,6 +36,8 @@ MUTANTS = [
     ("skip keeps the scale", "c->loss_scale *= 0.5;", "c->loss_scale *= 1.0;"),
     ("skip still counts a step", "c->skipped += 1;", "c->skipped += 1; c->t += 1;"),
     ("f16 subnormal off by one", "mag = ldexp((double)f, -24);", "mag = ldexp((double)f, -25);"),
+    ("accumulation ignores first", "double prev = first ? 0.0 : (double)acc[k];", "double prev = (double)acc[k];"),
+    ("accumulation drops the scale", "acc[k] = (float)(prev + scale * g);", "acc[k] = (float)(prev + g);"),
     ("overflow check misses NaN", "if (!isfinite(zo_load(gdtype, grads[r], k))) found |= 1;",
      "if (isinf(zo_load(gdtype, grads[r], k))) found |= 1;"),
 ]

@@ -388,3 +388,55 @@ def test_rounding_of_float32_values_matches_torch():
                           t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
     assert np.array_equal(oracle.rne16(f.astype(np.float64), "f16"),
                           t.to(torch.float16).view(torch.int16).numpy().view(np.uint16))
+
+
+# ------------------------------------------------------- micro-step accumulation
+
+def test_accumulating_the_same_gradient_gas_times_gives_it_back():
+    # "Let the engine own the microstep": with accumulation set to eight, one
+    # update follows eight backward calls; with the engine's 1/8 scaling the
+    # accumulated gradient of eight identical micro-batches is that gradient.
+    rng = np.random.default_rng(12)
+    g = [(rng.normal(0, 1e-3, 1000)).astype(np.float32) for _ in range(4)]
+    want = oracle.reduced_grads(g, "f32")
+    for gas in (1, 2, 8):
+        acc = np.full(1000, 123.0, dtype=np.float32)     # 'first' must discard old contents
+        for mu in range(gas):
+            oracle.accumulate(acc, g, "f32", 1.0 / gas, first=(mu == 0))
+        assert np.allclose(acc, want, rtol=1e-6, atol=0)
+
+
+def test_accumulation_is_the_mean_over_micro_batches_brute_force():
+    # The accumulated value against exact rational arithmetic: the sum over
+    # micro-batches of scale * (token-weighted rank mean), rounded once per
+    # micro-step to float32.
+    rng = np.random.default_rng(13)
+    R, gas, n = 3, 4, 50
+    acc = np.zeros(n, dtype=np.float32)
+    exact_acc = [Fraction(0)] * n
+    for mu in range(gas):
+        g = [(rng.integers(-4096, 4097, n) / 64).astype(np.float32) for _ in range(R)]
+        w = [int(x) for x in rng.integers(1, 4097, R)]
+        oracle.accumulate(acc, g, "f32", 0.25, first=(mu == 0), weights=w)
+        for k in range(n):
+            red = sum(Fraction(w[r]) * Fraction(float(g[r][k])) for r in range(R)) / sum(w)
+            v = exact_acc[k] + Fraction(1, 4) * red
+            exact_acc[k] = Fraction(float(np.float32(float(v))))   # stored as float32
+    assert all(Fraction(float(a)) == e for a, e in zip(acc, exact_acc))
+
+
+def test_scaling_twice_divides_twice():
+    # Dividing each loss by the accumulation count as well scales an
+    # already-averaged gradient a second time.
+    g = [np.full(4, 0.5, dtype=np.float32)]
+    acc = np.zeros(4, dtype=np.float32)
+    for mu in range(8):
+        oracle.accumulate(acc, g, "f32", 1.0 / 64, first=(mu == 0))
+    assert np.all(acc == np.float32(0.5 / 8))
+
+
+def test_accumulation_carries_inf_and_nan_to_the_step():
+    g = [np.array([1.0, np.inf, -np.inf, np.nan], dtype=np.float32)]
+    acc = np.zeros(4, dtype=np.float32)
+    oracle.accumulate(acc, g, "f32", 1.0, first=True)
+    assert acc[0] == 1.0 and np.isinf(acc[1]) and np.isinf(acc[2]) and np.isnan(acc[3])
