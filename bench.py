@@ -49,10 +49,21 @@ WORKLOADS = {
 }
 GRAD_BYTES = {"bf16": 2, "f16": 2, "f32": 4}
 
+# Gradient-accumulation workloads: micro-batches per update.  Each micro-batch
+# of R rank gradients is reduced into an fp32 accumulation array, and the
+# update is one fused step (R = 1, fp32) over that array.
+GAS = {"flat16m_gas4": 4}
+WORKLOADS["flat16m_gas4"] = ("flat", 16_777_259, 8, "bf16", "bf16", False)
 
-def bytes_per_param(R: int, gdt: str) -> int:
+
+def bytes_per_param(R: int, gdt: str, gas: int = 0) -> int:
     """Algorithmic HBM bytes per parameter: R gradient reads, fp32 master and
-    both moments read and written (24), one 16-bit parameter write (2)."""
+    both moments read and written (24), one 16-bit parameter write (2).  With
+    gas micro-batches per update: each micro-batch reads R gradients and
+    writes the fp32 accumulation array (all but the first also read it), and
+    the step reads that array instead of the R gradients."""
+    if gas:
+        return gas * (GRAD_BYTES[gdt] * R + 4) + (gas - 1) * 4 + 4 + 24 + 2
     return GRAD_BYTES[gdt] * R + 24 + 2
 
 
@@ -151,6 +162,19 @@ def build_workload(name: str, device):
     kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
     wl = synth.WORKLOADS.get(name.split("_")[0], 9)
     S = 65536.0 if scaled else 1.0
+    if name in GAS:
+        z = FlatZero(size, 1, "f32", pdt, device=device, loss_scale=S, alloc_grads=False)
+        gt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt]
+        z.micro = [torch.empty(size, dtype=gt, device=device) for _ in range(R)]
+        z.accum = torch.zeros(size, dtype=torch.float32, device=device)
+        z.load_master(synth.normal(z.P, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device))
+        for r, g in enumerate(z.micro):
+            synth.fill_normal_(g, 1e-3, synth.seed_for(wl, synth.KIND_GRAD, r, 1), scale=S)
+        z.gbufs = z.micro
+        z.check = scaled
+        z.gas = GAS[name]
+        z.micro_R, z.micro_gdt = R, gdt
+        return z
     if kind == "flat":
         z = FlatZero(size, R, gdt, pdt, device=device, loss_scale=S, two_set=scaled)
         gbufs = z.grads
@@ -172,6 +196,8 @@ def build_workload(name: str, device):
 
 
 def launches_per_step(z) -> int:
+    if getattr(z, "gas", 0):
+        return z.gas + 1
     if not z.check:
         return 1
     return 2  # two-set single pass + the restore kernel (a no-op unless skipped)
@@ -217,11 +243,22 @@ def run_gpu(args) -> None:
 
     z = build_workload(args.workload, device)
     stream = torch.cuda.current_stream(device)
-    step_args = z.step_args(hp=ADAMW, check=z.check)
-    from mixed_precision_adam_zero_b200 import zero_step_fused, zero_step_fused_list
-    if hasattr(z, "list"):
+    from mixed_precision_adam_zero_b200 import (ZERO_BF16, ZERO_F16, ZERO_F32, zero_accumulate_grads,
+                                                zero_step_fused, zero_step_fused_list)
+    if getattr(z, "gas", 0):
+        step_args = z.step_args(hp=ADAMW, check=z.check, grads=[z.accum])
+        gcode = {"bf16": ZERO_BF16, "f16": ZERO_F16, "f32": ZERO_F32}[z.micro_gdt]
+
+        def call():
+            for mu in range(z.gas):
+                zero_accumulate_grads(z.P, z.micro_R, grad_dtype=gcode, grads=z.micro, accum=z.accum,
+                                      scale=1.0 / z.gas, first=(mu == 0), stream=stream)
+            zero_step_fused(step_args, stream)
+    elif hasattr(z, "list"):
+        step_args = z.step_args(hp=ADAMW, check=z.check)
         call = lambda: zero_step_fused_list(step_args, z.list, stream)
     else:
+        step_args = z.step_args(hp=ADAMW, check=z.check)
         call = lambda: zero_step_fused(step_args, stream)
 
     def barrier():
@@ -280,7 +317,7 @@ def run_gpu(args) -> None:
     if rank == 0:
         kind, size, R, gdt, pdt, scaled = WORKLOADS[args.workload]
         P = z.P
-        bpp = bytes_per_param(R, gdt)
+        bpp = bytes_per_param(R, gdt, GAS.get(args.workload, 0))
         peaks = measured_peaks()
         peak = peaks.get("hbm_gbs")
         peak_src = "measured" if peak else "fallback"

@@ -295,6 +295,39 @@ int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t *numel,
  * zero_step_fused. */
 int zero_step_fused_noalloc(const zero_step_args *args, void *stream);
 
+/* ------------------------------------------------- micro-step accumulation */
+
+/* One micro-batch's contribution to the fp32 gradient accumulation array
+ * ("Deep dive: DeepSpeed": "Let the engine own the microstep" -- one update
+ * per gradient-accumulation window; "Communication volume isn't elapsed
+ * time" -- ZeRO-2/3 reduce and partition the gradient on every backward call
+ * and keep only the owned slice between calls; "Count state before choosing
+ * a stage" -- a 4-byte accumulation array, the 18-byte recipe).
+ * For every element i of the slice:
+ *   accum[i] = (first ? 0 : accum[i]) + scale * (sum_r w_r grad_r[i]) / sum(w)
+ * computed in float64 and rounded once to float32.  The loss scale is not
+ * undone here: after the last micro-batch, call zero_step_fused with R = 1,
+ * grad_dtype ZERO_F32 and grads = {accum}; the step unscales, checks for
+ * inf/NaN (which the sums carry) and skips exactly as for raw gradients.
+ * scale is typically 1/(micro-batches per update) when each micro-batch loss
+ * is a mean that was not divided by that count. */
+typedef struct zero_accum_args {
+    uint64_t P;                  /* elements of the flat vector; 0 is allowed */
+    uint32_t R;                  /* ranks, 1..ZERO_MAX_RANKS */
+    int32_t owner;               /* -1: all of [0,P); 0..R-1: that owner's slice */
+    int32_t grad_dtype;          /* ZERO_F32, ZERO_BF16 or ZERO_F16 */
+    int32_t first;               /* 1: start the window (accum ignored on input) */
+    const void *const *grads;    /* HOST array of R device pointers [P] */
+    const double *rank_weights;  /* HOST array of R weights, or NULL (equal) */
+    float *accum;                /* device [P] fp32 accumulation array */
+    double scale;                /* finite */
+} zero_accum_args;
+
+/* Launches one kernel; asynchronous on `stream`.  Errors: ZERO_EINVAL,
+ * ZERO_EALIGN (pointers must be 16-byte aligned), ZERO_ERANGE, ZERO_EOVERFLOW,
+ * ZERO_ECUDA. */
+int zero_accumulate_grads(const zero_accum_args *args, void *stream);
+
 /* --------------------------------------------------------------- gathers */
 
 /* params16[i] = round-to-nearest-even(master[i]) for i in [0,P): the cast of

@@ -40,7 +40,7 @@ EXPORTED = [
     "zero_ctrl_bytes", "zero_workspace_bytes", "zero_list_table_bytes", "zero_ctrl_init",
     "zero_ctrl_set", "zero_ctrl_read", "zero_workspace_init", "zero_step_fused",
     "zero_step_fused_list", "zero_list_table_build", "zero_gather_params",
-    "zero_gather_params_list", "zero_step_fused_noalloc",
+    "zero_gather_params_list", "zero_step_fused_noalloc", "zero_accumulate_grads",
 ]
 
 
@@ -77,6 +77,14 @@ class zero_step_args(ctypes.Structure):
                 ("ctrl", ctypes.c_void_p), ("workspace", ctypes.c_void_p)]
 
 
+class zero_accum_args(ctypes.Structure):
+    _fields_ = [("P", ctypes.c_uint64), ("R", ctypes.c_uint32), ("owner", ctypes.c_int32),
+                ("grad_dtype", ctypes.c_int32), ("first", ctypes.c_int32),
+                ("grads", ctypes.POINTER(ctypes.c_void_p)),
+                ("rank_weights", ctypes.POINTER(ctypes.c_double)), ("accum", ctypes.c_void_p),
+                ("scale", ctypes.c_double)]
+
+
 class zero_tensor_list(ctypes.Structure):
     _fields_ = [("table", ctypes.c_void_p), ("P", ctypes.c_uint64), ("T", ctypes.c_uint32),
                 ("R", ctypes.c_uint32), ("grad_dtype", ctypes.c_int32),
@@ -111,6 +119,7 @@ def _lib() -> ctypes.CDLL:
         L.zero_workspace_init.argtypes = [vp, vp]
         L.zero_step_fused.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_step_fused_noalloc.argtypes = [ctypes.POINTER(zero_step_args), vp]
+        L.zero_accumulate_grads.argtypes = [ctypes.POINTER(zero_accum_args), vp]
         L.zero_step_fused_list.argtypes = [ctypes.POINTER(zero_step_args), ctypes.POINTER(zero_tensor_list), vp]
         L.zero_list_table_build.argtypes = [u32, u32, u64p, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32,
                                             vp, sz, ctypes.POINTER(zero_tensor_list), vp]
@@ -267,3 +276,21 @@ def zero_gather_params(master, params16, param_dtype: int, P: int, stream=None) 
 def zero_gather_params_list(master, lst: zero_tensor_list, stream=None) -> None:
     _check(_lib().zero_gather_params_list(_ptr(master), ctypes.byref(lst), _stream(stream)),
            "zero_gather_params_list")
+
+
+def zero_accumulate_grads(P: int, R: int, *, grad_dtype: int, grads: Sequence, accum, scale: float,
+                          first: bool, rank_weights: Optional[Sequence[float]] = None, owner: int = -1,
+                          stream=None) -> None:
+    """One micro-batch into the fp32 accumulation array (see the C declaration)."""
+    a = zero_accum_args()
+    a.P, a.R, a.owner, a.grad_dtype, a.first = P, R, owner, grad_dtype, int(bool(first))
+    arr = (ctypes.c_void_p * len(grads))(*[_ptr(g) for g in grads])
+    a.grads = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    keep = [arr]
+    if rank_weights is not None:
+        w = (ctypes.c_double * len(rank_weights))(*[float(x) for x in rank_weights])
+        keep.append(w)
+        a.rank_weights = ctypes.cast(w, ctypes.POINTER(ctypes.c_double))
+    a.accum = _ptr(accum)
+    a.scale = float(scale)
+    _check(_lib().zero_accumulate_grads(ctypes.byref(a), _stream(stream)), "zero_accumulate_grads")

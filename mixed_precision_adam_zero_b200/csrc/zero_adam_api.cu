@@ -187,6 +187,25 @@ const void* gather_fn(int32_t param_dtype) {
                                     : (const void*)gather_kernel<__half, LIST>;
 }
 
+template <class G>
+const void* accum_fn_rc(uint32_t R) {
+    switch (R) {
+        case 1: return (const void*)accum_kernel<G, 1>;
+        case 2: return (const void*)accum_kernel<G, 2>;
+        case 4: return (const void*)accum_kernel<G, 4>;
+        case 8: return (const void*)accum_kernel<G, 8>;
+        default: return (const void*)accum_kernel<G, 0>;
+    }
+}
+
+const void* accum_fn(int32_t grad_dtype, uint32_t R) {
+    switch (grad_dtype) {
+        case ZERO_F32: return accum_fn_rc<float>(R);
+        case ZERO_BF16: return accum_fn_rc<__nv_bfloat16>(R);
+        default: return accum_fn_rc<__half>(R);
+    }
+}
+
 // ------------------------------------------------------------ argument checks
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -466,6 +485,52 @@ int zero_step_fused_list(const zero_step_args* a, const zero_tensor_list* l, voi
     kp.tab = device_table(l);
     kp.whole = a->owner < 0 ? 1 : 0;
     return run_step<true>(a, &kp, static_cast<cudaStream_t>(stream));
+}
+
+int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
+    if (a == nullptr || a->R == 0 || a->grads == nullptr) return ZERO_EINVAL;
+    if (a->R > ZERO_MAX_RANKS) return ZERO_ERANGE;
+    if (a->owner < -1 || a->owner >= (int64_t)a->R) return ZERO_EINVAL;
+    if (!is_grad_dtype(a->grad_dtype) || (a->first != 0 && a->first != 1)) return ZERO_EINVAL;
+    if (!std::isfinite(a->scale)) return ZERO_EINVAL;
+    if (a->P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
+    if (a->P > 0 && a->accum == nullptr) return ZERO_EINVAL;
+    if (!aligned16(a->accum)) return ZERO_EALIGN;
+    AccumParams ap;
+    std::memset(&ap, 0, sizeof ap);
+    double wsum = 0.0;
+    for (uint32_t r = 0; r < a->R; ++r) {
+        if (a->P > 0 && a->grads[r] == nullptr) return ZERO_EINVAL;
+        if (!aligned16(a->grads[r])) return ZERO_EALIGN;
+        const double wr = a->rank_weights ? a->rank_weights[r] : 1.0;
+        if (!finite_nonneg(wr)) return ZERO_EINVAL;
+        ap.grads[r] = a->grads[r];
+        ap.wt[r] = wr;
+        wsum += wr;
+    }
+    if (!(wsum > 0.0) || !std::isfinite(wsum)) return ZERO_EINVAL;
+    ap.inv_wsum = 1.0 / wsum;
+    ap.scale = a->scale;
+    ap.acc = a->accum;
+    ap.R = a->R;
+    ap.first = a->first;
+    if (a->owner < 0) {
+        ap.lo = 0;
+        ap.hi = a->P;
+    } else {
+        const unsigned __int128 P = a->P;
+        ap.lo = (uint64_t)((P * (uint32_t)a->owner) / a->R);
+        ap.hi = (uint64_t)((P * ((uint32_t)a->owner + 1u)) / a->R);
+    }
+    if (ap.lo >= ap.hi) return ZERO_OK;
+    int err = ZERO_OK;
+    const void* fn = accum_fn(a->grad_dtype, a->R);
+    const int ctas = resident_ctas(fn, &err);
+    if (err) return err;
+    const Shape sh = make_shape(ap.lo, ap.hi, ctas);
+    ap.base = sh.base;
+    ap.chunk = sh.chunk;
+    return launch(fn, sh, &ap, static_cast<cudaStream_t>(stream));
 }
 
 int zero_step_fused_noalloc(const zero_step_args* a, void* stream) {

@@ -595,6 +595,87 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant_
     }
 }
 
+// ------------------------------------------------------------ micro-step accumulation
+
+struct AccumParams {
+    const void* grads[ZERO_MAX_RANKS];  // rank r's micro-batch gradient [P]
+    double wt[ZERO_MAX_RANKS];          // rank weights
+    double inv_wsum;                    // 1 / sum(w)
+    double scale;                       // multiplies the reduced gradient
+    float* acc;                         // fp32 accumulation array [P]
+    uint64_t lo, hi, base, chunk;
+    uint32_t R;
+    int32_t first;                      // 1: acc starts from zero
+};
+
+// acc = (first ? 0 : acc) + scale * (sum_r w_r g_r) / sum(w), float64, one rounding.
+template <class G, int RC>
+__device__ __forceinline__ void accum_vec(const AccumParams& p, const GradPtrs<G, RC>& gp, uint64_t e) {
+    double acc[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.0;
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    if (!p.first) {
+        a0 = __ldcs(reinterpret_cast<const float4*>(p.acc + e));
+        a1 = __ldcs(reinterpret_cast<const float4*>(p.acc + e + 4));
+    }
+    const int R = RC > 0 ? RC : (int)p.R;
+    if constexpr (RC > 0) {
+        Raw8<G> raw[RC];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) raw[r] = load8<G>(gp[r], e);
+#pragma unroll
+        for (int r = 0; r < RC; ++r) {
+            float f[8];
+            unpack8(raw[r], f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = fma(p.wt[r], (double)f[k], acc[k]);
+        }
+    } else {
+        for (int r = 0; r < R; ++r) {
+            float f[8];
+            unpack8(load8<G>(gp[r], e), f);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = fma(p.wt[r], (double)f[k], acc[k]);
+        }
+    }
+    const float prev[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    float out[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) out[k] = (float)((double)prev[k] + p.scale * (acc[k] * p.inv_wsum));
+    __stcs(reinterpret_cast<float4*>(p.acc + e), make_float4(out[0], out[1], out[2], out[3]));
+    __stcs(reinterpret_cast<float4*>(p.acc + e + 4), make_float4(out[4], out[5], out[6], out[7]));
+}
+
+template <class G, int RC>
+__device__ __forceinline__ void accum_elem(const AccumParams& p, const GradPtrs<G, RC>& gp, uint64_t e) {
+    double acc = 0.0;
+    const int R = RC > 0 ? RC : (int)p.R;
+    for (int r = 0; r < R; ++r) {
+        bool b = false;
+        acc = fma(p.wt[r], (double)load1<G>(gp[r], e, b), acc);
+    }
+    const double prev = p.first ? 0.0 : (double)p.acc[e];
+    p.acc[e] = (float)(prev + p.scale * (acc * p.inv_wsum));
+}
+
+template <class G, int RC>
+__global__ void __launch_bounds__(kThreads) accum_kernel(const __grid_constant__ AccumParams p) {
+    uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
+    uint64_t b = a + p.chunk;
+    if (a < p.lo) a = p.lo;
+    if (b > p.hi) b = p.hi;
+    if (a >= b) return;
+    const GradPtrs<G, RC> gp(&p.grads[0]);
+    uint64_t va = (a + 7) & ~7ull, vb = b & ~7ull;
+    if (va > b) va = b;
+    if (vb < va) vb = va;
+    for (uint64_t e = a + threadIdx.x; e < va; e += kThreads) accum_elem<G, RC>(p, gp, e);
+    for (uint64_t e = va + (uint64_t)threadIdx.x * kVec; e < vb; e += (uint64_t)kThreads * kVec)
+        accum_vec<G, RC>(p, gp, e);
+    for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads) accum_elem<G, RC>(p, gp, e);
+}
+
 // ------------------------------------------------------------ control block
 
 __global__ void ctrl_set_kernel(zero_ctrl* c, zero_ctrl value) { *c = value; }

@@ -40,9 +40,11 @@ def assert_close(gpu: torch.Tensor, ref: np.ndarray, name: str) -> None:
     g = gpu.detach().double().cpu().numpy().ravel()
     ref = np.asarray(ref, dtype=np.float64).ravel()
     assert g.shape == ref.shape, name
-    err = np.abs(g - ref)
-    bound = TOL_REL * np.abs(ref) + TOL_ABS
-    bad = ~(err <= bound)
+    same = (g == ref) | (np.isnan(g) & np.isnan(ref))      # identical, including inf and NaN
+    with np.errstate(invalid="ignore"):
+        err = np.abs(g - ref)
+        bound = TOL_REL * np.abs(ref) + TOL_ABS
+        bad = ~(same | (err <= bound))
     if bad.any():
         i = int(np.flatnonzero(bad)[0])
         raise AssertionError(f"{name}: {int(bad.sum())} of {g.size} outside tolerance; first at {i}: "

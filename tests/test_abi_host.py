@@ -175,3 +175,24 @@ def test_noalloc_step_refuses_a_caller_workspace():
     with pytest.raises(za.ZeroError) as e:
         za.zero_step_fused_noalloc(a)
     assert e.value.status == za.ZERO_EINVAL
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(R=0, grads=[]), za.ZERO_EINVAL),
+    (dict(R=300, grads=[A] * 300), za.ZERO_ERANGE),
+    (dict(owner=4), za.ZERO_EINVAL),
+    (dict(grad_dtype=9), za.ZERO_EINVAL),
+    (dict(scale=float("nan")), za.ZERO_EINVAL),
+    (dict(accum=A + 4), za.ZERO_EALIGN),
+    (dict(accum=None), za.ZERO_EINVAL),
+    (dict(grads=[A, A + 2, A, A]), za.ZERO_EALIGN),
+    (dict(rank_weights=[1, 1, -1, 1]), za.ZERO_EINVAL),
+    (dict(P=2**62), za.ZERO_EOVERFLOW),
+])
+def test_accumulate_argument_errors(kw, status):
+    args = dict(P=1000, R=4, grad_dtype=za.ZERO_BF16, grads=[A] * 4, accum=A, scale=0.25, first=True)
+    args.update(kw)
+    P, R = args.pop("P"), args.pop("R")
+    with pytest.raises(za.ZeroError) as e:
+        za.zero_accumulate_grads(P, R, **args)
+    assert e.value.status == status
