@@ -57,6 +57,7 @@ extern "C" {
 #define ZERO_EOVERFLOW (-3) /* a byte size does not fit in 64 bits */
 #define ZERO_ERANGE (-4)    /* a count beyond a documented limit */
 #define ZERO_ECUDA (-5)     /* a CUDA runtime call or launch failed (zero_last_cuda_error) */
+#define ZERO_EIO (-6)       /* a checkpoint file could not be used (zero_checkpoint_error) */
 
 /* ------------------------------------------------------------------ dtypes */
 #define ZERO_F32 0  /* IEEE binary32 */
@@ -327,6 +328,41 @@ typedef struct zero_accum_args {
  * ZERO_EALIGN (pointers must be 16-byte aligned), ZERO_ERANGE, ZERO_EOVERFLOW,
  * ZERO_ECUDA. */
 int zero_accumulate_grads(const zero_accum_args *args, void *stream);
+
+/* ------------------------------------------------------------ checkpoints */
+
+/* Checkpoint files ("Deep dive: DeepSpeed", "Resume training and export
+ * weights separately": resuming a run needs the weights, both Adam moments
+ * and the step counter, and the next update must then agree with an
+ * uninterrupted run; exporting a model needs only the consolidated weights).
+ *
+ * A shard file holds one owner's slice (args->owner = r, the slice
+ * [floor(P*r/R), floor(P*(r+1)/R))) or, with owner = -1, the whole vector:
+ * a 128-byte header (magic "ZADAMCK1", R, P, owner, slice bounds, the control
+ * block with parity reset to 0), the slice of the fp32 master weights, first
+ * and second moments, and a 64-bit FNV-1a checksum.  Each owner writes and
+ * reads its own shard, as each data-parallel rank saves its partition.
+ * These calls are SYNCHRONOUS (they stage through host memory and wait for
+ * `stream`); they allocate host memory only.  Errors: ZERO_EINVAL, ZERO_EIO
+ * (text from zero_checkpoint_error), ZERO_ECUDA. */
+
+/* Write the current state set (ctrl.parity in two-set mode) of args->owner's
+ * slice and its control block to `path`.  Uses P, R, owner, master,
+ * exp_avg, exp_avg_sq and ctrl of args. */
+int zero_checkpoint_save(const char *path, const zero_step_args *args, void *stream);
+
+/* Restore a shard written for the same P, R and owner into state set 0 and
+ * the control block (parity 0); if args->params16 is given (flat layout),
+ * re-cast the 16-bit parameters of the slice from the restored masters. */
+int zero_checkpoint_load(const char *path, const zero_step_args *args, void *stream);
+
+/* Consolidate the fp32 master weights of shard files into HOST memory
+ * `weights` [P] (the weights-only export): the shards must all be for this P
+ * and their slices must tile [0, P) exactly; every checksum is verified. */
+int zero_checkpoint_consolidate(const char *const *paths, uint32_t n_paths, float *weights, uint64_t P);
+
+/* Text of the last checkpoint error of this thread. */
+const char *zero_checkpoint_error(void);
 
 /* --------------------------------------------------------------- gathers */
 

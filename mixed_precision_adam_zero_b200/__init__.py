@@ -26,6 +26,7 @@ ZERO_EALIGN = -2
 ZERO_EOVERFLOW = -3
 ZERO_ERANGE = -4
 ZERO_ECUDA = -5
+ZERO_EIO = -6
 
 ZERO_F32 = 0
 ZERO_BF16 = 1
@@ -41,6 +42,7 @@ EXPORTED = [
     "zero_ctrl_set", "zero_ctrl_read", "zero_workspace_init", "zero_step_fused",
     "zero_step_fused_list", "zero_list_table_build", "zero_gather_params",
     "zero_gather_params_list", "zero_step_fused_noalloc", "zero_accumulate_grads",
+    "zero_checkpoint_save", "zero_checkpoint_load", "zero_checkpoint_consolidate", "zero_checkpoint_error",
 ]
 
 
@@ -49,6 +51,8 @@ class ZeroError(RuntimeError):
         text = _lib().zero_status_string(status).decode()
         if status == ZERO_ECUDA:
             text += ": " + _lib().zero_last_cuda_error().decode()
+        if status == ZERO_EIO:
+            text += ": " + _lib().zero_checkpoint_error().decode()
         super().__init__(f"{where}: status {status} ({text})")
         self.status = status
 
@@ -120,6 +124,11 @@ def _lib() -> ctypes.CDLL:
         L.zero_step_fused.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_step_fused_noalloc.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_accumulate_grads.argtypes = [ctypes.POINTER(zero_accum_args), vp]
+        L.zero_checkpoint_save.argtypes = [ctypes.c_char_p, ctypes.POINTER(zero_step_args), vp]
+        L.zero_checkpoint_load.argtypes = [ctypes.c_char_p, ctypes.POINTER(zero_step_args), vp]
+        L.zero_checkpoint_consolidate.argtypes = [ctypes.POINTER(ctypes.c_char_p), u32,
+                                                  ctypes.POINTER(ctypes.c_float), u64]
+        L.zero_checkpoint_error.restype = ctypes.c_char_p
         L.zero_step_fused_list.argtypes = [ctypes.POINTER(zero_step_args), ctypes.POINTER(zero_tensor_list), vp]
         L.zero_list_table_build.argtypes = [u32, u32, u64p, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32,
                                             vp, sz, ctypes.POINTER(zero_tensor_list), vp]
@@ -294,3 +303,27 @@ def zero_accumulate_grads(P: int, R: int, *, grad_dtype: int, grads: Sequence, a
     a.accum = _ptr(accum)
     a.scale = float(scale)
     _check(_lib().zero_accumulate_grads(ctypes.byref(a), _stream(stream)), "zero_accumulate_grads")
+
+
+def zero_checkpoint_save(path: str, args: zero_step_args, stream=None) -> None:
+    _check(_lib().zero_checkpoint_save(os.fsencode(path), ctypes.byref(args), _stream(stream)),
+           "zero_checkpoint_save")
+
+
+def zero_checkpoint_load(path: str, args: zero_step_args, stream=None) -> None:
+    _check(_lib().zero_checkpoint_load(os.fsencode(path), ctypes.byref(args), _stream(stream)),
+           "zero_checkpoint_load")
+
+
+def zero_checkpoint_consolidate(paths: Sequence[str], P: int):
+    """fp32 weights [P] (numpy) consolidated from shard files."""
+    import numpy as np
+    out = np.empty(P, dtype=np.float32)
+    arr = (ctypes.c_char_p * len(paths))(*[os.fsencode(x) for x in paths])
+    _check(_lib().zero_checkpoint_consolidate(arr, len(paths), out.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), P),
+           "zero_checkpoint_consolidate")
+    return out
+
+
+def zero_checkpoint_error() -> str:
+    return _lib().zero_checkpoint_error().decode()

@@ -7,7 +7,8 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = [os.path.join(PKG, "csrc", "zero_adam_api.cu"), os.path.join(PKG, "csrc", "zero_adam_host.cpp")]
+SOURCES = [os.path.join(PKG, "csrc", "zero_adam_api.cu"), os.path.join(PKG, "csrc", "zero_adam_host.cpp"),
+           os.path.join(PKG, "csrc", "zero_adam_ckpt.cpp")]
 DEPS = SOURCES + [os.path.join(PKG, "csrc", "zero_adam_kernels.cuh"), os.path.join(PKG, "csrc", "zero_adam_bulk.cuh"),
                   os.path.join(ROOT, "include", "zero_adam.h")]
 OUT = os.path.join(PKG, "libzero_adam.so")

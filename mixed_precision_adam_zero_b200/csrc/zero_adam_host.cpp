@@ -50,6 +50,7 @@ const char* zero_status_string(int status) {
         case ZERO_EOVERFLOW: return "byte size overflows 64 bits";
         case ZERO_ERANGE: return "count beyond a documented limit";
         case ZERO_ECUDA: return "CUDA runtime error (see zero_last_cuda_error)";
+        case ZERO_EIO: return "checkpoint file error (see zero_checkpoint_error)";
         default: return "unknown status";
     }
 }
