@@ -329,6 +329,49 @@ typedef struct zero_accum_args {
  * ZERO_ECUDA. */
 int zero_accumulate_grads(const zero_accum_args *args, void *stream);
 
+/* ------------------------------------------------------------------ ZeRO-3 */
+
+/* ZeRO-3 partitions the 16-bit parameters too ("ZeRO" documentation page,
+ * stage 3; "Deep dive: DeepSpeed", "Stage 3 needs a live working set"): each
+ * rank keeps of every tensor of n elements a shard of s = ceil(n/R) elements
+ * -- rank r holding elements [r*s, min((r+1)*s, n)), the last shards padded --
+ * and a module's full view is gathered into a separate padded buffer of R*s
+ * elements before use (and may be released after).
+ *
+ * The optimizer step of one rank is zero_step_fused_list over that rank's
+ * shard tensors: a list whose tensor j has hi-lo elements, whose 16-bit
+ * parameters are the rank's shard buffer, and whose gradient pointer of rank
+ * r' is r''s full gradient of tensor j advanced by lo elements (the in-HBM
+ * reduce-scatter); master and moments are the rank's own flat shard state. */
+
+/* Shard of rank r of a tensor of n elements: *shard = ceil(n/R), and the
+ * rank holds elements [*lo, *hi) of the tensor (possibly empty).  Host only.
+ * ZERO_EINVAL if R == 0, r >= R or a pointer is NULL. */
+int zero3_shard_bounds(uint64_t n, uint32_t R, uint32_t r, uint64_t *lo, uint64_t *hi, uint64_t *shard);
+
+/* Parameter storage of one rank in elements (the same section's model):
+ * out[0] = resident shards (sum of ceil(n_j/R)), out[1] = gathered buffers
+ * (sum over the live tensors of R*ceil(n_j/R)), out[2] = their sum.  sizes:
+ * HOST array of T counts (all > 0); live: HOST array of n_live distinct
+ * tensor indices.  Host only.  ZERO_EINVAL on bad arguments, ZERO_EOVERFLOW. */
+int zero_parameter_storage(const uint64_t *sizes, uint32_t T, uint32_t R, const uint32_t *live,
+                           uint32_t n_live, uint64_t out[3]);
+
+/* Build a gather list (table as for zero_list_table_build, >=
+ * zero_list_table_bytes(T, R) bytes): numel = the tensors' true sizes,
+ * full = T device buffers of R*ceil(n_j/R) elements (the padded full views),
+ * shards = R*T device pointers, rank-major (shards[r*T + j], ceil(n_j/R)
+ * elements each), dtype ZERO_BF16 or ZERO_F16.  SYNCHRONOUS like the list
+ * build. */
+int zero3_gather_list_build(uint32_t T, uint32_t R, const uint64_t *numel, void *const *full,
+                            const void *const *shards, int32_t dtype, void *table, size_t table_bytes,
+                            zero_tensor_list *out, void *stream);
+
+/* full_j[r*s_j + k] = shard_{r,j}[k] for every tensor, rank and k < s_j,
+ * padding included: the module-level all-gather of ZeRO-3 on one GPU (2 bytes
+ * read and 2 written per padded element).  One kernel, asynchronous. */
+int zero3_gather(const zero_tensor_list *gather_list, void *stream);
+
 /* ------------------------------------------------------------ checkpoints */
 
 /* Checkpoint files ("Deep dive: DeepSpeed", "Resume training and export

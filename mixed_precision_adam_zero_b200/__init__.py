@@ -43,6 +43,7 @@ EXPORTED = [
     "zero_step_fused_list", "zero_list_table_build", "zero_gather_params",
     "zero_gather_params_list", "zero_step_fused_noalloc", "zero_accumulate_grads",
     "zero_checkpoint_save", "zero_checkpoint_load", "zero_checkpoint_consolidate", "zero_checkpoint_error",
+    "zero3_shard_bounds", "zero_parameter_storage", "zero3_gather_list_build", "zero3_gather",
 ]
 
 
@@ -129,6 +130,11 @@ def _lib() -> ctypes.CDLL:
         L.zero_checkpoint_consolidate.argtypes = [ctypes.POINTER(ctypes.c_char_p), u32,
                                                   ctypes.POINTER(ctypes.c_float), u64]
         L.zero_checkpoint_error.restype = ctypes.c_char_p
+        L.zero3_shard_bounds.argtypes = [u64, u32, u32, u64p, u64p, u64p]
+        L.zero_parameter_storage.argtypes = [u64p, u32, u32, ctypes.POINTER(ctypes.c_uint32), u32, u64p]
+        L.zero3_gather_list_build.argtypes = [u32, u32, u64p, ctypes.POINTER(vp), ctypes.POINTER(vp), i32,
+                                              vp, sz, ctypes.POINTER(zero_tensor_list), vp]
+        L.zero3_gather.argtypes = [ctypes.POINTER(zero_tensor_list), vp]
         L.zero_step_fused_list.argtypes = [ctypes.POINTER(zero_step_args), ctypes.POINTER(zero_tensor_list), vp]
         L.zero_list_table_build.argtypes = [u32, u32, u64p, ctypes.POINTER(vp), ctypes.POINTER(vp), i32, i32,
                                             vp, sz, ctypes.POINTER(zero_tensor_list), vp]
@@ -327,3 +333,37 @@ def zero_checkpoint_consolidate(paths: Sequence[str], P: int):
 
 def zero_checkpoint_error() -> str:
     return _lib().zero_checkpoint_error().decode()
+
+
+def zero3_shard_bounds(n: int, R: int, r: int) -> Tuple[int, int, int]:
+    """(lo, hi, shard): rank r holds elements [lo, hi) of a tensor of n; shard = ceil(n/R)."""
+    lo, hi, sh = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+    _check(_lib().zero3_shard_bounds(n, R, r, ctypes.byref(lo), ctypes.byref(hi), ctypes.byref(sh)),
+           "zero3_shard_bounds")
+    return lo.value, hi.value, sh.value
+
+
+def zero_parameter_storage(sizes: Sequence[int], R: int, live: Sequence[int]) -> Tuple[int, int, int]:
+    """(resident, gathered, total) elements of one rank's ZeRO-3 parameter storage."""
+    sz = (ctypes.c_uint64 * max(len(sizes), 1))(*sizes)
+    lv = (ctypes.c_uint32 * max(len(live), 1))(*live)
+    out = (ctypes.c_uint64 * 3)()
+    _check(_lib().zero_parameter_storage(sz, len(sizes), R, lv, len(live), out), "zero_parameter_storage")
+    return tuple(out)
+
+
+def zero3_gather_list_build(numel: Sequence[int], full: Sequence, shards: Sequence[Sequence], dtype: int,
+                            table, table_bytes: int, stream=None) -> zero_tensor_list:
+    """shards[r][j]: rank r's shard of tensor j; full[j]: its padded full view."""
+    T, R = len(numel), len(shards)
+    n = (ctypes.c_uint64 * T)(*numel)
+    f = (ctypes.c_void_p * T)(*[_ptr(x) for x in full])
+    g = (ctypes.c_void_p * (R * T))(*[_ptr(shards[r][j]) for r in range(R) for j in range(T)])
+    out = zero_tensor_list()
+    _check(_lib().zero3_gather_list_build(T, R, n, f, g, dtype, _ptr(table), table_bytes, ctypes.byref(out),
+                                          _stream(stream)), "zero3_gather_list_build")
+    return out
+
+
+def zero3_gather(gather_list: zero_tensor_list, stream=None) -> None:
+    _check(_lib().zero3_gather(ctypes.byref(gather_list), _stream(stream)), "zero3_gather")

@@ -604,6 +604,41 @@ int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t* numel, void* c
     return ZERO_OK;
 }
 
+int zero3_gather_list_build(uint32_t T, uint32_t R, const uint64_t* numel, void* const* full,
+                            const void* const* shards, int32_t dtype, void* table, size_t table_bytes,
+                            zero_tensor_list* out, void* stream) {
+    if (T == 0 || R == 0 || numel == nullptr) return ZERO_EINVAL;
+    std::vector<uint64_t> padded(T);
+    for (uint32_t j = 0; j < T; ++j) {
+        const uint64_t s = numel[j] / R + (numel[j] % R != 0 ? 1u : 0u);
+        if (s > (UINT64_MAX >> 4) / R) return ZERO_EOVERFLOW;
+        padded[j] = s * R;
+    }
+    return zero_list_table_build(T, R, padded.data(), full, shards, dtype, dtype, table, table_bytes, out, stream);
+}
+
+int zero3_gather(const zero_tensor_list* l, void* stream) {
+    int rc = check_list(l);
+    if (rc) return rc;
+    if (l->grad_dtype != l->param_dtype || l->param_dtype == ZERO_F32) return ZERO_EINVAL;
+    if (l->P == 0) return ZERO_OK;
+    Z3Params zp;
+    std::memset(&zp, 0, sizeof zp);
+    zp.tab = device_table(l);
+    zp.lo = 0;
+    zp.hi = l->P;
+    zp.R = l->R;
+    int err = ZERO_OK;
+    const void* fn = l->param_dtype == ZERO_BF16 ? (const void*)z3_gather_kernel<__nv_bfloat16>
+                                                 : (const void*)z3_gather_kernel<__half>;
+    const int ctas = resident_ctas(fn, &err);
+    if (err) return err;
+    const Shape sh = make_shape(0, l->P, ctas);
+    zp.base = sh.base;
+    zp.chunk = sh.chunk;
+    return launch(fn, sh, &zp, static_cast<cudaStream_t>(stream));
+}
+
 int zero_gather_params(const float* master, void* params16, int32_t param_dtype, uint64_t P, void* stream) {
     if (!is_param_dtype(param_dtype)) return ZERO_EINVAL;
     if (P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;

@@ -42,6 +42,45 @@ int zero_state_bytes(uint64_t P, uint32_t R, uint32_t param_b, uint32_t grad_b, 
     return ZERO_OK;
 }
 
+// "Deep dive: DeepSpeed", "Stage 3 needs a live working set": each rank
+// keeps of a tensor of n elements a shard of ceil(n/R) elements (the last
+// shards padded), rank r holding elements [r*s, min((r+1)*s, n)).
+int zero3_shard_bounds(uint64_t n, uint32_t R, uint32_t r, uint64_t* lo, uint64_t* hi, uint64_t* shard) {
+    if (R == 0 || r >= R || lo == nullptr || hi == nullptr || shard == nullptr) return ZERO_EINVAL;
+    const uint64_t s = n / R + (n % R != 0 ? 1u : 0u);
+    const unsigned __int128 a = (unsigned __int128)s * r, b = (unsigned __int128)s * (r + 1u);
+    *shard = s;
+    *lo = a < n ? (uint64_t)a : n;
+    *hi = b < n ? (uint64_t)b : n;
+    return ZERO_OK;
+}
+
+// The same section's storage model, in elements: resident shards of every
+// tensor, plus one separate full padded buffer (R shards) per live tensor.
+int zero_parameter_storage(const uint64_t* sizes, uint32_t T, uint32_t R, const uint32_t* live, uint32_t n_live,
+                           uint64_t out[3]) {
+    if (sizes == nullptr || T == 0 || R == 0 || out == nullptr || (n_live > 0 && live == nullptr))
+        return ZERO_EINVAL;
+    unsigned __int128 resident = 0, gathered = 0;
+    for (uint32_t j = 0; j < T; ++j) {
+        if (sizes[j] == 0) return ZERO_EINVAL;
+        resident += sizes[j] / R + (sizes[j] % R != 0 ? 1u : 0u);
+    }
+    for (uint32_t i = 0; i < n_live; ++i) {
+        if (live[i] >= T) return ZERO_EINVAL;
+        for (uint32_t k = 0; k < i; ++k)
+            if (live[k] == live[i]) return ZERO_EINVAL;
+        const uint64_t n = sizes[live[i]];
+        gathered += (unsigned __int128)(n / R + (n % R != 0 ? 1u : 0u)) * R;
+    }
+    const unsigned __int128 total = resident + gathered;
+    if (total > (unsigned __int128)UINT64_MAX) return ZERO_EOVERFLOW;
+    out[0] = (uint64_t)resident;
+    out[1] = (uint64_t)gathered;
+    out[2] = (uint64_t)total;
+    return ZERO_OK;
+}
+
 const char* zero_status_string(int status) {
     switch (status) {
         case ZERO_OK: return "ok";

@@ -595,6 +595,56 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant_
     }
 }
 
+// ------------------------------------------------------------ ZeRO-3 gather
+
+// Full padded views of tensors from their R rank shards.  The table is a
+// gather list: tensor j's element count is R * s_j (its padded full size),
+// params[j] is the full view buffer and grads[j*R + r] rank r's shard of s_j
+// elements, so full_j[r*s_j + k] = shard_{r,j}[k].  Launch space: the padded
+// concatenation [0, sum_j R*s_j).
+struct Z3Params {
+    Table tab;
+    uint64_t lo, hi, base, chunk;
+    uint32_t R;
+};
+
+template <class Pm>
+__global__ void __launch_bounds__(kThreads) z3_gather_kernel(const __grid_constant__ Z3Params p) {
+    uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
+    uint64_t b = a + p.chunk;
+    if (a < p.lo) a = p.lo;
+    if (b > p.hi) b = p.hi;
+    if (a >= b) return;
+    uint32_t j = find_tensor(p.tab, a);
+    uint64_t x = a;
+    while (x < b) {
+        const uint64_t t0 = p.tab.offs[j], t1 = p.tab.offs[j + 1];
+        const uint64_t s = (t1 - t0) / p.R;
+        unsigned short* full = static_cast<unsigned short*>(p.tab.params[j]);
+        while (x < b && x < t1) {
+            const uint64_t pos = x - t0;
+            const uint64_t r = pos / s;
+            const uint64_t k0 = pos - r * s;
+            uint64_t end = t0 + (r + 1) * s;
+            if (end > b) end = b;
+            const unsigned short* src = static_cast<const unsigned short*>(p.tab.grads[(uint64_t)j * p.R + r]);
+            const uint64_t n = end - x;
+            const bool vec = (p.tab.flags[j] & 1u) != 0u && (s & 7ull) == 0 && (k0 & 7ull) == 0;
+            if (vec) {
+                const uint64_t nv = n >> 3;
+                for (uint64_t v = threadIdx.x; v < nv; v += kThreads)
+                    __stcs(reinterpret_cast<uint4*>(full + pos) + v,
+                           __ldcs(reinterpret_cast<const uint4*>(src + k0) + v));
+                for (uint64_t e = (nv << 3) + threadIdx.x; e < n; e += kThreads) full[pos + e] = src[k0 + e];
+            } else {
+                for (uint64_t e = threadIdx.x; e < n; e += kThreads) full[pos + e] = src[k0 + e];
+            }
+            x = end;
+        }
+        ++j;
+    }
+}
+
 // ------------------------------------------------------------ micro-step accumulation
 
 struct AccumParams {

@@ -19,7 +19,7 @@ HEADER = os.path.join(ROOT, "include", "zero_adam.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(zero_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(zero3?_\w+)\s*\(", text)))
 
 
 def test_library_exports_every_declared_symbol():
@@ -196,3 +196,38 @@ def test_accumulate_argument_errors(kw, status):
     with pytest.raises(za.ZeroError) as e:
         za.zero_accumulate_grads(P, R, **args)
     assert e.value.status == status
+
+
+def test_zero3_shard_bounds_tile_each_tensor():
+    # "Stage 3 needs a live working set": shards of ceil(n/R) elements; the
+    # ranks' pieces tile [0, n) in order, the last ones possibly short or empty.
+    for n in list(range(1, 60)) + [51_463_168, 12_582_912, 2**40 + 3]:
+        for R in (1, 2, 3, 4, 7, 8, 64):
+            s = -(-n // R)
+            nxt = 0
+            for r in range(R):
+                lo, hi, sh = za.zero3_shard_bounds(n, R, r)
+                assert sh == s and lo == min(r * s, n) and hi == min((r + 1) * s, n)
+                assert lo == nxt
+                nxt = hi
+            assert nxt == n
+
+
+def test_parameter_storage_matches_the_oracle_and_the_pages():
+    from conftest import golden_rows
+    for row in golden_rows("parameter_storage.txt"):
+        sizes, ranks, live, want = [x.strip() for x in row.split("|")]
+        sizes = [int(x) for x in sizes.split(",")]
+        live = [] if live == "-" else [int(x) for x in live.split(",")]
+        assert za.zero_parameter_storage(sizes, int(ranks), live) == tuple(int(x) for x in want.split())
+    rng = random.Random(4)
+    for _ in range(200):
+        T = rng.randrange(1, 30)
+        sizes = [rng.randrange(1, 10**7) for _ in range(T)]
+        R = rng.randrange(1, 65)
+        live = rng.sample(range(T), rng.randrange(0, T + 1))
+        assert za.zero_parameter_storage(sizes, R, live) == oracle.parameter_storage(sizes, R, live)
+    for bad in [([4, 0], 2, []), ([4, 4], 2, [0, 0]), ([4, 4], 2, [2]), ([4], 0, [])]:
+        with pytest.raises(za.ZeroError) as e:
+            za.zero_parameter_storage(*bad)
+        assert e.value.status == za.ZERO_EINVAL

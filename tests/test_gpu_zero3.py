@@ -1,0 +1,82 @@
+"""ZeRO-3 on one GPU ("Stage 3 needs a live working set"): per-tensor padded
+shards, the module-level gather of full 16-bit views, and the optimizer step
+of every rank over its own shards -- which must give bitwise the same state
+and parameters as the ZeRO-2 step over the whole vector, since the update of
+an element does not depend on who owns it."""
+import pytest
+import torch
+
+import mixed_precision_adam_zero_b200 as za
+import synth
+from gpu_helpers import ADAMW_HP, grads_for_step
+from mixed_precision_adam_zero_b200.buffers import ListZero
+
+pytestmark = pytest.mark.gpu
+
+TDT = {"bf16": torch.bfloat16, "f16": torch.float16}
+CODE = {"bf16": za.ZERO_BF16, "f16": za.ZERO_F16}
+
+
+def _gather(numels, R, shards, dtype):
+    full = [torch.full((R * -(-n // R),), -1.0, dtype=TDT[dtype], device="cuda") for n in numels]
+    nb = za.zero_list_table_bytes(len(numels), R)
+    table = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    gl = za.zero3_gather_list_build(numels, full, shards, CODE[dtype], table, nb)
+    za.zero3_gather(gl)
+    torch.cuda.synchronize()
+    return full, table
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("R", [1, 3, 4, 8])
+def test_gather_is_the_concatenation_of_the_shards(dtype, R):
+    numels = [1000, 37, 4096 * 3 + 5, 2, 2048, 9, 50_000, 1]
+    shards = [[synth.normal(-(-n // R), 1.0, 1000 * r + j, device="cuda", dtype=TDT[dtype])
+               for j, n in enumerate(numels)] for r in range(R)]
+    full, _ = _gather(numels, R, shards, dtype)
+    for j in range(len(numels)):
+        want = torch.cat([shards[r][j] for r in range(R)])
+        assert torch.equal(full[j].view(torch.int16), want.view(torch.int16))
+
+
+@pytest.mark.parametrize("R", [3, 4])
+def test_rank_steps_over_shards_equal_the_whole_step(R):
+    numels = [1000, 37, 4096 * 3 + 5, 2048, 9, 50_000, 3]
+    T = len(numels)
+    whole = ListZero(numels, R, "bf16", "bf16")
+    P = whole.P
+    w0 = synth.normal(P, 0.02, 91, device="cuda")
+    whole.load_master(w0)
+    offs = [0]
+    for n in numels:
+        offs.append(offs[-1] + n)
+    bounds = [[za.zero3_shard_bounds(n, R, r) for n in numels] for r in range(R)]
+    # each rank: padded 16-bit shard buffers, and a list over its pieces whose
+    # gradients are views into every rank's full gradient (in-HBM reduce-scatter)
+    shard_bufs = [[torch.zeros(b[2], dtype=torch.bfloat16, device="cuda") for b in bounds[r]] for r in range(R)]
+    ranks = []
+    for r in range(R):
+        sizes = [hi - lo for lo, hi, _ in bounds[r]]
+        params = [shard_bufs[r][j][:sizes[j]] for j in range(T)]
+        grads = [[whole.grads[q][j][bounds[r][j][0]:bounds[r][j][1]] for j in range(T)] for q in range(R)]
+        z = ListZero(sizes, R, "bf16", "bf16", params16=params, grads=grads)
+        z.load_master(torch.cat([w0[offs[j] + lo:offs[j] + hi] for j, (lo, hi, _) in enumerate(bounds[r])]))
+        ranks.append(z)
+    for k in range(1, 4):
+        grads_for_step(91, k, whole.grads, 1e-3)
+        whole.step(hp=ADAMW_HP)
+        for z in ranks:
+            z.step(hp=ADAMW_HP)
+    torch.cuda.synchronize()
+    wm = whole.current()
+    for r, z in enumerate(ranks):
+        zm = z.current()
+        pos = 0
+        for j, (lo, hi, _) in enumerate(bounds[r]):
+            for a, b in zip(zm, wm):
+                assert torch.equal(a[pos:pos + hi - lo], b[offs[j] + lo:offs[j] + hi])
+            pos += hi - lo
+        assert z.ctrl().step == 3
+    full, _ = _gather(numels, R, shard_bufs, "bf16")
+    for j, n in enumerate(numels):
+        assert torch.equal(full[j][:n].view(torch.int16), whole.params16[j].view(torch.int16))
