@@ -54,6 +54,9 @@ GRAD_BYTES = {"bf16": 2, "f16": 2, "f32": 4}
 # update is one fused step (R = 1, fp32) over that array.
 GAS = {"flat16m_gas4": 4}
 WORKLOADS["flat16m_gas4"] = ("flat", 16_777_259, 8, "bf16", "bf16", False)
+# ZeRO-3 module gather: full padded 16-bit views of every GPT-2-medium tensor
+# from R = 4 rank shards (2 bytes read and 2 written per padded element).
+WORKLOADS["gpt2m_z3gather"] = ("z3gather", "gpt2m", 4, "bf16", "bf16", False)
 
 
 def bytes_per_param(R: int, gdt: str, gas: int = 0) -> int:
@@ -162,6 +165,27 @@ def build_workload(name: str, device):
     kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
     wl = synth.WORKLOADS.get(name.split("_")[0], 9)
     S = 65536.0 if scaled else 1.0
+    if kind == "z3gather":
+        from mixed_precision_adam_zero_b200 import ZERO_BF16, zero3_gather_list_build, zero_list_table_bytes
+        numels = [n for _, n in synth.gpt2_medium_tensors()]
+        shard = [-(-n // R) for n in numels]
+        sbufs = [torch.empty(sum(shard), dtype=torch.bfloat16, device=device) for _ in range(R)]
+        for r, sb in enumerate(sbufs):
+            synth.fill_normal_(sb, 0.02, synth.seed_for(wl, synth.KIND_MASTER, r))
+        fbuf = torch.empty(R * sum(shard), dtype=torch.bfloat16, device=device)
+        full = list(fbuf.split([R * s for s in shard]))
+        nb = zero_list_table_bytes(len(numels), R)
+        table = torch.zeros(nb, dtype=torch.uint8, device=device)
+        gl = zero3_gather_list_build(numels, full, [list(sb.split(shard)) for sb in sbufs], ZERO_BF16, table, nb)
+
+        class Z3:
+            pass
+        z = Z3()
+        z.P, z.gl, z.table, z.keep = R * sum(shard), gl, table, (sbufs, fbuf)
+        z.check, z.gbufs = False, sbufs
+        z.flat_p16 = fbuf
+        z.ctrl = lambda: type("C", (), {"step": 0})()
+        return z
     if name in GAS:
         z = FlatZero(size, 1, "f32", pdt, device=device, loss_scale=S, alloc_grads=False)
         gt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt]
@@ -196,6 +220,8 @@ def build_workload(name: str, device):
 
 
 def launches_per_step(z) -> int:
+    if hasattr(z, "gl"):
+        return 1
     if getattr(z, "gas", 0):
         return z.gas + 1
     if not z.check:
@@ -245,7 +271,10 @@ def run_gpu(args) -> None:
     stream = torch.cuda.current_stream(device)
     from mixed_precision_adam_zero_b200 import (ZERO_BF16, ZERO_F16, ZERO_F32, zero_accumulate_grads,
                                                 zero_step_fused, zero_step_fused_list)
-    if getattr(z, "gas", 0):
+    if hasattr(z, "gl"):
+        from mixed_precision_adam_zero_b200 import zero3_gather
+        call = lambda: zero3_gather(z.gl, stream)
+    elif getattr(z, "gas", 0):
         step_args = z.step_args(hp=ADAMW, check=z.check, grads=[z.accum])
         gcode = {"bf16": ZERO_BF16, "f16": ZERO_F16, "f32": ZERO_F32}[z.micro_gdt]
 
@@ -317,7 +346,7 @@ def run_gpu(args) -> None:
     if rank == 0:
         kind, size, R, gdt, pdt, scaled = WORKLOADS[args.workload]
         P = z.P
-        bpp = bytes_per_param(R, gdt, GAS.get(args.workload, 0))
+        bpp = 4 if kind == "z3gather" else bytes_per_param(R, gdt, GAS.get(args.workload, 0))
         peaks = measured_peaks()
         peak = peaks.get("hbm_gbs")
         peak_src = "measured" if peak else "fallback"
@@ -351,7 +380,8 @@ def run_gpu(args) -> None:
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
                 "traffic": traffic,
-                "kernel": ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") +
+                "kernel": "z3_gather_kernel" if kind == "z3gather" else
+                          ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") +
                           (" (flat)" if kind == "flat" else " (list)"),
                 "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms,
             },
