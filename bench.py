@@ -39,6 +39,8 @@ WORKLOADS = {
     "flat1p5b": ("flat", 1_500_000_000, 4, "bf16", "bf16", False),
     "flat1p5b_f32": ("flat", 1_500_000_000, 4, "f32", "bf16", False),
     "llama3b": ("list", "llama3b", 8, "bf16", "bf16", False),
+    # the fp16 case with one state set: overflow scan first, then the step
+    "gpt2m_inplace": ("list", "gpt2m", 4, "f16", "f16", True),
     # bandwidth sweep of the flat kernel, R = 8 bf16
     "sweep1m": ("flat", 1 << 20, 8, "bf16", "bf16", False),
     "sweep4m": ("flat", 1 << 22, 8, "bf16", "bf16", False),
@@ -165,6 +167,7 @@ def build_workload(name: str, device):
     kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
     wl = synth.WORKLOADS.get(name.split("_")[0], 9)
     S = 65536.0 if scaled else 1.0
+    two_set = scaled and not name.endswith("_inplace")
     if kind == "z3gather":
         from mixed_precision_adam_zero_b200 import ZERO_BF16, zero3_gather_list_build, zero_list_table_bytes
         numels = [n for _, n in synth.gpt2_medium_tensors()]
@@ -200,7 +203,7 @@ def build_workload(name: str, device):
         z.micro_R, z.micro_gdt = R, gdt
         return z
     if kind == "flat":
-        z = FlatZero(size, R, gdt, pdt, device=device, loss_scale=S, two_set=scaled)
+        z = FlatZero(size, R, gdt, pdt, device=device, loss_scale=S, two_set=two_set)
         gbufs = z.grads
     else:
         tensors = synth.gpt2_medium_tensors() if size == "gpt2m" else synth.llama_3b_tensors()
@@ -208,7 +211,7 @@ def build_workload(name: str, device):
         gt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
         gbufs = [torch.empty(sum(numels), dtype=gt[gdt], device=device) for _ in range(R)]
         pbuf = torch.empty(sum(numels), dtype=gt[pdt], device=device)
-        z = ListZero(numels, R, gdt, pdt, device=device, loss_scale=S, two_set=scaled,
+        z = ListZero(numels, R, gdt, pdt, device=device, loss_scale=S, two_set=two_set,
                      params16=list(pbuf.split(numels)), grads=[list(g.split(numels)) for g in gbufs])
         z.flat_p16 = pbuf
     z.load_master(synth.normal(z.P, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device))
@@ -226,7 +229,7 @@ def launches_per_step(z) -> int:
         return z.gas + 1
     if not z.check:
         return 1
-    return 2  # two-set single pass + the restore kernel (a no-op unless skipped)
+    return 2  # two-set: the pass + a restore kernel (no-op unless skipped); one set: a scan + the pass
 
 
 # ------------------------------------------------------------ ranks

@@ -507,9 +507,16 @@ __device__ __forceinline__ void scan_range(const G* g, uint64_t a, uint64_t b, b
         if (vb < va) vb = va;
     }
     for (uint64_t e = a + threadIdx.x; e < va; e += kThreads) (void)load1<G>(g, e, bad);
-    for (uint64_t e = va + (uint64_t)threadIdx.x * kVec; e < vb; e += (uint64_t)kThreads * kVec)
-        bad |= bad8(load8<G>(g, e));
-    for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads) (void)load1<G>(g, e, bad);
+    // four independent 16-byte loads in flight per thread per iteration
+    constexpr uint64_t kStride = (uint64_t)kThreads * kVec;
+    uint64_t e = va + (uint64_t)threadIdx.x * kVec;
+    for (; e + 3 * kStride < vb; e += 4 * kStride) {
+        const Raw8<G> r0 = load8<G>(g, e), r1 = load8<G>(g, e + kStride);
+        const Raw8<G> r2 = load8<G>(g, e + 2 * kStride), r3 = load8<G>(g, e + 3 * kStride);
+        bad |= bad8(r0) | bad8(r1) | bad8(r2) | bad8(r3);
+    }
+    for (; e < vb; e += kStride) bad |= bad8(load8<G>(g, e));
+    for (uint64_t x = vb + threadIdx.x; x < b; x += kThreads) (void)load1<G>(g, x, bad);
 }
 
 // Sets ws.found if any gradient of any rank in [lo, hi) is inf or NaN.
