@@ -639,9 +639,18 @@ __global__ void __launch_bounds__(kThreads) z3_gather_kernel(const __grid_consta
             const bool vec = (p.tab.flags[j] & 1u) != 0u && (s & 7ull) == 0 && (k0 & 7ull) == 0;
             if (vec) {
                 const uint64_t nv = n >> 3;
-                for (uint64_t v = threadIdx.x; v < nv; v += kThreads)
-                    __stcs(reinterpret_cast<uint4*>(full + pos) + v,
-                           __ldcs(reinterpret_cast<const uint4*>(src + k0) + v));
+                const uint4* in = reinterpret_cast<const uint4*>(src + k0);
+                uint4* out = reinterpret_cast<uint4*>(full + pos);
+                uint64_t v = threadIdx.x;
+                for (; v + 3 * kThreads < nv; v += 4 * kThreads) {  // four copies in flight
+                    const uint4 x0 = __ldcs(in + v), x1 = __ldcs(in + v + kThreads);
+                    const uint4 x2 = __ldcs(in + v + 2 * kThreads), x3 = __ldcs(in + v + 3 * kThreads);
+                    __stcs(out + v, x0);
+                    __stcs(out + v + kThreads, x1);
+                    __stcs(out + v + 2 * kThreads, x2);
+                    __stcs(out + v + 3 * kThreads, x3);
+                }
+                for (; v < nv; v += kThreads) __stcs(out + v, __ldcs(in + v));
                 for (uint64_t e = (nv << 3) + threadIdx.x; e < n; e += kThreads) full[pos + e] = src[k0 + e];
             } else {
                 for (uint64_t e = threadIdx.x; e < n; e += kThreads) full[pos + e] = src[k0 + e];
@@ -665,43 +674,66 @@ struct AccumParams {
     int32_t first;                      // 1: acc starts from zero
 };
 
-// acc = (first ? 0 : acc) + scale * (sum_r w_r g_r) / sum(w), float64, one rounding.
-template <class G, int RC>
-__device__ __forceinline__ void accum_vec(const AccumParams& p, const GradPtrs<G, RC>& gp, uint64_t e) {
-    double acc[8];
+// acc = (first ? 0 : acc) + scale * (sum_r w_r g_r) / sum(w), float64, one
+// rounding, for U vectors at e, e + stride, ...: every load of the U vectors
+// is issued before any arithmetic or store.  (U = 2 measured slower than
+// U = 1 on a B200: the extra registers cost resident CTAs.)
+template <class G, int RC, int U>
+__device__ __forceinline__ void accum_vec(const AccumParams& p, const GradPtrs<G, RC>& gp, uint64_t e,
+                                          uint64_t stride) {
+    float4 a0[U], a1[U];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) acc[k] = 0.0;
-    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+    for (int u = 0; u < U; ++u) {
+        a0[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        a1[u] = a0[u];
+    }
     if (!p.first) {
-        a0 = __ldcs(reinterpret_cast<const float4*>(p.acc + e));
-        a1 = __ldcs(reinterpret_cast<const float4*>(p.acc + e + 4));
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            a0[u] = __ldcs(reinterpret_cast<const float4*>(p.acc + e + u * stride));
+            a1[u] = __ldcs(reinterpret_cast<const float4*>(p.acc + e + u * stride + 4));
+        }
     }
-    const int R = RC > 0 ? RC : (int)p.R;
+    double acc[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[u][k] = 0.0;
     if constexpr (RC > 0) {
-        Raw8<G> raw[RC];
+        Raw8<G> raw[U][RC];
 #pragma unroll
-        for (int r = 0; r < RC; ++r) raw[r] = load8<G>(gp[r], e);
+        for (int u = 0; u < U; ++u)
 #pragma unroll
-        for (int r = 0; r < RC; ++r) {
-            float f[8];
-            unpack8(raw[r], f);
+            for (int r = 0; r < RC; ++r) raw[u][r] = load8<G>(gp[r], e + u * stride);
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = fma(p.wt[r], (double)f[k], acc[k]);
-        }
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+            for (int r = 0; r < RC; ++r) {
+                float f[8];
+                unpack8(raw[u][r], f);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[u][k] = fma(p.wt[r], (double)f[k], acc[u][k]);
+            }
     } else {
-        for (int r = 0; r < R; ++r) {
-            float f[8];
-            unpack8(load8<G>(gp[r], e), f);
+        for (int r = 0; r < (int)p.R; ++r) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = fma(p.wt[r], (double)f[k], acc[k]);
+            for (int u = 0; u < U; ++u) {
+                float f[8];
+                unpack8(load8<G>(gp[r], e + u * stride), f);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[u][k] = fma(p.wt[r], (double)f[k], acc[u][k]);
+            }
         }
     }
-    const float prev[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-    float out[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) out[k] = (float)((double)prev[k] + p.scale * (acc[k] * p.inv_wsum));
-    __stcs(reinterpret_cast<float4*>(p.acc + e), make_float4(out[0], out[1], out[2], out[3]));
-    __stcs(reinterpret_cast<float4*>(p.acc + e + 4), make_float4(out[4], out[5], out[6], out[7]));
+    for (int u = 0; u < U; ++u) {
+        const float prev[8] = {a0[u].x, a0[u].y, a0[u].z, a0[u].w, a1[u].x, a1[u].y, a1[u].z, a1[u].w};
+        float out[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) out[k] = (float)((double)prev[k] + p.scale * (acc[u][k] * p.inv_wsum));
+        __stcs(reinterpret_cast<float4*>(p.acc + e + u * stride), make_float4(out[0], out[1], out[2], out[3]));
+        __stcs(reinterpret_cast<float4*>(p.acc + e + u * stride + 4), make_float4(out[4], out[5], out[6], out[7]));
+    }
 }
 
 template <class G, int RC>
@@ -728,9 +760,10 @@ __global__ void __launch_bounds__(kThreads) accum_kernel(const __grid_constant__
     if (va > b) va = b;
     if (vb < va) vb = va;
     for (uint64_t e = a + threadIdx.x; e < va; e += kThreads) accum_elem<G, RC>(p, gp, e);
-    for (uint64_t e = va + (uint64_t)threadIdx.x * kVec; e < vb; e += (uint64_t)kThreads * kVec)
-        accum_vec<G, RC>(p, gp, e);
-    for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads) accum_elem<G, RC>(p, gp, e);
+    constexpr uint64_t kStride = (uint64_t)kThreads * kVec;
+    uint64_t e = va + (uint64_t)threadIdx.x * kVec;
+    for (; e < vb; e += kStride) accum_vec<G, RC, 1>(p, gp, e, kStride);
+    for (uint64_t x = vb + threadIdx.x; x < b; x += kThreads) accum_elem<G, RC>(p, gp, x);
 }
 
 // ------------------------------------------------------------ control block
