@@ -41,6 +41,9 @@ WORKLOADS = {
     "llama3b": ("list", "llama3b", 8, "bf16", "bf16", False),
     # the fp16 case with one state set: overflow scan first, then the step
     "gpt2m_inplace": ("list", "gpt2m", 4, "f16", "f16", True),
+    # GPT-2-medium's embeddings and first layer only (14 tensors, 65M
+    # parameters, about 2 GB on the device): a small case of the list kernel
+    "gpt2m_head": ("list", "gpt2m_head", 4, "f16", "f16", True),
     # bandwidth sweep of the flat kernel, R = 8 bf16
     "sweep1m": ("flat", 1 << 20, 8, "bf16", "bf16", False),
     "sweep4m": ("flat", 1 << 22, 8, "bf16", "bf16", False),
@@ -206,7 +209,8 @@ def build_workload(name: str, device):
         z = FlatZero(size, R, gdt, pdt, device=device, loss_scale=S, two_set=two_set)
         gbufs = z.grads
     else:
-        tensors = synth.gpt2_medium_tensors() if size == "gpt2m" else synth.llama_3b_tensors()
+        tensors = {"gpt2m": synth.gpt2_medium_tensors, "gpt2m_head": lambda: synth.gpt2_medium_tensors()[:14],
+                   "llama3b": synth.llama_3b_tensors}[size]()
         numels = [n for _, n in tensors]
         gt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
         gbufs = [torch.empty(sum(numels), dtype=gt[gdt], device=device) for _ in range(R)]

@@ -110,48 +110,18 @@ Kern bulk_kern() {
 
 template <class G, class Pm, bool LIST>
 Kern step_kern_rc(uint32_t R) {
-#ifndef ZADAM_REGISTER_PATH_ONLY
     switch (R) {
         case 1: return bulk_kern<G, Pm, 1, LIST>();
         case 2: return bulk_kern<G, Pm, 2, LIST>();
         case 4: return bulk_kern<G, Pm, 4, LIST>();
         case 8: return bulk_kern<G, Pm, 8, LIST>();
-        default: break;
+        default: return Kern{(const void*)step_kernel<G, Pm, 0, LIST>, 0u, kThreads};
     }
-#endif
-    return Kern{(const void*)step_kernel<G, Pm, 0, LIST>, 0u, kThreads};
 }
 
 template <class G, bool LIST>
 Kern step_kern_pm(int32_t param_dtype, uint32_t R) {
     return param_dtype == ZERO_BF16 ? step_kern_rc<G, __nv_bfloat16, LIST>(R) : step_kern_rc<G, __half, LIST>(R);
-}
-
-Kern step_kern(bool list, int32_t grad_dtype, int32_t param_dtype, uint32_t R);
-
-template <class G, class Pm, bool LIST>
-const void* step_fn_rc(uint32_t R) {
-    switch (R) {
-        case 1: return (const void*)step_kernel<G, Pm, 1, LIST>;
-        case 2: return (const void*)step_kernel<G, Pm, 2, LIST>;
-        case 4: return (const void*)step_kernel<G, Pm, 4, LIST>;
-        case 8: return (const void*)step_kernel<G, Pm, 8, LIST>;
-        default: return (const void*)step_kernel<G, Pm, 0, LIST>;
-    }
-}
-
-template <class G, bool LIST>
-const void* step_fn_pm(int32_t param_dtype, uint32_t R) {
-    return param_dtype == ZERO_BF16 ? step_fn_rc<G, __nv_bfloat16, LIST>(R) : step_fn_rc<G, __half, LIST>(R);
-}
-
-template <bool LIST>
-const void* step_fn(int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
-    switch (grad_dtype) {
-        case ZERO_F32: return step_fn_pm<float, LIST>(param_dtype, R);
-        case ZERO_BF16: return step_fn_pm<__nv_bfloat16, LIST>(param_dtype, R);
-        default: return step_fn_pm<__half, LIST>(param_dtype, R);
-    }
 }
 
 template <bool LIST>
@@ -164,12 +134,7 @@ Kern step_kern_gd(int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
 }
 
 Kern step_kern(bool list, int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
-#ifdef ZADAM_REGISTER_PATH_ONLY
-    return Kern{list ? step_fn<true>(grad_dtype, param_dtype, R) : step_fn<false>(grad_dtype, param_dtype, R), 0u,
-                kThreads};
-#else
     return list ? step_kern_gd<true>(grad_dtype, param_dtype, R) : step_kern_gd<false>(grad_dtype, param_dtype, R);
-#endif
 }
 
 template <bool LIST>

@@ -643,14 +643,14 @@ __global__ void __launch_bounds__(kThreads) z3_gather_kernel(const __grid_consta
                 uint4* out = reinterpret_cast<uint4*>(full + pos);
                 uint64_t v = threadIdx.x;
                 for (; v + 3 * kThreads < nv; v += 4 * kThreads) {  // four copies in flight
-                    const uint4 x0 = __ldcs(in + v), x1 = __ldcs(in + v + kThreads);
-                    const uint4 x2 = __ldcs(in + v + 2 * kThreads), x3 = __ldcs(in + v + 3 * kThreads);
-                    __stcs(out + v, x0);
-                    __stcs(out + v + kThreads, x1);
-                    __stcs(out + v + 2 * kThreads, x2);
-                    __stcs(out + v + 3 * kThreads, x3);
+                    const uint4 x0 = in[v], x1 = in[v + kThreads];
+                    const uint4 x2 = in[v + 2 * kThreads], x3 = in[v + 3 * kThreads];
+                    out[v] = x0;
+                    out[v + kThreads] = x1;
+                    out[v + 2 * kThreads] = x2;
+                    out[v + 3 * kThreads] = x3;
                 }
-                for (; v < nv; v += kThreads) __stcs(out + v, __ldcs(in + v));
+                for (; v < nv; v += kThreads) out[v] = in[v];
                 for (uint64_t e = (nv << 3) + threadIdx.x; e < n; e += kThreads) full[pos + e] = src[k0 + e];
             } else {
                 for (uint64_t e = threadIdx.x; e < n; e += kThreads) full[pos + e] = src[k0 + e];
