@@ -226,6 +226,20 @@ def build_workload(name: str, device):
     return z
 
 
+def roofline_kernel(workload: str) -> str:
+    """The kernel (or, for accumulation, the launch sequence of one step) the
+    roofline fraction is measured on."""
+    kind, size, R, gdt, pdt, scaled = WORKLOADS[workload]
+    if kind == "z3gather":
+        return "z3_gather_kernel"
+    step = ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") + (" (flat)" if kind == "flat" else " (list)")
+    gas = GAS.get(workload, 0)
+    if gas:
+        acc = "accum_bulk_kernel" if R in (1, 2, 4, 8) else "accum_kernel"
+        return f"{gas} x {acc} + step_bulk_kernel (flat, R = 1 f32)"
+    return step
+
+
 def launches_per_step(z) -> int:
     if hasattr(z, "gl"):
         return 1
@@ -276,19 +290,21 @@ def run_gpu(args) -> None:
 
     z = build_workload(args.workload, device)
     stream = torch.cuda.current_stream(device)
-    from mixed_precision_adam_zero_b200 import (ZERO_BF16, ZERO_F16, ZERO_F32, zero_accumulate_grads,
-                                                zero_step_fused, zero_step_fused_list)
+    from mixed_precision_adam_zero_b200 import (ZERO_BF16, ZERO_F16, ZERO_F32, make_accum_args,
+                                                zero_accumulate_grads, zero_step_fused, zero_step_fused_list)
     if hasattr(z, "gl"):
         from mixed_precision_adam_zero_b200 import zero3_gather
         call = lambda: zero3_gather(z.gl, stream)
     elif getattr(z, "gas", 0):
         step_args = z.step_args(hp=ADAMW, check=z.check, grads=[z.accum])
         gcode = {"bf16": ZERO_BF16, "f16": ZERO_F16, "f32": ZERO_F32}[z.micro_gdt]
+        micro_args = [make_accum_args(z.P, z.micro_R, grad_dtype=gcode, grads=z.micro, accum=z.accum,
+                                      scale=1.0 / z.gas, first=(mu == 0), workspace=z.workspace,
+                                      ctrl=z.ctrl_buf) for mu in range(z.gas)]
 
         def call():
-            for mu in range(z.gas):
-                zero_accumulate_grads(z.P, z.micro_R, grad_dtype=gcode, grads=z.micro, accum=z.accum,
-                                      scale=1.0 / z.gas, first=(mu == 0), stream=stream)
+            for a in micro_args:
+                zero_accumulate_grads(a, stream=stream)
             zero_step_fused(step_args, stream)
     elif hasattr(z, "list"):
         step_args = z.step_args(hp=ADAMW, check=z.check)
@@ -387,9 +403,7 @@ def run_gpu(args) -> None:
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
                 "traffic": traffic,
-                "kernel": "z3_gather_kernel" if kind == "z3gather" else
-                          ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") +
-                          (" (flat)" if kind == "flat" else " (list)"),
+                "kernel": roofline_kernel(args.workload),
                 "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms,
             },
             "e2e": {

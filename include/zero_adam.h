@@ -322,10 +322,23 @@ typedef struct zero_accum_args {
     const double *rank_weights;  /* HOST array of R weights, or NULL (equal) */
     float *accum;                /* device [P] fp32 accumulation array */
     double scale;                /* finite */
+    void *workspace;             /* NULL, or a device workspace as in
+                                    zero_step_args (all zero on entry, left
+                                    all zero; not shared with a launch that
+                                    may overlap this one on the GPU) */
+    void *ctrl;                  /* NULL iff workspace is NULL; else a device
+                                    zero_ctrl whose device_error receives a
+                                    device-side wait timeout (nothing else of
+                                    it is read or written) */
 } zero_accum_args;
 
-/* Launches one kernel; asynchronous on `stream`.  Errors: ZERO_EINVAL,
- * ZERO_EALIGN (pointers must be 16-byte aligned), ZERO_ERANGE, ZERO_EOVERFLOW,
+/* Launches one kernel; asynchronous on `stream`.  With a workspace and
+ * R = 1, 2, 4 or 8 the kernel stages its tiles in shared memory by bulk
+ * copies and hands them out dynamically (the faster path); otherwise, and
+ * always for other R, it streams through registers and touches neither.
+ * Both give bitwise identical sums.  Errors: ZERO_EINVAL (also: exactly one
+ * of workspace and ctrl given), ZERO_EALIGN (accum, grads and workspace must
+ * be 16-byte aligned, ctrl 8-byte aligned), ZERO_ERANGE, ZERO_EOVERFLOW,
  * ZERO_ECUDA. */
 int zero_accumulate_grads(const zero_accum_args *args, void *stream);
 

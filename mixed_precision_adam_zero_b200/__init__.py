@@ -87,7 +87,7 @@ class zero_accum_args(ctypes.Structure):
                 ("grad_dtype", ctypes.c_int32), ("first", ctypes.c_int32),
                 ("grads", ctypes.POINTER(ctypes.c_void_p)),
                 ("rank_weights", ctypes.POINTER(ctypes.c_double)), ("accum", ctypes.c_void_p),
-                ("scale", ctypes.c_double)]
+                ("scale", ctypes.c_double), ("workspace", ctypes.c_void_p), ("ctrl", ctypes.c_void_p)]
 
 
 class zero_tensor_list(ctypes.Structure):
@@ -293,22 +293,36 @@ def zero_gather_params_list(master, lst: zero_tensor_list, stream=None) -> None:
            "zero_gather_params_list")
 
 
-def zero_accumulate_grads(P: int, R: int, *, grad_dtype: int, grads: Sequence, accum, scale: float,
-                          first: bool, rank_weights: Optional[Sequence[float]] = None, owner: int = -1,
-                          stream=None) -> None:
-    """One micro-batch into the fp32 accumulation array (see the C declaration)."""
+def make_accum_args(P: int, R: int, *, grad_dtype: int, grads: Sequence, accum, scale: float, first: bool,
+                    rank_weights: Optional[Sequence[float]] = None, owner: int = -1, workspace=None,
+                    ctrl=None) -> zero_accum_args:
+    """Fill a zero_accum_args (the returned struct keeps its host arrays alive)."""
     a = zero_accum_args()
     a.P, a.R, a.owner, a.grad_dtype, a.first = P, R, owner, grad_dtype, int(bool(first))
     arr = (ctypes.c_void_p * len(grads))(*[_ptr(g) for g in grads])
+    a._grads_keep = arr
     a.grads = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
-    keep = [arr]
     if rank_weights is not None:
         w = (ctypes.c_double * len(rank_weights))(*[float(x) for x in rank_weights])
-        keep.append(w)
+        a._weights_keep = w
         a.rank_weights = ctypes.cast(w, ctypes.POINTER(ctypes.c_double))
     a.accum = _ptr(accum)
     a.scale = float(scale)
-    _check(_lib().zero_accumulate_grads(ctypes.byref(a), _stream(stream)), "zero_accumulate_grads")
+    a.workspace, a.ctrl = _ptr(workspace), _ptr(ctrl)
+    return a
+
+
+def zero_accumulate_grads(args, R: Optional[int] = None, *, stream=None, **kw) -> None:
+    """One micro-batch into the fp32 accumulation array (see the C declaration).
+
+    `args` is a zero_accum_args from make_accum_args, or P, followed by R and
+    make_accum_args' keywords.  With `workspace` and `ctrl` (device buffers as
+    for a step call) the shared-memory staged kernel runs for R in 1, 2, 4, 8."""
+    if not isinstance(args, zero_accum_args):
+        args = make_accum_args(args, R, **kw)
+    elif R is not None or kw:
+        raise TypeError("a zero_accum_args takes no further arguments")
+    _check(_lib().zero_accumulate_grads(ctypes.byref(args), _stream(stream)), "zero_accumulate_grads")
 
 
 def zero_checkpoint_save(path: str, args: zero_step_args, stream=None) -> None:

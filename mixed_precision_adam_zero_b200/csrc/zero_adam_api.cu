@@ -152,22 +152,38 @@ const void* gather_fn(int32_t param_dtype) {
                                     : (const void*)gather_kernel<__half, LIST>;
 }
 
+// Accumulation: the bulk kernel for a compile-time rank count when the
+// caller gives a workspace, else the register kernel.
+template <class G, int RC>
+Kern accum_bulk_kern() {
+    return Kern{(const void*)accum_bulk_kernel<G, RC>, AccumShape<G, RC>::kSmem, kBulkThreads};
+}
+
 template <class G>
-const void* accum_fn_rc(uint32_t R) {
+Kern accum_kern_rc(uint32_t R, bool bulk) {
+    if (bulk) {
+        switch (R) {
+            case 1: return accum_bulk_kern<G, 1>();
+            case 2: return accum_bulk_kern<G, 2>();
+            case 4: return accum_bulk_kern<G, 4>();
+            case 8: return accum_bulk_kern<G, 8>();
+            default: break;
+        }
+    }
     switch (R) {
-        case 1: return (const void*)accum_kernel<G, 1>;
-        case 2: return (const void*)accum_kernel<G, 2>;
-        case 4: return (const void*)accum_kernel<G, 4>;
-        case 8: return (const void*)accum_kernel<G, 8>;
-        default: return (const void*)accum_kernel<G, 0>;
+        case 1: return Kern{(const void*)accum_kernel<G, 1>, 0u, kThreads};
+        case 2: return Kern{(const void*)accum_kernel<G, 2>, 0u, kThreads};
+        case 4: return Kern{(const void*)accum_kernel<G, 4>, 0u, kThreads};
+        case 8: return Kern{(const void*)accum_kernel<G, 8>, 0u, kThreads};
+        default: return Kern{(const void*)accum_kernel<G, 0>, 0u, kThreads};
     }
 }
 
-const void* accum_fn(int32_t grad_dtype, uint32_t R) {
+Kern accum_kern(int32_t grad_dtype, uint32_t R, bool bulk) {
     switch (grad_dtype) {
-        case ZERO_F32: return accum_fn_rc<float>(R);
-        case ZERO_BF16: return accum_fn_rc<__nv_bfloat16>(R);
-        default: return accum_fn_rc<__half>(R);
+        case ZERO_F32: return accum_kern_rc<float>(R, bulk);
+        case ZERO_BF16: return accum_kern_rc<__nv_bfloat16>(R, bulk);
+        default: return accum_kern_rc<__half>(R, bulk);
     }
 }
 
@@ -461,6 +477,8 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     if (a->P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
     if (a->P > 0 && a->accum == nullptr) return ZERO_EINVAL;
     if (!aligned16(a->accum)) return ZERO_EALIGN;
+    if ((a->workspace == nullptr) != (a->ctrl == nullptr)) return ZERO_EINVAL;
+    if (!aligned16(a->workspace) || (reinterpret_cast<uintptr_t>(a->ctrl) & 7u) != 0) return ZERO_EALIGN;
     AccumParams ap;
     std::memset(&ap, 0, sizeof ap);
     double wsum = 0.0;
@@ -477,6 +495,8 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     ap.inv_wsum = 1.0 / wsum;
     ap.scale = a->scale;
     ap.acc = a->accum;
+    ap.ws = static_cast<Workspace*>(a->workspace);
+    ap.ctrl = static_cast<zero_ctrl*>(a->ctrl);
     ap.R = a->R;
     ap.first = a->first;
     if (a->owner < 0) {
@@ -489,13 +509,13 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     }
     if (ap.lo >= ap.hi) return ZERO_OK;
     int err = ZERO_OK;
-    const void* fn = accum_fn(a->grad_dtype, a->R);
-    const int ctas = resident_ctas(fn, &err);
+    const Kern k = accum_kern(a->grad_dtype, a->R, a->workspace != nullptr);
+    const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;
     const Shape sh = make_shape(ap.lo, ap.hi, ctas);
     ap.base = sh.base;
     ap.chunk = sh.chunk;
-    return launch(fn, sh, &ap, static_cast<cudaStream_t>(stream));
+    return launch(k.fn, sh, &ap, static_cast<cudaStream_t>(stream), k.smem, k.threads);
 }
 
 int zero_step_fused_noalloc(const zero_step_args* a, void* stream) {

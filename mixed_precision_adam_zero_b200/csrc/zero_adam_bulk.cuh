@@ -333,14 +333,74 @@ __device__ __forceinline__ StateIO state_io(const StepParams& p) {
     return StateIO{p.w[par], p.m[par], p.v[par], p.w[out], p.m[out], p.v[out]};
 }
 
-// Flat call: tiles are handed out dynamically.  The launch's vector body
-// [round_up(lo, 8), round_down(hi, 8)) is cut into kTile-element tiles, and
-// each CTA's producer claims the next one from a counter in the workspace,
-// one claim ahead of use so the atomic's latency overlaps the copies.  All
-// CTAs then finish within about one tile of each other, whatever the speed
-// of their SM.  The tile id travels to the consumers in a per-stage slot,
-// written before the stage's barrier is armed; kEndTile marks the end.
+// Flat calls: tiles are handed out dynamically.  The launch's vector body
+// [va, vb) is cut into kTile-element tiles, and each CTA's producer claims
+// the next one from a counter in the workspace, one claim ahead of use so
+// the atomic's latency overlaps the copies.  All CTAs then finish within
+// about one tile of each other, whatever the speed of their SM.  The tile id
+// travels to the consumers in a per-stage slot, written before the stage's
+// barrier is armed; kEndTile marks the end.
 constexpr uint32_t kEndTile = 0xFFFFFFFFu;
+
+__device__ __forceinline__ uint32_t flat_tile_count(uint64_t va, uint64_t vb) {
+    return va < vb ? (uint32_t)((vb - va + kTile - 1) / kTile) : 0u;
+}
+
+// Producer side (one thread): `issue(st, e0, n)` arms full[st] and starts
+// the copies of the tile [e0, e0 + n) into stage st.
+template <int D, class Issue>
+__device__ __forceinline__ void flat_produce(Workspace* ws, uint64_t va, uint64_t vb, uint64_t* full,
+                                             uint64_t* empty, uint32_t* slot, Issue&& issue) {
+    const uint32_t ntiles = flat_tile_count(va, vb);
+    uint32_t next = atomicAdd(&ws->next_tile, 1u);
+    uint32_t k = 0;
+    bool ok = true;
+    for (;; ++k) {
+        const int st = (int)(k % D);
+        if (k >= (uint32_t)D && !mbar_wait_bounded(&empty[st], ((k / D) - 1u) & 1u)) {
+            ok = false;
+            break;
+        }
+        const uint32_t tile = next;
+        if (tile >= ntiles) {
+            slot[st] = kEndTile;
+            mbar_arrive(&full[st]);
+            break;
+        }
+        next = atomicAdd(&ws->next_tile, 1u);
+        slot[st] = tile;
+        const uint64_t e0 = va + (uint64_t)tile * kTile;
+        const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
+        issue(st, e0, n);
+    }
+    if (!ok) {
+        // Do not leave while copies of this CTA may still land in its shared
+        // memory: wait (bounded) for the last tile of every stage.
+        atomicOr(&ws->error, 1u);
+        for (uint32_t j = k > (uint32_t)D ? k - D : 0u; j < k; ++j)
+            (void)mbar_wait_bounded(&full[j % D], (j / D) & 1u);
+    }
+}
+
+// Consumer side (every consumer thread): `consume(st, e0, n)` reads stage st.
+template <int D, class Consume>
+__device__ __forceinline__ void flat_consume(Workspace* ws, uint64_t va, uint64_t vb, uint64_t* full,
+                                             uint64_t* empty, const uint32_t* slot, Consume&& consume) {
+    for (uint32_t k = 0;; ++k) {
+        const int st = (int)(k % D);
+        if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
+            atomicOr(&ws->error, 1u);
+            break;
+        }
+        const uint32_t tile = slot[st];
+        if (tile == kEndTile) break;
+        const uint64_t e0 = va + (uint64_t)tile * kTile;
+        const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
+        consume(st, e0, n);
+        __syncwarp();
+        if ((threadIdx.x & 31u) == 0u) mbar_arrive(&empty[st]);
+    }
+}
 
 template <class G, class Pm, int RC>
 __device__ __forceinline__ void flat_dynamic(const StepParams& p, uint64_t* full, uint64_t* empty,
@@ -349,58 +409,23 @@ __device__ __forceinline__ void flat_dynamic(const StepParams& p, uint64_t* full
     constexpr int D = Sh::kStages;
     const uint64_t va = (p.lo + 7) & ~7ull;
     const uint64_t vb = p.hi & ~7ull;
-    const uint32_t ntiles = va < vb ? (uint32_t)((vb - va + kTile - 1) / kTile) : 0u;
     if (threadIdx.x == kConsumers) {
         const StateIO io = state_io(p);
         const G* gb[RC];
 #pragma unroll
         for (int r = 0; r < RC; ++r) gb[r] = static_cast<const G*>(p.grads[r]);
-        uint32_t next = atomicAdd(&p.ws->next_tile, 1u);
-        uint32_t k = 0;
-        bool ok = true;
-        for (;; ++k) {
-            const int st = (int)(k % D);
-            if (k >= (uint32_t)D && !mbar_wait_bounded(&empty[st], ((k / D) - 1u) & 1u)) {
-                ok = false;
-                break;
-            }
-            const uint32_t tile = next;
-            if (tile >= ntiles) {
-                slot[st] = kEndTile;
-                mbar_arrive(&full[st]);
-                break;
-            }
-            next = atomicAdd(&p.ws->next_tile, 1u);
-            slot[st] = tile;
-            const uint64_t e0 = va + (uint64_t)tile * kTile;
-            const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
+        flat_produce<D>(p.ws, va, vb, full, empty, slot, [&](int st, uint64_t e0, uint32_t n) {
             bulk_issue<G, RC>(io, gb, ring + st * Sh::kStage, &full[st], e0, e0, n);
-        }
-        if (!ok) {
-            atomicOr(&p.ws->error, 1u);
-            for (uint32_t j = k > (uint32_t)D ? k - D : 0u; j < k; ++j)
-                (void)mbar_wait_bounded(&full[j % D], (j / D) & 1u);
-        }
+        });
     } else if (threadIdx.x < kConsumers) {
         const StateIO io = state_io(p);
         const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
         Pm* pp = static_cast<Pm*>(p.params16);
-        for (uint32_t k = 0;; ++k) {
-            const int st = (int)(k % D);
-            if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
-                atomicOr(&p.ws->error, 1u);
-                break;
-            }
-            const uint32_t tile = slot[st];
-            if (tile == kEndTile) break;
-            const uint64_t e0 = va + (uint64_t)tile * kTile;
-            const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
+        flat_consume<D>(p.ws, va, vb, full, empty, slot, [&](int st, uint64_t e0, uint32_t n) {
             const unsigned char* stage = ring + st * Sh::kStage;
             for (uint32_t q = 4u * threadIdx.x; q < n; q += 4u * kConsumers)
                 bulk_group<G, Pm, RC>(p, s, stage, q, e0 + q, e0 + q, io.wo, io.mo, io.vo, pp, bad);
-            __syncwarp();
-            if ((threadIdx.x & 31u) == 0u) mbar_arrive(&empty[st]);
-        }
+        });
     }
 }
 
@@ -626,6 +651,122 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
         }
     }
     finish_step(p, bad);
+}
+
+// ------------------------------------------------------------ micro-step accumulation
+
+// Stage of the accumulation kernel: [R gradient slices][acc slice]; the acc
+// slice is loaded only when the window continues (first == 0).
+template <class G, int RC>
+struct AccumShape {
+    static constexpr uint32_t kGradSlice = kTile * sizeof(G);
+    static constexpr uint32_t kStage = RC * kGradSlice + kTile * 4u;
+    static constexpr int kBudget = 200 * 1024;
+    static constexpr int kStages = (kBudget / kStage) > 8 ? 8 : (kBudget / kStage);
+    static constexpr uint32_t kSmem = kBarBytes + kGpBytes + kStages * kStage;
+    static_assert(kStages >= 2, "stage too large for the ring");
+    static_assert(kStage % 1024 == 0, "stages must stay 1024-byte aligned");
+};
+
+// Four consecutive elements at flat index e (offset q in the stage): the
+// arithmetic of accum_vec, element for element, so the register and the
+// bulk kernels give bitwise identical sums.
+template <class G, int RC>
+__device__ __forceinline__ void accum_group(const AccumParams& p, const unsigned char* stage, uint32_t q,
+                                            uint64_t e) {
+    using Sh = AccumShape<G, RC>;
+    Raw4<G> raw[RC];
+#pragma unroll
+    for (int r = 0; r < RC; ++r) raw[r] = lds4<G>(stage + r * Sh::kGradSlice + q * sizeof(G));
+    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!p.first) a4 = *reinterpret_cast<const float4*>(stage + RC * Sh::kGradSlice + q * 4u);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int r = 0; r < RC; ++r) {
+        float f[4];
+        unpack4(raw[r], f);
+        const double c = p.wt[r];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[k] = fma(c, (double)f[k], acc[k]);
+    }
+    const float prev[4] = {a4.x, a4.y, a4.z, a4.w};
+    float out[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) out[k] = (float)((double)prev[k] + p.scale * (acc[k] * p.inv_wsum));
+    __stcs(reinterpret_cast<float4*>(p.acc + e), make_float4(out[0], out[1], out[2], out[3]));
+}
+
+// Last CTA to finish: move a wait timeout into ctrl->device_error and leave
+// the workspace ready for the next launch.
+__device__ __forceinline__ void finish_accum(const AccumParams& p) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        Workspace* ws = p.ws;
+        __threadfence();
+        const unsigned prev = atomicAdd(&ws->arrive, 1u);
+        if (prev == gridDim.x - 1) {
+            __threadfence();
+            const unsigned err = atomicOr(&ws->error, 0u);
+            if (err) p.ctrl->device_error = err;
+            ws->error = 0u;
+            ws->next_tile = 0u;
+            ws->arrive = 0u;
+            __threadfence();
+        }
+    }
+}
+
+// acc[lo, hi) = (first ? 0 : acc) + scale * (sum_r w_r g_r) / sum(w), with
+// the tiles of the vector body streamed through the shared-memory ring and
+// handed out dynamically, as in the flat step; CTA 0 takes the ragged ends.
+template <class G, int RC>
+__global__ void __launch_bounds__(kBulkThreads, 1) accum_bulk_kernel(const __grid_constant__ AccumParams p) {
+    using Sh = AccumShape<G, RC>;
+    constexpr int D = Sh::kStages;
+    constexpr uint32_t kConsumerWarps = kConsumers / 32;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = reinterpret_cast<uint64_t*>(smem + 64);
+    uint32_t* slot = reinterpret_cast<uint32_t*>(smem + 128);
+    unsigned char* ring = smem + kBarBytes + kGpBytes;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < D; ++i) {
+            mbar_init(&full[i], 1u);
+            mbar_init(&empty[i], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const uint64_t va = (p.lo + 7) & ~7ull;
+    const uint64_t vb = p.hi & ~7ull;
+    if (threadIdx.x == kConsumers) {
+        const G* gb[RC];
+#pragma unroll
+        for (int r = 0; r < RC; ++r) gb[r] = static_cast<const G*>(p.grads[r]);
+        const bool load_acc = !p.first;
+        flat_produce<D>(p.ws, va, vb, full, empty, slot, [&](int st, uint64_t e0, uint32_t n) {
+            unsigned char* stage = ring + st * Sh::kStage;
+            const uint32_t gbytes = n * (uint32_t)sizeof(G);
+            mbar_expect_tx(&full[st], RC * gbytes + (load_acc ? n * 4u : 0u));
+#pragma unroll
+            for (int r = 0; r < RC; ++r) bulk_g2s(stage + r * Sh::kGradSlice, gb[r] + e0, gbytes, &full[st]);
+            if (load_acc) bulk_g2s(stage + RC * Sh::kGradSlice, p.acc + e0, n * 4u, &full[st]);
+        });
+    } else if (threadIdx.x < kConsumers) {
+        flat_consume<D>(p.ws, va, vb, full, empty, slot, [&](int st, uint64_t e0, uint32_t n) {
+            const unsigned char* stage = ring + st * Sh::kStage;
+            for (uint32_t q = 4u * threadIdx.x; q < n; q += 4u * kConsumers) accum_group<G, RC>(p, stage, q, e0 + q);
+        });
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        const GradPtrs<G, RC> gp(&p.grads[0]);
+        uint64_t ha = va > p.hi ? p.hi : va;
+        uint64_t tb = vb < ha ? ha : vb;
+        for (uint64_t e = p.lo + threadIdx.x; e < ha; e += kBulkThreads) accum_elem<G, RC>(p, gp, e);
+        for (uint64_t e = tb + threadIdx.x; e < p.hi; e += kBulkThreads) accum_elem<G, RC>(p, gp, e);
+    }
+    finish_accum(p);
 }
 
 }  // namespace zadam

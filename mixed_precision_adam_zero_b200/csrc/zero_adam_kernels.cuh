@@ -669,6 +669,8 @@ struct AccumParams {
     double inv_wsum;                    // 1 / sum(w)
     double scale;                       // multiplies the reduced gradient
     float* acc;                         // fp32 accumulation array [P]
+    Workspace* ws;                      // bulk kernel: tile counter and error flag
+    zero_ctrl* ctrl;                    // bulk kernel: receives device_error
     uint64_t lo, hi, base, chunk;
     uint32_t R;
     int32_t first;                      // 1: acc starts from zero

@@ -188,6 +188,10 @@ def test_noalloc_step_refuses_a_caller_workspace():
     (dict(grads=[A, A + 2, A, A]), za.ZERO_EALIGN),
     (dict(rank_weights=[1, 1, -1, 1]), za.ZERO_EINVAL),
     (dict(P=2**62), za.ZERO_EOVERFLOW),
+    (dict(workspace=A), za.ZERO_EINVAL),            # a workspace needs a ctrl
+    (dict(ctrl=A), za.ZERO_EINVAL),                 # and a ctrl a workspace
+    (dict(workspace=A + 8, ctrl=A), za.ZERO_EALIGN),
+    (dict(workspace=A, ctrl=A + 4), za.ZERO_EALIGN),
 ])
 def test_accumulate_argument_errors(kw, status):
     args = dict(P=1000, R=4, grad_dtype=za.ZERO_BF16, grads=[A] * 4, accum=A, scale=0.25, first=True)

@@ -18,9 +18,12 @@ pytestmark = pytest.mark.gpu
 DT = {"bf16": za.ZERO_BF16, "f16": za.ZERO_F16, "f32": za.ZERO_F32}
 
 
-def _run(P, R, gdt, gas, updates, token=True, S0=1.0, check=False, bad=None, two_set=False, seed=51):
-    """`updates` optimizer steps of `gas` micro-batches each."""
+def _run(P, R, gdt, gas, updates, token=True, S0=1.0, check=False, bad=None, two_set=False, seed=51, staged=True):
+    """`updates` optimizer steps of `gas` micro-batches each; `staged`: the
+    accumulation gets the step's workspace and ctrl (shared-memory staged
+    kernel for R in 1, 2, 4, 8), else none (register kernel)."""
     z = FlatZero(P, 1, "f32", "bf16", two_set=two_set, loss_scale=S0, alloc_grads=False)
+    ws = dict(workspace=z.workspace, ctrl=z.ctrl_buf) if staged else {}
     acc = torch.zeros(P, dtype=torch.float32, device="cuda")
     micro = [torch.zeros(P, dtype={"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt],
                          device="cuda") for _ in range(R)]
@@ -35,7 +38,7 @@ def _run(P, R, gdt, gas, updates, token=True, S0=1.0, check=False, bad=None, two
                 micro[1][P // 2] = math.inf
             wts = [float(x) for x in synth.token_counts(R, seed, 100 * u + mu)] if token else None
             za.zero_accumulate_grads(P, R, grad_dtype=DT[gdt], grads=micro, accum=acc, scale=1.0 / gas,
-                                     first=(mu == 0), rank_weights=wts)
+                                     first=(mu == 0), rank_weights=wts, **ws)
             oracle.accumulate(oacc, [host_grad(g) for g in micro], gdt, 1.0 / gas, first=(mu == 0), weights=wts)
         torch.cuda.synchronize()
         assert_close(acc, oacc.astype(np.float64), f"accumulated gradient, update {u}")
@@ -44,17 +47,86 @@ def _run(P, R, gdt, gas, updates, token=True, S0=1.0, check=False, bad=None, two
         assert bool(z.ctrl().last_skipped) == skipped
     torch.cuda.synchronize()
     compare_full(z, st, z.params16)
+    assert z.ctrl().device_error == 0
+    assert not z.workspace.any()
     return z, st
 
 
-@pytest.mark.parametrize("gdt,R", [("bf16", 8), ("bf16", 4), ("f16", 4), ("f32", 4), ("bf16", 3), ("bf16", 1)])
-def test_accumulate_then_step(gdt, R):
-    _run(P=60_013, R=R, gdt=gdt, gas=4, updates=3)
+@pytest.mark.parametrize("staged", [True, False])
+@pytest.mark.parametrize("gdt,R", [("bf16", 8), ("bf16", 4), ("f16", 4), ("f32", 4), ("f32", 8), ("bf16", 3),
+                                   ("bf16", 2), ("bf16", 1)])
+def test_accumulate_then_step(gdt, R, staged):
+    _run(P=60_013, R=R, gdt=gdt, gas=4, updates=3, staged=staged)
 
 
-def test_accumulate_equal_weights_ragged_sizes():
-    for P in (1, 7, 2049, 100_003):
-        _run(P=P, R=8, gdt="bf16", gas=2, updates=2, token=False)
+@pytest.mark.parametrize("staged", [True, False])
+def test_accumulate_equal_weights_ragged_sizes(staged):
+    # 2048-element tiles: one tile, a tile and one element, several tiles and
+    # a ragged tail, and sizes below one vector of 8.
+    for P in (1, 7, 2048, 2049, 3 * 2048 + 13, 100_003):
+        _run(P=P, R=8, gdt="bf16", gas=2, updates=2, token=False, staged=staged)
+
+
+def _micro(P, R, dt, seed):
+    return [synth.normal(P, 1e-3, seed + r, device="cuda", dtype=dt) for r in range(R)]
+
+
+@pytest.mark.parametrize("gdt", ["bf16", "f16", "f32"])
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+def test_staged_and_register_kernels_agree_bitwise(gdt, R):
+    tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt]
+    P = 37 * 2048 + 5
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ctrl = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    staged = torch.full((P,), 0.25, device="cuda")
+    plain = staged.clone()
+    wts = [float(x) for x in synth.token_counts(R, 5, R)]
+    for mu, first in enumerate((True, False, False)):
+        g = _micro(P, R, tdt, 300 + 10 * mu)
+        za.zero_accumulate_grads(P, R, grad_dtype=DT[gdt], grads=g, accum=staged, scale=1 / 3, first=first,
+                                 rank_weights=wts, workspace=ws, ctrl=ctrl)
+        za.zero_accumulate_grads(P, R, grad_dtype=DT[gdt], grads=g, accum=plain, scale=1 / 3, first=first,
+                                 rank_weights=wts)
+    torch.cuda.synchronize()
+    assert torch.equal(staged.view(torch.int32), plain.view(torch.int32))
+    assert not ws.any() and not ctrl.any()
+
+
+def test_staged_per_owner_equals_whole_bitwise():
+    P, R = 9 * 2048 + 77, 4
+    g = _micro(P, R, torch.bfloat16, 90)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ctrl = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    whole = torch.full((P,), -1.5, device="cuda")
+    part = whole.clone()
+    for first in (True, False):
+        za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=g, accum=whole, scale=0.5, first=first)
+        for r in range(R):
+            za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=g, accum=part, scale=0.5, first=first,
+                                     owner=r, workspace=ws, ctrl=ctrl)
+    torch.cuda.synchronize()
+    assert torch.equal(whole.view(torch.int32), part.view(torch.int32))
+    assert not ws.any() and not ctrl.any()
+
+
+def test_staged_accumulation_full_size_against_the_oracle():
+    # The accumulation of the 16,777,259-parameter, R = 8 bf16 workload in
+    # the benchmark's launch configuration: two micro-batches, every element
+    # against the oracle.
+    P, R = 16_777_259, 8
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ctrl = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    acc = torch.empty(P, device="cuda")
+    oacc = np.zeros(P, dtype=np.float32)
+    for mu in range(2):
+        g = _micro(P, R, torch.bfloat16, 500 + 10 * mu)
+        wts = [float(x) for x in synth.token_counts(R, 6, mu)]
+        za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=g, accum=acc, scale=0.5, first=(mu == 0),
+                                 rank_weights=wts, workspace=ws, ctrl=ctrl)
+        oracle.accumulate(oacc, [host_grad(x) for x in g], "bf16", 0.5, first=(mu == 0), weights=wts)
+    torch.cuda.synchronize()
+    assert_close(acc, oacc.astype(np.float64), "full-size accumulated gradient")
+    assert not ws.any() and not ctrl.any()
 
 
 @pytest.mark.parametrize("two_set", [False, True])
