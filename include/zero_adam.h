@@ -224,6 +224,16 @@ int zero_ctrl_read(const void *ctrl, zero_ctrl *out, void *stream);
 /* Zero a workspace of ZERO_WORKSPACE_BYTES (cudaMemsetAsync). */
 int zero_workspace_init(void *workspace, void *stream);
 
+/* Health check of the device-side timeout path (the pages have no
+ * counterpart): launches one block whose thread waits, through the same
+ * bounded wait as the staged kernels, on a shared-memory barrier that nothing
+ * arrives at.  The wait gives up after its limit (about 2 s of GPU time) and
+ * the kernel sets ctrl->device_error to 1, then exits normally: no trap, no
+ * fault, the context stays usable.  Asynchronous on `stream`; read the
+ * result with zero_ctrl_read.  Errors: ZERO_EINVAL (NULL ctrl), ZERO_EALIGN
+ * (ctrl not 8-byte aligned), ZERO_ECUDA. */
+int zero_selftest_wait_timeout(void *ctrl, void *stream);
+
 /* ------------------------------------------------------------- the step */
 
 /* One fused ZeRO-2/3 optimizer step over a flat parameter vector:

@@ -41,7 +41,7 @@ EXPORTED = [
     "zero_ctrl_bytes", "zero_workspace_bytes", "zero_list_table_bytes", "zero_ctrl_init",
     "zero_ctrl_set", "zero_ctrl_read", "zero_workspace_init", "zero_step_fused",
     "zero_step_fused_list", "zero_list_table_build", "zero_gather_params",
-    "zero_gather_params_list", "zero_step_fused_noalloc", "zero_accumulate_grads",
+    "zero_gather_params_list", "zero_step_fused_noalloc", "zero_accumulate_grads", "zero_selftest_wait_timeout",
     "zero_checkpoint_save", "zero_checkpoint_load", "zero_checkpoint_consolidate", "zero_checkpoint_error",
     "zero3_shard_bounds", "zero_parameter_storage", "zero3_gather_list_build", "zero3_gather",
 ]
@@ -122,6 +122,7 @@ def _lib() -> ctypes.CDLL:
         L.zero_ctrl_set.argtypes = [vp, ctypes.POINTER(zero_ctrl), vp]
         L.zero_ctrl_read.argtypes = [vp, ctypes.POINTER(zero_ctrl), vp]
         L.zero_workspace_init.argtypes = [vp, vp]
+        L.zero_selftest_wait_timeout.argtypes = [vp, vp]
         L.zero_step_fused.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_step_fused_noalloc.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_accumulate_grads.argtypes = [ctypes.POINTER(zero_accum_args), vp]
@@ -223,6 +224,12 @@ def zero_ctrl_read(ctrl, stream=None) -> zero_ctrl:
 
 def zero_workspace_init(workspace, stream=None) -> None:
     _check(_lib().zero_workspace_init(_ptr(workspace), _stream(stream)), "zero_workspace_init")
+
+
+def zero_selftest_wait_timeout(ctrl, stream=None) -> None:
+    """Run the device-side timeout path once: sets ctrl.device_error to 1
+    after about 2 s of GPU time (see the C declaration)."""
+    _check(_lib().zero_selftest_wait_timeout(_ptr(ctrl), _stream(stream)), "zero_selftest_wait_timeout")
 
 
 def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master, exp_avg, exp_avg_sq,

@@ -432,6 +432,14 @@ int zero_ctrl_read(const void* ctrl, zero_ctrl* out, void* stream) {
     return e == cudaSuccess ? ZERO_OK : zadam_record_cuda(e);
 }
 
+int zero_selftest_wait_timeout(void* ctrl, void* stream) {
+    if (ctrl == nullptr) return ZERO_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(ctrl) & 7u) != 0) return ZERO_EALIGN;
+    Shape sh{0, 0, 1};
+    zero_ctrl* c = static_cast<zero_ctrl*>(ctrl);
+    return launch((const void*)wait_timeout_probe_kernel, sh, &c, static_cast<cudaStream_t>(stream), 0, 32);
+}
+
 int zero_workspace_init(void* workspace, void* stream) {
     if (workspace == nullptr) return ZERO_EINVAL;
     if (!aligned16(workspace)) return ZERO_EALIGN;

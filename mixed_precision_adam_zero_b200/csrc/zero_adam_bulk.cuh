@@ -1,27 +1,28 @@
-// zero_adam_bulk.cuh -- the step (flat buffer or tensor list) with
-// shared-memory staging by 1-D bulk asynchronous copies (the TMA engine's
-// cp.async.bulk, no tensor map, no multicast).
+// zero_adam_bulk.cuh -- the step (flat buffer or tensor list) and the
+// micro-step accumulation with shared-memory staging by 1-D bulk
+// asynchronous copies (the TMA engine's cp.async.bulk, no tensor map, no
+// multicast).
 //
-// Why: the register-staged kernel holds each thread's loads in registers, so
+// Why: the register-staged kernels hold each thread's loads in registers, so
 // the bytes a SM keeps in flight are bounded by registers x resident warps.
-// Here one thread per CTA streams tiles of every input array (R gradient
-// slices and the master, m and v slices) into a ring of shared-memory
-// stages, several tiles ahead of the 256 threads that consume them; the bytes
-// in flight are set by the ring size (about 170 KB per SM), not by registers.
+// Here one producer thread per CTA streams tiles of every input array (R
+// gradient slices and the master, m and v slices) into a ring of
+// shared-memory stages, several tiles ahead of the consumer warps; the bytes
+// in flight are set by the ring size (up to 200 KB per SM), not by
+// registers.
 //
 // Per tile of n <= kTile elements (n a multiple of 8, every source 16-byte
 // aligned): stage = [R gradient slices][w][m][v], each slice contiguous.
-// Thread t of the 512 consumes the 4 elements [4t, 4t+4), so every
-// shared-memory read is conflict-free and every global store is coalesced.
-// Sixteen consumer warps per SM keep the per-tile arithmetic (a float64
-// reduction, an IEEE divide and square root per element) well below the
-// tile's DRAM time; with eight the two were close and the kernel lost ~10 %.  The arithmetic per element is exactly
+// Consumer thread t handles the 4-element groups [4t, 4t+4), [4t + 4C, ...)
+// (C consumer threads), so every shared-memory read is conflict-free and
+// every global store is coalesced.  The arithmetic per element is exactly
 // that of step_kernel (adam1 and the float64 rank reduction), so the two
 // kernels give bitwise identical results.
 //
 // Waits on the stage barriers are bounded (by %globaltimer): a wait that
-// gives up records an error in the workspace, the CTA stops consuming, waits
-// (again bounded) for the copies it issued, and finishes normally.
+// gives up marks the CTA as timed out, the CTA stops consuming, waits (again
+// bounded) for the copies it issued, and finishes normally; the grid's
+// epilogue then sets zero_ctrl.device_error.
 #pragma once
 
 #include "zero_adam_kernels.cuh"
@@ -38,6 +39,12 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr int kBarBytes = 384;                  // full and empty stage barriers (at most 2 x 8 x 8 B), padded
 constexpr int kGpBytes = 640;                   // gradient bases of a tensor (scalar pass of a list);
                                                 // pads the header so the stage ring starts 1024-B aligned
+
+// Set to 1 by any thread of the CTA whose bounded wait gave up; thread 0
+// clears it before the CTA's first wait and folds it into the arrival.
+static __shared__ unsigned int s_timed_out;
+
+__device__ __forceinline__ void note_timeout() { s_timed_out = 1u; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -334,9 +341,10 @@ __device__ __forceinline__ StateIO state_io(const StepParams& p) {
 }
 
 // Flat calls: tiles are handed out dynamically.  The launch's vector body
-// [va, vb) is cut into kTile-element tiles, and each CTA's producer claims
-// the next one from a counter in the workspace, one claim ahead of use so
-// the atomic's latency overlaps the copies.  All CTAs then finish within
+// [va, vb) is cut into kTile-element tiles.  CTA b starts on tile b without
+// asking anyone; after that each CTA's producer claims the next tile from a
+// counter in the workspace (claims number the tiles from gridDim.x on), one
+// claim ahead of use so the atomic's latency overlaps the copies.  All CTAs then finish within
 // about one tile of each other, whatever the speed of their SM.  The tile id
 // travels to the consumers in a per-stage slot, written before the stage's
 // barrier is armed; kEndTile marks the end.
@@ -352,7 +360,7 @@ template <int D, class Issue>
 __device__ __forceinline__ void flat_produce(Workspace* ws, uint64_t va, uint64_t vb, uint64_t* full,
                                              uint64_t* empty, uint32_t* slot, Issue&& issue) {
     const uint32_t ntiles = flat_tile_count(va, vb);
-    uint32_t next = atomicAdd(&ws->next_tile, 1u);
+    uint32_t next = blockIdx.x;
     uint32_t k = 0;
     bool ok = true;
     for (;; ++k) {
@@ -367,7 +375,7 @@ __device__ __forceinline__ void flat_produce(Workspace* ws, uint64_t va, uint64_
             mbar_arrive(&full[st]);
             break;
         }
-        next = atomicAdd(&ws->next_tile, 1u);
+        next = gridDim.x + atomicAdd(&ws->next_tile, 1u);
         slot[st] = tile;
         const uint64_t e0 = va + (uint64_t)tile * kTile;
         const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
@@ -376,7 +384,7 @@ __device__ __forceinline__ void flat_produce(Workspace* ws, uint64_t va, uint64_
     if (!ok) {
         // Do not leave while copies of this CTA may still land in its shared
         // memory: wait (bounded) for the last tile of every stage.
-        atomicOr(&ws->error, 1u);
+        note_timeout();
         for (uint32_t j = k > (uint32_t)D ? k - D : 0u; j < k; ++j)
             (void)mbar_wait_bounded(&full[j % D], (j / D) & 1u);
     }
@@ -389,7 +397,7 @@ __device__ __forceinline__ void flat_consume(Workspace* ws, uint64_t va, uint64_
     for (uint32_t k = 0;; ++k) {
         const int st = (int)(k % D);
         if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
-            atomicOr(&ws->error, 1u);
+            note_timeout();
             break;
         }
         const uint32_t tile = slot[st];
@@ -443,8 +451,9 @@ struct TileDesc {
 // take the vector path) is [offs[j], round_down(offs[j+1], 8)); the bodies
 // are cut into kTile tiles, numbered across tensors (tab.tiles holds the
 // running count), and handed out dynamically like the flat call's tiles.
-// Tile ids a producer claims only grow, so it finds each tile's tensor by
-// scanning forward from the previous one.
+// As for flat calls, CTA b starts on tile b and claims the rest.  Tile ids
+// a producer gets only grow, so it finds each tile's tensor by scanning
+// forward from the previous one.
 template <class G, class Pm, int RC>
 __device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full, uint64_t* empty,
                                              TileDesc* desc, unsigned char* ring, bool& bad) {
@@ -459,7 +468,7 @@ __device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full
         uint32_t jn = 0;           // scan position
         uint64_t t0 = 0, bb = 0, tfirst = 0;
         void* params = nullptr;
-        uint64_t next = atomicAdd(&p.ws->next_tile, 1u);
+        uint64_t next = blockIdx.x;
         if (next < ntiles) jn = find_tensor_by_tile(t, next);
         uint32_t k = 0;
         bool ok = true;
@@ -475,7 +484,7 @@ __device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full
                 mbar_arrive(&full[st]);
                 break;
             }
-            next = atomicAdd(&p.ws->next_tile, 1u);
+            next = (uint64_t)gridDim.x + atomicAdd(&p.ws->next_tile, 1u);
             while (t.tiles[jn + 1] <= tile) ++jn;
             if (jn != j) {
                 j = jn;
@@ -492,7 +501,7 @@ __device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full
             bulk_issue<G, RC>(io, gb, ring + st * Sh::kStage, &full[st], e0, e0 - t0, n);
         }
         if (!ok) {
-            atomicOr(&p.ws->error, 1u);
+            note_timeout();
             for (uint32_t i = k > (uint32_t)D ? k - D : 0u; i < k; ++i)
                 (void)mbar_wait_bounded(&full[i % D], (i / D) & 1u);
         }
@@ -502,7 +511,7 @@ __device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full
         for (uint32_t k = 0;; ++k) {
             const int st = (int)(k % D);
             if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
-                atomicOr(&p.ws->error, 1u);
+                note_timeout();
                 break;
             }
             const TileDesc d = desc[st];
@@ -572,7 +581,7 @@ __device__ __forceinline__ void list_static(const StepParams& p, uint64_t a, uin
         if (!ok) {
             // Do not leave while copies of this CTA may still land in its
             // shared memory: wait (bounded) for the last tile of every stage.
-            atomicOr(&p.ws->error, 1u);
+            note_timeout();
             for (uint32_t j = k > (uint32_t)D ? k - D : 0u; j < k; ++j)
                 (void)mbar_wait_bounded(&full[j % D], (j / D) & 1u);
         }
@@ -586,7 +595,7 @@ __device__ __forceinline__ void list_static(const StepParams& p, uint64_t a, uin
         for (uint32_t k = 0; cw.next(p, e0, n); ++k) {
             const int st = (int)(k % D);
             if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
-                atomicOr(&p.ws->error, 1u);
+                note_timeout();
                 break;
             }
             const unsigned char* stage = ring + st * Sh::kStage;
@@ -616,6 +625,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
     uint64_t b = a + p.chunk;
     if (a < p.lo) a = p.lo;
     if (b > p.hi) b = p.hi;
+    if (threadIdx.x == 0) s_timed_out = 0u;
     bool skip = false;
     if (p.check == 2) skip = *reinterpret_cast<volatile const unsigned*>(&p.ws->found) != 0u;
     bool bad = false;
@@ -650,7 +660,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
             bulk_scalar_pass<G, Pm, RC, false>(p, s, p.lo, p.hi, io, bad, s_gp);
         }
     }
-    finish_step(p, bad);
+    finish_step(p, bad, s_timed_out != 0u);
 }
 
 // ------------------------------------------------------------ micro-step accumulation
@@ -696,22 +706,19 @@ __device__ __forceinline__ void accum_group(const AccumParams& p, const unsigned
     __stcs(reinterpret_cast<float4*>(p.acc + e), make_float4(out[0], out[1], out[2], out[3]));
 }
 
-// Last CTA to finish: move a wait timeout into ctrl->device_error and leave
-// the workspace ready for the next launch.
+// Last CTA to finish: record a wait timeout in ctrl->device_error and leave
+// the workspace ready for the next launch (the packed arrival of
+// finish_step, without the found field).
 __device__ __forceinline__ void finish_accum(const AccumParams& p) {
     __syncthreads();
     if (threadIdx.x == 0) {
         Workspace* ws = p.ws;
-        __threadfence();
-        const unsigned prev = atomicAdd(&ws->arrive, 1u);
-        if (prev == gridDim.x - 1) {
-            __threadfence();
-            const unsigned err = atomicOr(&ws->error, 0u);
-            if (err) p.ctrl->device_error = err;
-            ws->error = 0u;
+        const unsigned long long mine = Arrival::mine(false, s_timed_out != 0u);
+        const unsigned long long all = atomicAdd(&ws->arrive, mine) + mine;
+        if (Arrival::count(all) == gridDim.x) {
+            if (Arrival::any_timeout(all)) p.ctrl->device_error = 1u;
             ws->next_tile = 0u;
-            ws->arrive = 0u;
-            __threadfence();
+            ws->arrive = 0ull;
         }
     }
 }
@@ -730,6 +737,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) accum_bulk_kernel(const __gri
     uint32_t* slot = reinterpret_cast<uint32_t*>(smem + 128);
     unsigned char* ring = smem + kBarBytes + kGpBytes;
     if (threadIdx.x == 0) {
+        s_timed_out = 0u;
         for (int i = 0; i < D; ++i) {
             mbar_init(&full[i], 1u);
             mbar_init(&empty[i], kConsumerWarps);
@@ -767,6 +775,19 @@ __global__ void __launch_bounds__(kBulkThreads, 1) accum_bulk_kernel(const __gri
         for (uint64_t e = tb + threadIdx.x; e < p.hi; e += kBulkThreads) accum_elem<G, RC>(p, gp, e);
     }
     finish_accum(p);
+}
+
+// ------------------------------------------------------------ timeout health check
+
+// One thread waits on a barrier that nothing arrives at; the bounded wait
+// gives up and the kernel records the timeout as the staged kernels do.
+__global__ void wait_timeout_probe_kernel(zero_ctrl* c) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1u);
+        fence_mbar_init();
+        if (!mbar_wait_bounded(&bar, 0u)) c->device_error = 1u;
+    }
 }
 
 }  // namespace zadam

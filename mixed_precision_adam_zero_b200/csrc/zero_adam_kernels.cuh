@@ -41,13 +41,32 @@ constexpr int kVec = 8;        // elements per vector
 
 // Scratch of one step call (ZERO_WORKSPACE_BYTES).  All zero between calls.
 struct Workspace {
-    unsigned int arrive;     // CTAs of the running launch that have finished
-    unsigned int found;      // nonzero: some gradient was inf or NaN
-    unsigned int error;      // nonzero: a bounded device-side wait gave up
-    unsigned int next_tile;  // flat bulk step: the next tile to hand out
+    unsigned long long arrive;  // CTAs of the running launch that have finished, packed (see Arrival)
+    unsigned int found;         // two-pass check: the scan kernel saw an inf or NaN
+    unsigned int next_tile;     // dynamic tiles: claims made so far
     unsigned int pad[60];
 };
 static_assert(sizeof(Workspace) == ZERO_WORKSPACE_BYTES, "workspace size");
+
+// A CTA's arrival adds 1 to the count field, and 1 to the found field if it
+// saw an inf or NaN, and 1 to the timeout field if one of its bounded waits
+// gave up.  One 64-bit atomic carries all three, so the CTA that completes
+// the count knows the whole grid's flags from the value its own atomic
+// returns, with no fence and no second read (a grid has < 2^21 CTAs).
+struct Arrival {
+    static constexpr int kBits = 21;
+    static constexpr unsigned long long kMask = (1ull << kBits) - 1ull;
+    static constexpr unsigned long long kFound = 1ull << kBits;
+    static constexpr unsigned long long kTimeout = 1ull << (2 * kBits);
+    static __device__ __forceinline__ unsigned long long mine(bool found, bool timeout) {
+        return 1ull | (found ? kFound : 0ull) | (timeout ? kTimeout : 0ull);
+    }
+    static __device__ __forceinline__ unsigned long long count(unsigned long long v) { return v & kMask; }
+    static __device__ __forceinline__ bool any_found(unsigned long long v) { return ((v >> kBits) & kMask) != 0ull; }
+    static __device__ __forceinline__ bool any_timeout(unsigned long long v) {
+        return ((v >> (2 * kBits)) & kMask) != 0ull;
+    }
+};
 
 struct Hyper {
     float b1, b2, omb1, omb2, eps, lr_wd;  // float32 per-element constants
@@ -411,17 +430,19 @@ __device__ __forceinline__ uint32_t find_tensor_by_tile(const Table& t, uint64_t
     return lo;
 }
 
-// Grid-level epilogue: the last CTA to finish updates the control block.
-__device__ __forceinline__ void finish_step(const StepParams& p, bool bad) {
+// Grid-level epilogue: the last CTA to finish updates the control block and
+// clears the workspace for the next launch.  Every other access to the
+// control block and the workspace in this launch happened before the
+// accessing CTA's arrival, and the next launch sees the writes at the kernel
+// boundary.  Only thread 0's `timed_out` is used.
+__device__ __forceinline__ void finish_step(const StepParams& p, bool bad, bool timed_out = false) {
     const int any = __syncthreads_or(bad ? 1 : 0);
     if (threadIdx.x == 0) {
         Workspace* ws = p.ws;
-        if (any) atomicOr(&ws->found, 1u);
-        __threadfence();
-        const unsigned prev = atomicAdd(&ws->arrive, 1u);
-        if (prev == gridDim.x - 1) {
-            __threadfence();
-            const unsigned found = p.check ? atomicOr(&ws->found, 0u) : 0u;
+        const unsigned long long mine = Arrival::mine(any != 0, timed_out);
+        const unsigned long long all = atomicAdd(&ws->arrive, mine) + mine;
+        if (Arrival::count(all) == gridDim.x) {
+            const bool found = p.check == 1 ? Arrival::any_found(all) : (p.check == 2 && ws->found != 0u);
             zero_ctrl* c = p.ctrl;
             if (found) {
                 c->loss_scale *= 0.5f;
@@ -441,13 +462,10 @@ __device__ __forceinline__ void finish_step(const StepParams& p, bool bad) {
                     c->growth_tracker = gt;
                 }
             }
-            const unsigned err = atomicOr(&ws->error, 0u);
-            if (err) c->device_error = err;
+            if (Arrival::any_timeout(all)) c->device_error = 1u;
             ws->found = 0u;
-            ws->error = 0u;
             ws->next_tile = 0u;
-            ws->arrive = 0u;
-            __threadfence();
+            ws->arrive = 0ull;
         }
     }
 }

@@ -165,6 +165,13 @@ def test_gather_and_ctrl_argument_errors():
         assert e.value.status == status
 
 
+def test_wait_timeout_selftest_argument_errors():
+    for ctrl, status in ((None, za.ZERO_EINVAL), (A + 4, za.ZERO_EALIGN)):
+        with pytest.raises(za.ZeroError) as e:
+            za.zero_selftest_wait_timeout(ctrl)
+        assert e.value.status == status
+
+
 def test_list_table_bytes():
     T, R = 292, 4
     assert za.zero_list_table_bytes(T, R) == 8 * (T + 1) + 8 * T + 8 * T * R + ((4 * T + 15) // 16) * 16 + 8 * (T + 1)
