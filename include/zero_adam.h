@@ -340,16 +340,25 @@ typedef struct zero_accum_args {
                                     zero_ctrl whose device_error receives a
                                     device-side wait timeout (nothing else of
                                     it is read or written) */
+    int32_t path;                /* ZERO_PATH_AUTO (0), ZERO_PATH_REGISTER or
+                                    ZERO_PATH_STAGED (see below) */
 } zero_accum_args;
 
-/* Launches one kernel; asynchronous on `stream`.  With a workspace and
- * R = 1, 2, 4 or 8 the kernel stages its tiles in shared memory by bulk
- * copies and hands them out dynamically (the faster path); otherwise, and
- * always for other R, it streams through registers and touches neither.
- * Both give bitwise identical sums.  Errors: ZERO_EINVAL (also: exactly one
- * of workspace and ctrl given), ZERO_EALIGN (accum, grads and workspace must
- * be 16-byte aligned, ctrl 8-byte aligned), ZERO_ERANGE, ZERO_EOVERFLOW,
- * ZERO_ECUDA. */
+#define ZERO_PATH_AUTO 0
+#define ZERO_PATH_REGISTER 1
+#define ZERO_PATH_STAGED 2
+
+/* Launches one kernel; asynchronous on `stream`.  The staged kernel stages
+ * its tiles in shared memory by bulk copies and hands them out dynamically;
+ * it needs a workspace and ctrl and R = 1, 2, 4 or 8.  The register kernel
+ * streams through registers and touches neither workspace nor ctrl.  Both
+ * give bitwise identical sums.  ZERO_PATH_AUTO takes the staged kernel when
+ * it is possible and the launch's range holds at least 12*2^20 elements
+ * (where it is the faster one), else the register kernel.  Errors:
+ * ZERO_EINVAL (also: exactly one of workspace and ctrl given; an unknown
+ * path; ZERO_PATH_STAGED without a workspace or with another R),
+ * ZERO_EALIGN (accum, grads and workspace must be 16-byte aligned, ctrl
+ * 8-byte aligned), ZERO_ERANGE, ZERO_EOVERFLOW, ZERO_ECUDA. */
 int zero_accumulate_grads(const zero_accum_args *args, void *stream);
 
 /* ------------------------------------------------------------------ ZeRO-3 */

@@ -35,6 +35,7 @@ ZERO_F16 = 2
 ZERO_MAX_RANKS = 256
 ZERO_WORKSPACE_BYTES = 256
 ZERO_NOALLOC_SCRATCH_BYTES = 256
+ZERO_PATH_AUTO, ZERO_PATH_REGISTER, ZERO_PATH_STAGED = 0, 1, 2
 
 EXPORTED = [
     "zero_partition_bounds", "zero_state_bytes", "zero_status_string", "zero_last_cuda_error",
@@ -87,7 +88,8 @@ class zero_accum_args(ctypes.Structure):
                 ("grad_dtype", ctypes.c_int32), ("first", ctypes.c_int32),
                 ("grads", ctypes.POINTER(ctypes.c_void_p)),
                 ("rank_weights", ctypes.POINTER(ctypes.c_double)), ("accum", ctypes.c_void_p),
-                ("scale", ctypes.c_double), ("workspace", ctypes.c_void_p), ("ctrl", ctypes.c_void_p)]
+                ("scale", ctypes.c_double), ("workspace", ctypes.c_void_p), ("ctrl", ctypes.c_void_p),
+                ("path", ctypes.c_int32)]
 
 
 class zero_tensor_list(ctypes.Structure):
@@ -302,7 +304,7 @@ def zero_gather_params_list(master, lst: zero_tensor_list, stream=None) -> None:
 
 def make_accum_args(P: int, R: int, *, grad_dtype: int, grads: Sequence, accum, scale: float, first: bool,
                     rank_weights: Optional[Sequence[float]] = None, owner: int = -1, workspace=None,
-                    ctrl=None) -> zero_accum_args:
+                    ctrl=None, path: int = ZERO_PATH_AUTO) -> zero_accum_args:
     """Fill a zero_accum_args (the returned struct keeps its host arrays alive)."""
     a = zero_accum_args()
     a.P, a.R, a.owner, a.grad_dtype, a.first = P, R, owner, grad_dtype, int(bool(first))
@@ -316,6 +318,7 @@ def make_accum_args(P: int, R: int, *, grad_dtype: int, grads: Sequence, accum, 
     a.accum = _ptr(accum)
     a.scale = float(scale)
     a.workspace, a.ctrl = _ptr(workspace), _ptr(ctrl)
+    a.path = path
     return a
 
 
@@ -324,7 +327,8 @@ def zero_accumulate_grads(args, R: Optional[int] = None, *, stream=None, **kw) -
 
     `args` is a zero_accum_args from make_accum_args, or P, followed by R and
     make_accum_args' keywords.  With `workspace` and `ctrl` (device buffers as
-    for a step call) the shared-memory staged kernel runs for R in 1, 2, 4, 8."""
+    for a step call) the shared-memory staged kernel can run for R in 1, 2, 4,
+    8 (`path` chooses; by default it runs from 12*2^20 elements up)."""
     if not isinstance(args, zero_accum_args):
         args = make_accum_args(args, R, **kw)
     elif R is not None or kw:

@@ -199,6 +199,9 @@ def test_noalloc_step_refuses_a_caller_workspace():
     (dict(ctrl=A), za.ZERO_EINVAL),                 # and a ctrl a workspace
     (dict(workspace=A + 8, ctrl=A), za.ZERO_EALIGN),
     (dict(workspace=A, ctrl=A + 4), za.ZERO_EALIGN),
+    (dict(path=3), za.ZERO_EINVAL),
+    (dict(path=za.ZERO_PATH_STAGED), za.ZERO_EINVAL),                 # staged needs a workspace
+    (dict(R=3, grads=[A] * 3, workspace=A, ctrl=A, path=za.ZERO_PATH_STAGED), za.ZERO_EINVAL),
 ])
 def test_accumulate_argument_errors(kw, status):
     args = dict(P=1000, R=4, grad_dtype=za.ZERO_BF16, grads=[A] * 4, accum=A, scale=0.25, first=True)

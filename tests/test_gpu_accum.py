@@ -16,6 +16,7 @@ from mixed_precision_adam_zero_b200.buffers import FlatZero
 pytestmark = pytest.mark.gpu
 
 DT = {"bf16": za.ZERO_BF16, "f16": za.ZERO_F16, "f32": za.ZERO_F32}
+STAGED = za.ZERO_PATH_STAGED
 
 
 def _run(P, R, gdt, gas, updates, token=True, S0=1.0, check=False, bad=None, two_set=False, seed=51, staged=True):
@@ -23,7 +24,8 @@ def _run(P, R, gdt, gas, updates, token=True, S0=1.0, check=False, bad=None, two
     accumulation gets the step's workspace and ctrl (shared-memory staged
     kernel for R in 1, 2, 4, 8), else none (register kernel)."""
     z = FlatZero(P, 1, "f32", "bf16", two_set=two_set, loss_scale=S0, alloc_grads=False)
-    ws = dict(workspace=z.workspace, ctrl=z.ctrl_buf) if staged else {}
+    ws = dict(workspace=z.workspace, ctrl=z.ctrl_buf, path=STAGED if R in (1, 2, 4, 8) else za.ZERO_PATH_AUTO) \
+        if staged else dict(path=za.ZERO_PATH_REGISTER)
     acc = torch.zeros(P, dtype=torch.float32, device="cuda")
     micro = [torch.zeros(P, dtype={"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt],
                          device="cuda") for _ in range(R)]
@@ -84,9 +86,9 @@ def test_staged_and_register_kernels_agree_bitwise(gdt, R):
     for mu, first in enumerate((True, False, False)):
         g = _micro(P, R, tdt, 300 + 10 * mu)
         za.zero_accumulate_grads(P, R, grad_dtype=DT[gdt], grads=g, accum=staged, scale=1 / 3, first=first,
-                                 rank_weights=wts, workspace=ws, ctrl=ctrl)
+                                 rank_weights=wts, workspace=ws, ctrl=ctrl, path=STAGED)
         za.zero_accumulate_grads(P, R, grad_dtype=DT[gdt], grads=g, accum=plain, scale=1 / 3, first=first,
-                                 rank_weights=wts)
+                                 rank_weights=wts, path=za.ZERO_PATH_REGISTER)
     torch.cuda.synchronize()
     assert torch.equal(staged.view(torch.int32), plain.view(torch.int32))
     assert not ws.any() and not ctrl.any()
@@ -103,7 +105,7 @@ def test_staged_per_owner_equals_whole_bitwise():
         za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=g, accum=whole, scale=0.5, first=first)
         for r in range(R):
             za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=g, accum=part, scale=0.5, first=first,
-                                     owner=r, workspace=ws, ctrl=ctrl)
+                                     owner=r, workspace=ws, ctrl=ctrl, path=STAGED)
     torch.cuda.synchronize()
     assert torch.equal(whole.view(torch.int32), part.view(torch.int32))
     assert not ws.any() and not ctrl.any()
@@ -111,7 +113,8 @@ def test_staged_per_owner_equals_whole_bitwise():
 
 def test_staged_accumulation_full_size_against_the_oracle():
     # The accumulation of the 16,777,259-parameter, R = 8 bf16 workload in
-    # the benchmark's launch configuration: two micro-batches, every element
+    # the benchmark's launch configuration (the automatic choice, which is
+    # the staged kernel at this size): two micro-batches, every element
     # against the oracle.
     P, R = 16_777_259, 8
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
@@ -149,3 +152,24 @@ def test_per_owner_accumulation_equals_whole_bitwise():
                                      first=first, owner=r)
     torch.cuda.synchronize()
     assert torch.equal(whole, part)
+
+
+def test_automatic_path_around_the_size_threshold():
+    # Ranges just below and just above 12*2^20 elements: the automatic choice
+    # switches kernels there, and every choice gives the same bits.
+    R = 2
+    for P in ((12 << 20) - 1, (12 << 20) + 13):
+        g = _micro(P, R, torch.bfloat16, 700)
+        ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        ctrl = torch.zeros(64, dtype=torch.uint8, device="cuda")
+        out = {}
+        for path in (za.ZERO_PATH_AUTO, za.ZERO_PATH_REGISTER, za.ZERO_PATH_STAGED):
+            acc = torch.full((P,), 0.5, device="cuda")
+            for first in (True, False):
+                za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=g, accum=acc, scale=0.5,
+                                         first=first, workspace=ws, ctrl=ctrl, path=path)
+            out[path] = acc
+        torch.cuda.synchronize()
+        assert torch.equal(out[0].view(torch.int32), out[1].view(torch.int32))
+        assert torch.equal(out[0].view(torch.int32), out[2].view(torch.int32))
+        assert not ws.any() and not ctrl.any()
