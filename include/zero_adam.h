@@ -143,7 +143,12 @@ typedef struct zero_step_args {
                                      updated element (the ZeRO-2 retained
                                      gradient slice); NULL: not written */
     zero_adam_hparams hp;
-    int32_t check_nonfinite;      /* 1: skip the step on any inf/NaN gradient */
+    int32_t check_nonfinite;      /* 1: skip the step on any inf/NaN gradient;
+                                     2: skip it if the workspace's inf/NaN
+                                     word (ZERO_WORKSPACE_FOUND_OFFSET) is
+                                     set, i.e. the decision was taken by
+                                     zero_scan_nonfinite calls; the call
+                                     clears the word */
     uint32_t growth_interval;     /* check on: S doubles after this many
                                      consecutive applied steps; 0: never */
     void *ctrl;                   /* device zero_ctrl */
@@ -153,7 +158,34 @@ typedef struct zero_step_args {
                                      call leaves it all zero again.  Calls
                                      that may overlap on the GPU need separate
                                      workspaces. */
+    /* Data-parallel across GPUs (flat call only; 0 / NULL otherwise).  The
+     * call updates one owner's slice [lo, hi) as above; then: */
+    uint64_t state_offset;        /* master, exp_avg, exp_avg_sq and
+                                     reduced_out hold elements from flat index
+                                     state_offset on (element i at index
+                                     i - state_offset), so a rank allocates
+                                     only [state_offset, hi).  A multiple of 8,
+                                     at most lo; 0 for arrays of P elements. */
+    uint32_t n_push;              /* 0..ZERO_MAX_PUSH */
+    uint32_t reserved;            /* zero */
+    void *const *push_params16;   /* HOST array of n_push device pointers,
+                                     each [P] of param_dtype: the other ranks'
+                                     replicated 16-bit parameters (peer
+                                     mappings).  Every updated 16-bit value is
+                                     stored there as well as into params16:
+                                     the parameter all-gather, fused into the
+                                     step. */
 } zero_step_args;
+
+/* Most push targets of one call (an NVLink domain's GPUs). */
+#define ZERO_MAX_PUSH 72
+
+/* Byte offset of the inf/NaN word in a workspace: a uint32, nonzero once a
+ * zero_scan_nonfinite call found an inf or NaN.  Between the scans and a
+ * step with check_nonfinite = 2 the caller may combine the word across
+ * processes (e.g. an all-reduce MAX of it), so that every rank takes the
+ * same skip decision. */
+#define ZERO_WORKSPACE_FOUND_OFFSET 8
 
 /* Device-resident description of a TENSOR LIST: T parameter tensors whose
  * concatenation, in list order and without padding, is the flat vector the
@@ -223,6 +255,14 @@ int zero_ctrl_read(const void *ctrl, zero_ctrl *out, void *stream);
 
 /* Zero a workspace of ZERO_WORKSPACE_BYTES (cudaMemsetAsync). */
 int zero_workspace_init(void *workspace, void *stream);
+
+/* Overflow scan of one gradient buffer (the check of "Loss scaling", taken
+ * ahead of a step with check_nonfinite = 2): sets the workspace's inf/NaN
+ * word if any of grad[0, n) is inf or NaN, and otherwise leaves it as it
+ * is, so several scans accumulate.  grad: device, 16-byte aligned, of
+ * grad_dtype.  Asynchronous on `stream`.  Errors: ZERO_EINVAL, ZERO_EALIGN,
+ * ZERO_EOVERFLOW, ZERO_ECUDA. */
+int zero_scan_nonfinite(const void *grad, int32_t grad_dtype, uint64_t n, void *workspace, void *stream);
 
 /* Health check of the device-side timeout path (the pages have no
  * counterpart): launches one block whose thread waits, through the same

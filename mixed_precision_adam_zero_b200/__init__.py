@@ -36,6 +36,8 @@ ZERO_MAX_RANKS = 256
 ZERO_WORKSPACE_BYTES = 256
 ZERO_NOALLOC_SCRATCH_BYTES = 256
 ZERO_PATH_AUTO, ZERO_PATH_REGISTER, ZERO_PATH_STAGED = 0, 1, 2
+ZERO_MAX_PUSH = 72
+ZERO_WORKSPACE_FOUND_OFFSET = 8
 
 EXPORTED = [
     "zero_partition_bounds", "zero_state_bytes", "zero_status_string", "zero_last_cuda_error",
@@ -43,6 +45,7 @@ EXPORTED = [
     "zero_ctrl_set", "zero_ctrl_read", "zero_workspace_init", "zero_step_fused",
     "zero_step_fused_list", "zero_list_table_build", "zero_gather_params",
     "zero_gather_params_list", "zero_step_fused_noalloc", "zero_accumulate_grads", "zero_selftest_wait_timeout",
+    "zero_scan_nonfinite",
     "zero_checkpoint_save", "zero_checkpoint_load", "zero_checkpoint_consolidate", "zero_checkpoint_error",
     "zero3_shard_bounds", "zero_parameter_storage", "zero3_gather_list_build", "zero3_gather",
 ]
@@ -80,7 +83,9 @@ class zero_step_args(ctypes.Structure):
                 ("exp_avg_sq", ctypes.c_void_p * 2), ("params16", ctypes.c_void_p),
                 ("reduced_out", ctypes.c_void_p), ("hp", zero_adam_hparams),
                 ("check_nonfinite", ctypes.c_int32), ("growth_interval", ctypes.c_uint32),
-                ("ctrl", ctypes.c_void_p), ("workspace", ctypes.c_void_p)]
+                ("ctrl", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("state_offset", ctypes.c_uint64), ("n_push", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
+                ("push_params16", ctypes.POINTER(ctypes.c_void_p))]
 
 
 class zero_accum_args(ctypes.Structure):
@@ -125,6 +130,7 @@ def _lib() -> ctypes.CDLL:
         L.zero_ctrl_read.argtypes = [vp, ctypes.POINTER(zero_ctrl), vp]
         L.zero_workspace_init.argtypes = [vp, vp]
         L.zero_selftest_wait_timeout.argtypes = [vp, vp]
+        L.zero_scan_nonfinite.argtypes = [vp, i32, u64, vp, vp]
         L.zero_step_fused.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_step_fused_noalloc.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_accumulate_grads.argtypes = [ctypes.POINTER(zero_accum_args), vp]
@@ -228,6 +234,12 @@ def zero_workspace_init(workspace, stream=None) -> None:
     _check(_lib().zero_workspace_init(_ptr(workspace), _stream(stream)), "zero_workspace_init")
 
 
+def zero_scan_nonfinite(grad, grad_dtype: int, n: int, workspace, stream=None) -> None:
+    """Set the workspace's inf/NaN word if grad[0, n) holds an inf or NaN."""
+    _check(_lib().zero_scan_nonfinite(_ptr(grad), grad_dtype, n, _ptr(workspace), _stream(stream)),
+           "zero_scan_nonfinite")
+
+
 def zero_selftest_wait_timeout(ctrl, stream=None) -> None:
     """Run the device-side timeout path once: sets ctrl.device_error to 1
     after about 2 s of GPU time (see the C declaration)."""
@@ -238,8 +250,9 @@ def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master,
                    ctrl, workspace, grads: Optional[Sequence] = None, params16=None,
                    rank_weights: Optional[Sequence[float]] = None, owner: int = -1,
                    hp: Tuple[float, float, float, float, float] = (1e-3, 0.9, 0.999, 1e-8, 0.0),
-                   check_nonfinite: bool = False, growth_interval: int = 0, reduced_out=None,
-                   master2=None, exp_avg2=None, exp_avg_sq2=None) -> zero_step_args:
+                   check_nonfinite: int = 0, growth_interval: int = 0, reduced_out=None,
+                   master2=None, exp_avg2=None, exp_avg_sq2=None, state_offset: int = 0,
+                   push_params16: Optional[Sequence] = None) -> zero_step_args:
     """Fill a zero_step_args (the returned struct keeps its host arrays alive)."""
     a = zero_step_args()
     a.P, a.R, a.owner = P, R, owner
@@ -257,9 +270,15 @@ def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master,
     a.params16 = _ptr(params16)
     a.reduced_out = _ptr(reduced_out)
     a.hp = zero_adam_hparams(*[float(x) for x in hp])
-    a.check_nonfinite = int(bool(check_nonfinite))
+    a.check_nonfinite = int(check_nonfinite)
     a.growth_interval = growth_interval
     a.ctrl, a.workspace = _ptr(ctrl), _ptr(workspace)
+    a.state_offset = state_offset
+    if push_params16:
+        arr = (ctypes.c_void_p * len(push_params16))(*[_ptr(t) for t in push_params16])
+        a._push_keep = arr
+        a.push_params16 = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+        a.n_push = len(push_params16)
     return a
 
 

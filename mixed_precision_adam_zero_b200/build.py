@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 SOURCES = [os.path.join(PKG, "csrc", "zero_adam_api.cu"), os.path.join(PKG, "csrc", "zero_adam_host.cpp"),
            os.path.join(PKG, "csrc", "zero_adam_ckpt.cpp")]
 DEPS = SOURCES + [os.path.join(PKG, "csrc", "zero_adam_kernels.cuh"), os.path.join(PKG, "csrc", "zero_adam_bulk.cuh"),
-                  os.path.join(ROOT, "include", "zero_adam.h")]
+                  os.path.join(PKG, "csrc", "zero_adam_internal.h"), os.path.join(ROOT, "include", "zero_adam.h")]
 OUT = os.path.join(PKG, "libzero_adam.so")
 
 NVCC_FLAGS = [

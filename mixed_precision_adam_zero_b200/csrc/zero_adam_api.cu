@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "zero_adam.h"
+#include "zero_adam_internal.h"
 #include "zero_adam_kernels.cuh"
 #include "zero_adam_bulk.cuh"
 
@@ -102,39 +103,43 @@ int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st, unsig
 // ------------------------------------------------------------ kernel tables
 
 // Calls with a compile-time rank count stage their tiles through shared
-// memory with bulk copies; other rank counts use the register path.
-template <class G, class Pm, int RC, bool LIST>
+// memory with bulk copies; other rank counts use the register path.  PUSH:
+// flat calls that also store the 16-bit values into other replicas.
+template <class G, class Pm, int RC, bool LIST, bool PUSH>
 Kern bulk_kern() {
-    return Kern{(const void*)step_bulk_kernel<G, Pm, RC, LIST>, BulkShape<G, RC>::kSmem, kBulkThreads};
+    return Kern{(const void*)step_bulk_kernel<G, Pm, RC, LIST, PUSH>, BulkShape<G, RC>::kSmem, kBulkThreads};
 }
 
-template <class G, class Pm, bool LIST>
+template <class G, class Pm, bool LIST, bool PUSH>
 Kern step_kern_rc(uint32_t R) {
     switch (R) {
-        case 1: return bulk_kern<G, Pm, 1, LIST>();
-        case 2: return bulk_kern<G, Pm, 2, LIST>();
-        case 4: return bulk_kern<G, Pm, 4, LIST>();
-        case 8: return bulk_kern<G, Pm, 8, LIST>();
-        default: return Kern{(const void*)step_kernel<G, Pm, 0, LIST>, 0u, kThreads};
+        case 1: return bulk_kern<G, Pm, 1, LIST, PUSH>();
+        case 2: return bulk_kern<G, Pm, 2, LIST, PUSH>();
+        case 4: return bulk_kern<G, Pm, 4, LIST, PUSH>();
+        case 8: return bulk_kern<G, Pm, 8, LIST, PUSH>();
+        default: return Kern{(const void*)step_kernel<G, Pm, 0, LIST, PUSH>, 0u, kThreads};
     }
 }
 
-template <class G, bool LIST>
+template <class G, bool LIST, bool PUSH>
 Kern step_kern_pm(int32_t param_dtype, uint32_t R) {
-    return param_dtype == ZERO_BF16 ? step_kern_rc<G, __nv_bfloat16, LIST>(R) : step_kern_rc<G, __half, LIST>(R);
+    return param_dtype == ZERO_BF16 ? step_kern_rc<G, __nv_bfloat16, LIST, PUSH>(R)
+                                    : step_kern_rc<G, __half, LIST, PUSH>(R);
 }
 
-template <bool LIST>
+template <bool LIST, bool PUSH>
 Kern step_kern_gd(int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
     switch (grad_dtype) {
-        case ZERO_F32: return step_kern_pm<float, LIST>(param_dtype, R);
-        case ZERO_BF16: return step_kern_pm<__nv_bfloat16, LIST>(param_dtype, R);
-        default: return step_kern_pm<__half, LIST>(param_dtype, R);
+        case ZERO_F32: return step_kern_pm<float, LIST, PUSH>(param_dtype, R);
+        case ZERO_BF16: return step_kern_pm<__nv_bfloat16, LIST, PUSH>(param_dtype, R);
+        default: return step_kern_pm<__half, LIST, PUSH>(param_dtype, R);
     }
 }
 
-Kern step_kern(bool list, int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
-    return list ? step_kern_gd<true>(grad_dtype, param_dtype, R) : step_kern_gd<false>(grad_dtype, param_dtype, R);
+Kern step_kern(bool list, bool push, int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
+    if (list) return step_kern_gd<true, false>(grad_dtype, param_dtype, R);
+    return push ? step_kern_gd<false, true>(grad_dtype, param_dtype, R)
+                : step_kern_gd<false, false>(grad_dtype, param_dtype, R);
 }
 
 template <bool LIST>
@@ -215,7 +220,10 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     if (a->R > ZERO_MAX_RANKS) return ZERO_ERANGE;
     if (a->owner < -1 || a->owner >= (int64_t)a->R) return ZERO_EINVAL;
     if (!is_grad_dtype(a->grad_dtype) || !is_param_dtype(a->param_dtype)) return ZERO_EINVAL;
-    if (a->check_nonfinite != 0 && a->check_nonfinite != 1) return ZERO_EINVAL;
+    if (a->check_nonfinite < 0 || a->check_nonfinite > 2) return ZERO_EINVAL;
+    if (a->n_push > ZERO_MAX_PUSH) return ZERO_ERANGE;
+    if (a->reserved != 0u || (a->n_push > 0 && a->push_params16 == nullptr)) return ZERO_EINVAL;
+    if ((a->state_offset & 7u) != 0) return ZERO_EALIGN;
     if (a->P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
     int rc = check_hparams(a->hp);
     if (rc) return rc;
@@ -244,13 +252,24 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     for (uint32_t r = 0; r < a->R; ++r) kp->wt[r] = a->rank_weights ? a->rank_weights[r] : 1.0;
     kp->wsum = wsum;
 
+    // State arrays that start at flat index state_offset: the kernels index
+    // them by the flat index, so hand them pointers moved back by that much
+    // (only indices >= state_offset are ever dereferenced).
+    const uintptr_t back = (uintptr_t)(a->state_offset * sizeof(float));
+    auto shift = [back](float* q) { return q ? reinterpret_cast<float*>(reinterpret_cast<uintptr_t>(q) - back) : q; };
     for (int k = 0; k < 2; ++k) {
         const int src = two ? k : 0;
-        kp->w[k] = a->master[src];
-        kp->m[k] = a->exp_avg[src];
-        kp->v[k] = a->exp_avg_sq[src];
+        kp->w[k] = shift(a->master[src]);
+        kp->m[k] = shift(a->exp_avg[src]);
+        kp->v[k] = shift(a->exp_avg_sq[src]);
     }
-    kp->reduced = a->reduced_out;
+    kp->reduced = shift(a->reduced_out);
+    for (uint32_t i = 0; i < a->n_push; ++i) {
+        if (a->P > 0 && a->push_params16[i] == nullptr) return ZERO_EINVAL;
+        if (!aligned16(a->push_params16[i])) return ZERO_EALIGN;
+        kp->push[i] = a->push_params16[i];
+    }
+    kp->npush = a->n_push;
     const zero_adam_hparams& h = a->hp;
     kp->h.b1 = (float)h.beta1;
     kp->h.b2 = (float)h.beta2;
@@ -282,12 +301,15 @@ template <bool LIST>
 int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
     uint64_t lo, hi;
     owner_range(a, &lo, &hi);
+    if (a->state_offset > lo && lo < hi) return ZERO_EINVAL;
     kp->lo = lo;
     kp->hi = hi;
     int err = ZERO_OK;
     const bool check = a->check_nonfinite != 0;
-    const bool single_pass = check && kp->two_set && a->owner < 0;
-    if (check && !single_pass) {
+    const bool single_pass = a->check_nonfinite == 1 && kp->two_set && a->owner < 0;
+    if (a->check_nonfinite == 2) {
+        kp->check = 2;  // zero_scan_nonfinite calls (and the caller) decided
+    } else if (check && !single_pass) {
         // Scan every rank's whole gradient first; the step then reads the flag.
         StepParams sp = *kp;
         const void* sfn = scan_fn<LIST>(a->grad_dtype);
@@ -303,7 +325,7 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
     } else {
         kp->check = check ? 1 : 0;
     }
-    const Kern k = step_kern(LIST, a->grad_dtype, a->param_dtype, a->R);
+    const Kern k = step_kern(LIST, kp->npush > 0, a->grad_dtype, a->param_dtype, a->R);
     const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;
     const Shape sh = make_shape(lo, hi, ctas);
@@ -404,6 +426,29 @@ int noalloc_scratch(void** out) {
 
 // =================================================================== C ABI
 
+int zadam_host::cast_slice(const float* master, uint64_t state_offset, void* params16, int32_t param_dtype,
+                           uint64_t lo, uint64_t hi, void* stream) {
+    if (!is_param_dtype(param_dtype) || master == nullptr || params16 == nullptr) return ZERO_EINVAL;
+    if ((state_offset & 7u) != 0 || state_offset > lo || !aligned16(master) || !aligned16(params16))
+        return ZERO_EALIGN;
+    if (lo >= hi) return ZERO_OK;
+    GatherParams gp;
+    std::memset(&gp, 0, sizeof gp);
+    const float* w = reinterpret_cast<const float*>(reinterpret_cast<uintptr_t>(master) - state_offset * 4u);
+    gp.w[0] = gp.w[1] = w;
+    gp.params16 = params16;
+    gp.lo = lo;
+    gp.hi = hi;
+    int err = ZERO_OK;
+    const void* fn = gather_fn<false>(param_dtype);
+    const int ctas = resident_ctas(fn, &err);
+    if (err) return err;
+    const Shape sh = make_shape(lo, hi, ctas);
+    gp.base = sh.base;
+    gp.chunk = sh.chunk;
+    return launch(fn, sh, &gp, static_cast<cudaStream_t>(stream));
+}
+
 extern "C" {
 
 const char* zero_last_cuda_error(void) { return g_cuda_error; }
@@ -436,6 +481,28 @@ int zero_ctrl_read(const void* ctrl, zero_ctrl* out, void* stream) {
     cudaError_t e = cudaMemcpyAsync(out, ctrl, sizeof(zero_ctrl), cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     return e == cudaSuccess ? ZERO_OK : zadam_record_cuda(e);
+}
+
+int zero_scan_nonfinite(const void* grad, int32_t grad_dtype, uint64_t n, void* workspace, void* stream) {
+    if (!is_grad_dtype(grad_dtype) || workspace == nullptr || (n > 0 && grad == nullptr)) return ZERO_EINVAL;
+    if (!aligned16(grad) || !aligned16(workspace)) return ZERO_EALIGN;
+    if (n > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
+    if (n == 0) return ZERO_OK;
+    StepParams sp;
+    std::memset(&sp, 0, sizeof sp);
+    sp.grads[0] = grad;
+    sp.R = 1;
+    sp.ws = static_cast<Workspace*>(workspace);
+    sp.lo = 0;
+    sp.hi = n;
+    int err = ZERO_OK;
+    const void* fn = scan_fn<false>(grad_dtype);
+    const int ctas = resident_ctas(fn, &err);
+    if (err) return err;
+    const Shape sh = make_shape(0, n, ctas);
+    sp.base = sh.base;
+    sp.chunk = sh.chunk;
+    return launch(fn, sh, &sp, static_cast<cudaStream_t>(stream));
 }
 
 int zero_selftest_wait_timeout(void* ctrl, void* stream) {
@@ -475,6 +542,7 @@ int zero_step_fused_list(const zero_step_args* a, const zero_tensor_list* l, voi
     if (rc) return rc;
     if ((rc = check_list(l))) return rc;
     if (a->grads != nullptr || a->params16 != nullptr) return ZERO_EINVAL;
+    if (a->state_offset != 0 || a->n_push != 0) return ZERO_EINVAL;  // multi-GPU fields: flat calls only
     if (a->P != l->P || a->R != l->R || a->grad_dtype != l->grad_dtype || a->param_dtype != l->param_dtype)
         return ZERO_EINVAL;
     kp.tab = device_table(l);

@@ -157,7 +157,7 @@ struct BulkShape {
 // Four consecutive elements at flat index e (tile-relative offset q in the
 // stage, index le within the tensor's 16-bit parameters), reduced, updated
 // and stored.
-template <class G, class Pm, int RC>
+template <class G, class Pm, int RC, bool PUSH = false>
 __device__ __forceinline__ void bulk_group(const StepParams& p, const Scal& s, const unsigned char* stage,
                                            uint32_t q, uint64_t e, uint64_t le, float* wo, float* mo, float* vo,
                                            Pm* pp, bool& bad) {
@@ -195,6 +195,8 @@ __device__ __forceinline__ void bulk_group(const StepParams& p, const Scal& s, c
     o.x = pack2<Pm>(w[0], w[1]);
     o.y = pack2<Pm>(w[2], w[3]);
     __stcs(reinterpret_cast<uint2*>(pp + le), o);
+    if constexpr (PUSH)
+        for (uint32_t i = 0; i < p.npush; ++i) __stcs(reinterpret_cast<uint2*>(static_cast<Pm*>(p.push[i]) + le), o);
     if (p.reduced != nullptr) __stcs(reinterpret_cast<float4*>(p.reduced + e), make_float4(g[0], g[1], g[2], g[3]));
 }
 
@@ -288,7 +290,7 @@ struct TileWalk {
 };
 
 // Scalar pass over everything the tile walk leaves out.
-template <class G, class Pm, int RC, bool LIST>
+template <class G, class Pm, int RC, bool LIST, bool PUSH = false>
 __device__ __forceinline__ void bulk_scalar_pass(const StepParams& p, const Scal& s, uint64_t a, uint64_t b,
                                                  const StateIO& io, bool& bad, const void** s_gp) {
     if constexpr (!LIST) {
@@ -297,8 +299,10 @@ __device__ __forceinline__ void bulk_scalar_pass(const StepParams& p, const Scal
         uint64_t va = (a + 7) & ~7ull, vb = b & ~7ull;
         if (va > b) va = b;
         if (vb < va) vb = va;
-        for (uint64_t e = a + threadIdx.x; e < va; e += kBulkThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e, io, bad);
-        for (uint64_t e = vb + threadIdx.x; e < b; e += kBulkThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e, io, bad);
+        for (uint64_t e = a + threadIdx.x; e < va; e += kBulkThreads)
+            elem_step<G, Pm, RC, PUSH>(p, s, gp, pp, e, e, io, bad);
+        for (uint64_t e = vb + threadIdx.x; e < b; e += kBulkThreads)
+            elem_step<G, Pm, RC, PUSH>(p, s, gp, pp, e, e, io, bad);
     } else {
         uint32_t j = find_tensor(p.tab, a);
         uint64_t x = a;
@@ -410,7 +414,7 @@ __device__ __forceinline__ void flat_consume(Workspace* ws, uint64_t va, uint64_
     }
 }
 
-template <class G, class Pm, int RC>
+template <class G, class Pm, int RC, bool PUSH = false>
 __device__ __forceinline__ void flat_dynamic(const StepParams& p, uint64_t* full, uint64_t* empty,
                                              uint32_t* slot, unsigned char* ring, bool& bad) {
     using Sh = BulkShape<G, RC>;
@@ -432,7 +436,7 @@ __device__ __forceinline__ void flat_dynamic(const StepParams& p, uint64_t* full
         flat_consume<D>(p.ws, va, vb, full, empty, slot, [&](int st, uint64_t e0, uint32_t n) {
             const unsigned char* stage = ring + st * Sh::kStage;
             for (uint32_t q = 4u * threadIdx.x; q < n; q += 4u * kConsumers)
-                bulk_group<G, Pm, RC>(p, s, stage, q, e0 + q, e0 + q, io.wo, io.mo, io.vo, pp, bad);
+                bulk_group<G, Pm, RC, PUSH>(p, s, stage, q, e0 + q, e0 + q, io.wo, io.mo, io.vo, pp, bad);
         });
     }
 }
@@ -609,8 +613,11 @@ __device__ __forceinline__ void list_static(const StepParams& p, uint64_t a, uin
     }
 }
 
-template <class G, class Pm, int RC, bool LIST>
+// PUSH (flat calls only): every 16-bit value is also stored into the
+// p.npush other replicas in p.push.
+template <class G, class Pm, int RC, bool LIST, bool PUSH = false>
 __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid_constant__ StepParams p) {
+    static_assert(!(LIST && PUSH), "parameter push is for flat calls");
     using Sh = BulkShape<G, RC>;
     constexpr int D = Sh::kStages;
     constexpr uint32_t kConsumerWarps = kConsumers / 32;
@@ -643,7 +650,7 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
             if (p.whole) list_dynamic<G, Pm, RC>(p, full, empty, reinterpret_cast<TileDesc*>(slot), ring, bad);
             else list_static<G, Pm, RC>(p, a, b, full, empty, ring, bad);
         } else {
-            flat_dynamic<G, Pm, RC>(p, full, empty, slot, ring, bad);
+            flat_dynamic<G, Pm, RC, PUSH>(p, full, empty, slot, ring, bad);
         }
         __syncthreads();
         // Ragged heads and tails, and tensors that cannot take the vector path
@@ -657,10 +664,10 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
                 if (a < b) bulk_scalar_pass<G, Pm, RC, true>(p, s, a, b, io, bad, s_gp);
             }
         } else if (blockIdx.x == 0) {
-            bulk_scalar_pass<G, Pm, RC, false>(p, s, p.lo, p.hi, io, bad, s_gp);
+            bulk_scalar_pass<G, Pm, RC, false, PUSH>(p, s, p.lo, p.hi, io, bad, s_gp);
         }
     }
-    finish_step(p, bad, s_timed_out != 0u);
+    finish_step<PUSH>(p, bad, s_timed_out != 0u);
 }
 
 // ------------------------------------------------------------ micro-step accumulation

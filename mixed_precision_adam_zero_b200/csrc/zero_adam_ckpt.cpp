@@ -29,6 +29,7 @@
 #include <vector>
 
 #include "zero_adam.h"
+#include "zero_adam_internal.h"
 
 namespace {
 
@@ -92,6 +93,10 @@ int check_args(const zero_step_args* a, const char* path) {
     const bool two = a->master[1] != nullptr || a->exp_avg[1] != nullptr || a->exp_avg_sq[1] != nullptr;
     if (two && (a->master[1] == nullptr || a->exp_avg[1] == nullptr || a->exp_avg_sq[1] == nullptr))
         return ZERO_EINVAL;
+    if ((a->state_offset & 7u) != 0) return ZERO_EALIGN;
+    uint64_t lo, hi;
+    slice_of(a, &lo, &hi);
+    if (a->state_offset > lo && lo < hi) return ZERO_EINVAL;
     return ZERO_OK;
 }
 
@@ -178,7 +183,7 @@ int zero_checkpoint_save(const char* path, const zero_step_args* a, void* stream
     std::vector<float> stage((size_t)(n < kChunk ? (n > 0 ? n : 1) : kChunk));
     const float* arrays[3] = {a->master[set], a->exp_avg[set], a->exp_avg_sq[set]};
     for (const float* arr : arrays) {
-        if ((rc = write_array(f, arr + h.lo, n, stage, sum, st, path))) {
+        if ((rc = write_array(f, arr + (h.lo - a->state_offset), n, stage, sum, st, path))) {
             std::fclose(f);
             return rc;
         }
@@ -211,7 +216,7 @@ int zero_checkpoint_load(const char* path, const zero_step_args* a, void* stream
     std::vector<float> stage((size_t)(n < kChunk ? (n > 0 ? n : 1) : kChunk));
     float* arrays[3] = {a->master[0], a->exp_avg[0], a->exp_avg_sq[0]};
     for (float* arr : arrays) {
-        if ((rc = read_array(f, arr + lo, n, stage, sum, st, path))) {
+        if ((rc = read_array(f, arr + (lo - a->state_offset), n, stage, sum, st, path))) {
             std::fclose(f);
             return rc;
         }
@@ -220,6 +225,12 @@ int zero_checkpoint_load(const char* path, const zero_step_args* a, void* stream
     std::fclose(f);
     if (rc) return rc;
     if ((rc = zero_ctrl_set(a->ctrl, &h.ctrl, stream))) return rc;
+    if (a->params16 != nullptr && n > 0 && a->state_offset != 0) {
+        // Arrays of this rank's slice only: re-cast exactly [lo, hi) into
+        // the local 16-bit parameters (the other ranks' replicas receive
+        // the slice from the caller).
+        return zadam_host::cast_slice(a->master[0], a->state_offset, a->params16, a->param_dtype, lo, hi, stream);
+    }
     if (a->params16 != nullptr && n > 0) {
         // The 16-bit parameters follow from the restored masters.  The cast
         // runs over the slice widened to multiples of 8 elements (the cast's

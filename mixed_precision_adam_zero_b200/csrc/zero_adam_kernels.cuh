@@ -91,6 +91,7 @@ struct StepParams {
     float* m[2];
     float* v[2];
     void* params16;                     // flat call: 16-bit parameters [P]
+    void* push[ZERO_MAX_PUSH];          // flat call: other ranks' 16-bit parameters [P]
     float* reduced;                     // optional reduced-gradient output
     Table tab;                          // list call
     uint64_t lo, hi;                    // elements this launch updates
@@ -103,6 +104,7 @@ struct StepParams {
     int32_t two_set;  // 1: read set ctrl.parity, write the other set
     int32_t check;    // 0: none; 1: detect inf/NaN in this pass; 2: a scan decided
     int32_t whole;    // 1: the launch covers every owner's slice ([0, P))
+    uint32_t npush;   // entries of push in use
 };
 
 struct GatherParams {
@@ -289,7 +291,7 @@ struct StateIO {
 // ------------------------------------------------------------ step bodies
 
 // One 8-element vector at flat index e (multiple of 8); le = e - tensor start.
-template <class G, class Pm, int RC>
+template <class G, class Pm, int RC, bool PUSH = false>
 __device__ __forceinline__ void vec_step(const StepParams& p, const Scal& s, const GradPtrs<G, RC>& gp,
                                          Pm* pp, uint64_t e, uint64_t le, const StateIO& io, bool& bad) {
     double acc[8];
@@ -364,6 +366,8 @@ __device__ __forceinline__ void vec_step(const StepParams& p, const Scal& s, con
     o.z = pack2<Pm>(w[4], w[5]);
     o.w = pack2<Pm>(w[6], w[7]);
     __stcs(reinterpret_cast<uint4*>(pp + le), o);
+    if constexpr (PUSH)
+        for (uint32_t i = 0; i < p.npush; ++i) __stcs(reinterpret_cast<uint4*>(static_cast<Pm*>(p.push[i]) + le), o);
     if (p.reduced != nullptr) {
         __stcs(reinterpret_cast<float4*>(p.reduced + e), make_float4(g[0], g[1], g[2], g[3]));
         __stcs(reinterpret_cast<float4*>(p.reduced + e + 4), make_float4(g[4], g[5], g[6], g[7]));
@@ -371,7 +375,7 @@ __device__ __forceinline__ void vec_step(const StepParams& p, const Scal& s, con
 }
 
 // One element (heads, tails and tensors that cannot take the vector path).
-template <class G, class Pm, int RC>
+template <class G, class Pm, int RC, bool PUSH = false>
 __device__ __forceinline__ void elem_step(const StepParams& p, const Scal& s, const GradPtrs<G, RC>& gp,
                                           Pm* pp, uint64_t e, uint64_t le, const StateIO& io, bool& bad) {
     double acc = 0.0;
@@ -388,12 +392,15 @@ __device__ __forceinline__ void elem_step(const StepParams& p, const Scal& s, co
     io.wo[e] = w;
     io.mo[e] = m;
     io.vo[e] = v;
-    reinterpret_cast<unsigned short*>(pp)[le] = cvt1<Pm>(w);
+    const unsigned short h = cvt1<Pm>(w);
+    reinterpret_cast<unsigned short*>(pp)[le] = h;
+    if constexpr (PUSH)
+        for (uint32_t i = 0; i < p.npush; ++i) static_cast<unsigned short*>(p.push[i])[le] = h;
     if (p.reduced != nullptr) p.reduced[e] = g;
 }
 
 // Flat range [a, b) of one tensor that starts at flat index toff.
-template <class G, class Pm, int RC>
+template <class G, class Pm, int RC, bool PUSH = false>
 __device__ __forceinline__ void run_segment(const StepParams& p, const Scal& s, const GradPtrs<G, RC>& gp,
                                             Pm* pp, uint64_t toff, uint64_t a, uint64_t b, bool vec_ok,
                                             const StateIO& io, bool& bad) {
@@ -404,10 +411,12 @@ __device__ __forceinline__ void run_segment(const StepParams& p, const Scal& s, 
         vb = b & ~7ull;
         if (vb < va) vb = va;
     }
-    for (uint64_t e = a + threadIdx.x; e < va; e += kThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e - toff, io, bad);
+    for (uint64_t e = a + threadIdx.x; e < va; e += kThreads)
+        elem_step<G, Pm, RC, PUSH>(p, s, gp, pp, e, e - toff, io, bad);
     for (uint64_t e = va + (uint64_t)threadIdx.x * kVec; e < vb; e += (uint64_t)kThreads * kVec)
-        vec_step<G, Pm, RC>(p, s, gp, pp, e, e - toff, io, bad);
-    for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads) elem_step<G, Pm, RC>(p, s, gp, pp, e, e - toff, io, bad);
+        vec_step<G, Pm, RC, PUSH>(p, s, gp, pp, e, e - toff, io, bad);
+    for (uint64_t e = vb + threadIdx.x; e < b; e += kThreads)
+        elem_step<G, Pm, RC, PUSH>(p, s, gp, pp, e, e - toff, io, bad);
 }
 
 // Index of the tensor holding flat element x (offs[j] <= x < offs[j+1]).
@@ -435,7 +444,11 @@ __device__ __forceinline__ uint32_t find_tensor_by_tile(const Table& t, uint64_t
 // control block and the workspace in this launch happened before the
 // accessing CTA's arrival, and the next launch sees the writes at the kernel
 // boundary.  Only thread 0's `timed_out` is used.
+template <bool PUSH = false>
 __device__ __forceinline__ void finish_step(const StepParams& p, bool bad, bool timed_out = false) {
+    // Stores into other GPUs' parameter buffers are performed before the CTA
+    // completes, whatever orders the peers' next reads after this kernel.
+    if constexpr (PUSH) __threadfence_system();
     const int any = __syncthreads_or(bad ? 1 : 0);
     if (threadIdx.x == 0) {
         Workspace* ws = p.ws;
@@ -470,7 +483,7 @@ __device__ __forceinline__ void finish_step(const StepParams& p, bool bad, bool 
     }
 }
 
-template <class G, class Pm, int RC, bool LIST>
+template <class G, class Pm, int RC, bool LIST, bool PUSH = false>
 __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ StepParams p) {
     __shared__ const void* s_gp[LIST ? ZERO_MAX_RANKS : 1];
     const zero_ctrl* c = p.ctrl;
@@ -489,7 +502,7 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ 
     if (!skip && a < b) {
         if constexpr (!LIST) {
             const GradPtrs<G, RC> gp(&p.grads[0]);
-            run_segment<G, Pm, RC>(p, s, gp, static_cast<Pm*>(p.params16), 0ull, a, b, true, io, bad);
+            run_segment<G, Pm, RC, PUSH>(p, s, gp, static_cast<Pm*>(p.params16), 0ull, a, b, true, io, bad);
         } else {
             uint32_t j = find_tensor(p.tab, a);
             uint64_t x = a;
@@ -510,7 +523,7 @@ __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ 
             }
         }
     }
-    finish_step(p, bad);
+    finish_step<PUSH>(p, bad);
 }
 
 // ------------------------------------------------------------ overflow scan

@@ -34,8 +34,9 @@ def test_library_exports_every_declared_symbol():
 def test_struct_layouts_match_the_header():
     assert za.zero_ctrl_bytes() == ctypes.sizeof(za.zero_ctrl) == 40
     assert za.zero_workspace_bytes() == za.ZERO_WORKSPACE_BYTES == 256
-    # zero_step_args: 5 ints + 2 host pointers + 8 device pointers + hparams + 2 ints + 2 pointers
-    assert ctypes.sizeof(za.zero_step_args) == 8 + 4 * 4 + 8 * 2 + 8 * 8 + 40 + 8 + 16
+    # zero_step_args: 5 ints + 2 host pointers + 8 device pointers + hparams + 2 ints + 2 pointers,
+    # then state_offset, n_push, reserved and the push array
+    assert ctypes.sizeof(za.zero_step_args) == 8 + 4 * 4 + 8 * 2 + 8 * 8 + 40 + 8 + 16 + 8 + 4 + 4 + 8
 
 
 def test_partition_bounds_match_the_oracle_bit_exactly():
@@ -121,10 +122,17 @@ def _args(**over):
     (dict(master2=A), za.ZERO_EINVAL),          # second set incomplete
     (dict(P=2**62), za.ZERO_EOVERFLOW),
     (dict(check_nonfinite=True, reduced_out=A + 4), za.ZERO_EALIGN),
+    (dict(check_nonfinite=3), za.ZERO_EINVAL),
+    (dict(state_offset=4, owner=1), za.ZERO_EALIGN),         # not a multiple of 8
+    (dict(state_offset=256, owner=1), za.ZERO_EINVAL),       # owner 1 of (1000, 4) starts at 250
+    (dict(state_offset=8), za.ZERO_EINVAL),                  # the all-owner call starts at 0
+    (dict(push_params16=[A] * 73), za.ZERO_ERANGE),
+    (dict(push_params16=[A, A + 2]), za.ZERO_EALIGN),
+    (dict(push_params16=[A, None]), za.ZERO_EINVAL),
 ])
 def test_step_argument_errors_are_rejected_on_the_host(over, status):
     a = _args(**over)
-    if "check_nonfinite" in over:
+    if over.get("check_nonfinite") is True:
         a.check_nonfinite = 1
     with pytest.raises(za.ZeroError) as e:
         za.zero_step_fused(a)
@@ -159,6 +167,31 @@ def test_gather_and_ctrl_argument_errors():
          za.ZERO_EINVAL),
         (lambda: za.zero_list_table_build([4, 4], [A, None], [[A, A]], za.ZERO_BF16, za.ZERO_BF16, A, 1 << 20),
          za.ZERO_EINVAL),
+    ]:
+        with pytest.raises(za.ZeroError) as e:
+            call()
+        assert e.value.status == status
+
+
+def test_multi_gpu_fields_are_flat_only():
+    lst = za.zero_tensor_list()
+    lst.table, lst.P, lst.T, lst.R, lst.grad_dtype, lst.param_dtype, lst.table_bytes = A, 1000, 1, 4, \
+        za.ZERO_BF16, za.ZERO_BF16, 1 << 20
+    for over in (dict(push_params16=[A]), dict(state_offset=8, owner=1)):
+        a = _args(grads=None, params16=None, **over)
+        with pytest.raises(za.ZeroError) as e:
+            za.zero_step_fused_list(a, lst)
+        assert e.value.status == za.ZERO_EINVAL
+
+
+def test_scan_argument_errors():
+    for call, status in [
+        (lambda: za.zero_scan_nonfinite(A, 9, 10, A), za.ZERO_EINVAL),
+        (lambda: za.zero_scan_nonfinite(None, za.ZERO_F16, 10, A), za.ZERO_EINVAL),
+        (lambda: za.zero_scan_nonfinite(A, za.ZERO_F16, 10, None), za.ZERO_EINVAL),
+        (lambda: za.zero_scan_nonfinite(A + 2, za.ZERO_F16, 10, A), za.ZERO_EALIGN),
+        (lambda: za.zero_scan_nonfinite(A, za.ZERO_F16, 10, A + 8), za.ZERO_EALIGN),
+        (lambda: za.zero_scan_nonfinite(A, za.ZERO_F16, 2**62, A), za.ZERO_EOVERFLOW),
     ]:
         with pytest.raises(za.ZeroError) as e:
             call()

@@ -1,0 +1,228 @@
+"""GPU checks of the multi-GPU ZeRO-2 step (state offset, fused parameter
+push, scan + shared skip decision).
+
+With one GPU the R ranks are emulated inside one process: every rank has
+its own state slice, control block, workspace and 16-bit replica, the R
+owner calls run one after another (no kernel waits on another), and the
+cross-rank all-reduce of the inf/NaN word is a maximum taken on the host.
+Every rank must end bitwise equal to the single-call step over the same
+gradients (itself checked against the oracle elsewhere).  A second test runs
+two real processes on the one GPU, mapping each other's buffers through CUDA
+IPC and synchronising through gloo."""
+import datetime
+import os
+import socket
+import sys
+import types
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import mixed_precision_adam_zero_b200 as za
+import oracle
+import synth
+from conftest import ROOT
+from gpu_helpers import ADAMW_HP, compare_full, grads_for_step, host_grad, ohp
+from mixed_precision_adam_zero_b200.buffers import DTYPES, FlatZero
+from mixed_precision_adam_zero_b200.zero2 import rank_slice
+
+pytestmark = pytest.mark.gpu
+
+FOUND = slice(za.ZERO_WORKSPACE_FOUND_OFFSET, za.ZERO_WORKSPACE_FOUND_OFFSET + 4)
+
+
+def _ranks(P, R, gdt, pdt, w0, S0):
+    pcode, ptorch = DTYPES[pdt]
+    out = []
+    for r in range(R):
+        lo, hi, off, n = rank_slice(P, R, r)
+        k = types.SimpleNamespace(lo=lo, hi=hi, off=off)
+        k.master = torch.full((n,), float("nan"), device="cuda")    # spare elements must never be read
+        k.master[lo - off:hi - off].copy_(w0[lo:hi])
+        k.exp_avg = torch.zeros(n, device="cuda")
+        k.exp_avg_sq = torch.zeros(n, device="cuda")
+        k.params16 = torch.zeros(P, dtype=ptorch, device="cuda")
+        za.zero_gather_params(w0, k.params16, pcode, P)
+        k.ctrl = torch.zeros(64, dtype=torch.uint8, device="cuda")
+        za.zero_ctrl_init(k.ctrl, S0)
+        k.ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+        out.append(k)
+    return out
+
+
+def _emulated_step(ranks, grads, P, R, gdt, pdt, check, wts):
+    gcode, pcode = DTYPES[gdt][0], DTYPES[pdt][0]
+    if check:
+        for r, k in enumerate(ranks):
+            za.zero_scan_nonfinite(grads[r], gcode, P, k.ws)
+        word = torch.stack([k.ws[FOUND].view(torch.int32) for k in ranks]).max()   # the all-reduce (MAX)
+        for k in ranks:
+            k.ws[FOUND].view(torch.int32).fill_(int(word.item()))
+    for r, k in enumerate(ranks):
+        a = za.make_step_args(P, R, grad_dtype=gcode, param_dtype=pcode, master=k.master, exp_avg=k.exp_avg,
+                              exp_avg_sq=k.exp_avg_sq, ctrl=k.ctrl, workspace=k.ws, grads=grads,
+                              params16=k.params16, rank_weights=wts, owner=r, hp=ADAMW_HP,
+                              check_nonfinite=2 if check else 0, state_offset=k.off,
+                              push_params16=[o.params16 for j, o in enumerate(ranks) if j != r])
+        za.zero_step_fused(a)
+
+
+def _compare(ranks, ref):
+    w, m, v = ref.current()
+    rc = ref.ctrl()
+    for r, k in enumerate(ranks):
+        assert torch.equal(k.params16.view(torch.int16), ref.params16.view(torch.int16)), f"params16 of rank {r}"
+        a, b = k.lo - k.off, k.hi - k.off
+        for mine, full, name in ((k.master, w, "master"), (k.exp_avg, m, "m"), (k.exp_avg_sq, v, "v")):
+            assert torch.equal(mine[a:b].view(torch.int32), full[k.lo:k.hi].view(torch.int32)), f"{name} of {r}"
+        c = za.zero_ctrl_read(k.ctrl)
+        assert (c.step, c.skipped, c.loss_scale, c.device_error) == (rc.step, rc.skipped, rc.loss_scale, 0)
+        assert not k.ws.any()
+
+
+def _run(P, R, gdt="bf16", pdt="bf16", steps=3, check=False, S0=1.0, bad=(), token=False, seed=81):
+    ref = FlatZero(P, R, gdt, pdt, loss_scale=S0)
+    w0 = synth.normal(P, 0.02, seed, device="cuda")
+    ref.load_master(w0)
+    ranks = _ranks(P, R, gdt, pdt, w0, S0)
+    for t in range(1, steps + 1):
+        grads_for_step(seed, t, ref.grads, 1e-3, scale=ref.ctrl().loss_scale)
+        if t in bad and P:
+            ref.grads[t % R][(P * 2) // 3] = float("inf")
+        wts = [float(x) for x in synth.token_counts(R, seed, t)] if token else None
+        _emulated_step(ranks, ref.grads, P, R, gdt, pdt, check, wts)
+        ref.step(hp=ADAMW_HP, check=check, rank_weights=wts)
+    torch.cuda.synchronize()
+    _compare(ranks, ref)
+    return ref, ranks
+
+
+@pytest.mark.parametrize("R", [1, 2, 4, 8, 3])
+def test_emulated_ranks_equal_the_single_call_bitwise(R):
+    _run(P=200_003, R=R)
+
+
+@pytest.mark.parametrize("gdt,pdt", [("f32", "bf16"), ("bf16", "f16"), ("f16", "f16")])
+def test_emulated_ranks_dtypes_and_token_weights(gdt, pdt):
+    _run(P=100_019, R=4, gdt=gdt, pdt=pdt, token=True)
+
+
+def test_emulated_ranks_share_the_skip_decision():
+    # fp16 gradients x 2^16; one rank's inf at step 2 skips the step on every
+    # rank (scale halved everywhere), and the next steps apply again.
+    ref, ranks = _run(P=80_021, R=4, gdt="f16", pdt="f16", steps=4, check=True, S0=65536.0, bad=(2,))
+    c = ref.ctrl()
+    assert (c.step, c.skipped, c.loss_scale) == (3, 1, 32768.0)
+
+
+@pytest.mark.parametrize("P,R", [(5, 8), (8, 8), (61, 8), (2048 * 8 + 3, 8)])
+def test_emulated_ranks_small_and_empty_slices(P, R):
+    _run(P=P, R=R, steps=2)
+
+
+def test_emulated_ranks_against_the_oracle():
+    P, R = 30_011, 4
+    ref, ranks = _run(P=P, R=R, steps=2, seed=83)
+    # the single call was the reference above; pin the pair to the oracle too
+    st = oracle.State.create(synth.normal(P, 0.02, 83, device="cuda").double().cpu().numpy())
+    g = [torch.zeros(P, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    for t in (1, 2):
+        grads_for_step(83, t, g, 1e-3)
+        oracle.step(st, [host_grad(x) for x in g], "bf16", ohp(ADAMW_HP))
+    compare_full(ref, st, ranks[2].params16)
+
+
+def test_checkpoint_of_an_offset_slice_round_trips(tmp_path):
+    P, R = 50_017, 4
+    ref, ranks = _run(P=P, R=R, steps=2)
+    k = ranks[1]
+    a = za.make_step_args(P, R, grad_dtype=za.ZERO_BF16, param_dtype=za.ZERO_BF16, master=k.master,
+                          exp_avg=k.exp_avg, exp_avg_sq=k.exp_avg_sq, ctrl=k.ctrl, workspace=k.ws,
+                          grads=ref.grads, params16=k.params16, owner=1, hp=ADAMW_HP, state_offset=k.off)
+    path = str(tmp_path / "rank1.zck")
+    za.zero_checkpoint_save(path, a)
+    saved = [x.clone() for x in (k.master, k.exp_avg, k.exp_avg_sq, k.params16)]
+    for x in (k.master, k.exp_avg, k.exp_avg_sq):
+        x[k.lo - k.off:k.hi - k.off].fill_(7.0)
+    k.params16.zero_()
+    za.zero_checkpoint_load(path, a)
+    torch.cuda.synchronize()
+    lo, hi = k.lo - k.off, k.hi - k.off
+    for x, y in zip((k.master, k.exp_avg, k.exp_avg_sq), saved):
+        assert torch.equal(x[lo:hi].view(torch.int32), y[lo:hi].view(torch.int32))
+    # exactly the slice is re-cast; nothing outside it is written
+    assert torch.equal(k.params16[k.lo:k.hi].view(torch.int16), saved[3][k.lo:k.hi].view(torch.int16))
+    assert not k.params16[:k.lo].view(torch.int16).any() and not k.params16[k.hi:].view(torch.int16).any()
+
+
+# ---------------------------------------------------------------- two processes, one GPU, CUDA IPC
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _ipc_worker(rank, world, port, P, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import synth as sy
+    from gpu_helpers import ADAMW_HP as HP, grads_for_step as fill
+    from mixed_precision_adam_zero_b200.buffers import FlatZero as Flat
+    from mixed_precision_adam_zero_b200.zero2 import Zero2Rank
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    status = "ok"
+    try:
+        z = Zero2Rank(P, "bf16", "bf16")
+        w0 = sy.normal(P, 0.02, 91, device="cuda")
+        z.load_master(w0)
+        everyone = [torch.zeros(P, dtype=torch.bfloat16, device="cuda") for _ in range(world)]
+        for t in (1, 2, 3):
+            fill(91, t, everyone, 1e-3)                 # every rank draws all gradients, keeps its own
+            z.grad.copy_(everyone[rank])
+            z.step(HP, tokens=10 * (rank + 1) + t)
+        torch.cuda.synchronize()
+        ref = Flat(P, world, "bf16", "bf16")
+        ref.load_master(w0)
+        for t in (1, 2, 3):
+            fill(91, t, ref.grads, 1e-3)
+            ref.step(hp=HP, rank_weights=[float(10 * (r + 1) + t) for r in range(world)])
+        torch.cuda.synchronize()
+        w, m, v = ref.current()
+        mine = z.owned()
+        if not torch.equal(z.params16.view(torch.int16), ref.params16.view(torch.int16)):
+            status = "params16 differ"
+        for x, y in zip(mine, (w, m, v)):
+            if not torch.equal(x.view(torch.int32), y[z.lo:z.hi].view(torch.int32)):
+                status = "state differs"
+        c = z.ctrl()
+        if c.step != 3 or c.device_error != 0:
+            status = f"ctrl {c.step} {c.device_error}"
+        dist.barrier()
+        del z
+    except Exception as e:                              # reported, then the process exits non-zero
+        status = f"{type(e).__name__}: {e}"
+    finally:
+        q.put((rank, status))
+        dist.destroy_process_group()
+
+
+def test_two_processes_share_one_gpu_through_cuda_ipc():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ipc_worker, args=(r, 2, port, 100_003, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(300)
+        if p.exitcode is None:
+            p.kill()
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    assert got == [(0, "ok"), (1, "ok")]
+    assert [p.exitcode for p in procs] == [0, 0]
