@@ -236,7 +236,9 @@ const char *zero_last_cuda_error(void);
 size_t zero_ctrl_bytes(void);      /* sizeof(zero_ctrl) */
 size_t zero_workspace_bytes(void); /* ZERO_WORKSPACE_BYTES */
 
-/* Bytes of device memory a tensor-list table for T tensors and R ranks needs. */
+/* Bytes of device memory a tensor-list table for T tensors and R ranks needs
+ * (the tensors' description plus 16 bytes of scratch counters that
+ * zero3_gather uses and leaves zero). */
 size_t zero_list_table_bytes(uint32_t T, uint32_t R);
 
 /* ---------------------------------------------------------- control block */
@@ -441,7 +443,10 @@ int zero3_gather_list_build(uint32_t T, uint32_t R, const uint64_t *numel, void 
 
 /* full_j[r*s_j + k] = shard_{r,j}[k] for every tensor, rank and k < s_j,
  * padding included: the module-level all-gather of ZeRO-3 on one GPU (2 bytes
- * read and 2 written per padded element).  One kernel, asynchronous. */
+ * read and 2 written per padded element).  One kernel, asynchronous; it hands
+ * out work through the table's scratch counters, so calls that may overlap
+ * on the GPU must not share a gather list.  ZERO_EOVERFLOW beyond 2^32 - 2^16
+ * chunks of 32768 elements. */
 int zero3_gather(const zero_tensor_list *gather_list, void *stream);
 
 /* ------------------------------------------------------------ checkpoints */

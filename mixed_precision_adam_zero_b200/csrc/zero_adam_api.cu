@@ -358,7 +358,7 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
 
 // Host copy of a list's table layout: byte offsets of each array.
 struct TableLayout {
-    size_t offs, params, grads, flags, tiles, total;
+    size_t offs, params, grads, flags, tiles, scratch, total;
 };
 
 TableLayout table_layout(uint32_t T, uint32_t R) {
@@ -368,7 +368,8 @@ TableLayout table_layout(uint32_t T, uint32_t R) {
     L.grads = L.params + 8ull * T;
     L.flags = L.grads + 8ull * (size_t)T * R;
     L.tiles = L.flags + ((4ull * T + 15) & ~15ull);
-    L.total = L.tiles + 8ull * ((size_t)T + 1);
+    L.scratch = L.tiles + 8ull * ((size_t)T + 1);
+    L.total = L.scratch + 16;
     return L;
 }
 
@@ -381,6 +382,7 @@ Table device_table(const zero_tensor_list* l) {
     t.grads = reinterpret_cast<const void* const*>(base + L.grads);
     t.flags = reinterpret_cast<const uint32_t*>(base + L.flags);
     t.tiles = reinterpret_cast<const uint64_t*>(base + L.tiles);
+    t.scratch = reinterpret_cast<unsigned int*>(const_cast<char*>(base) + L.scratch);
     t.T = l->T;
     return t;
 }
@@ -706,9 +708,9 @@ int zero3_gather(const zero_tensor_list* l, void* stream) {
                                                  : (const void*)z3_gather_kernel<__half>;
     const int ctas = resident_ctas(fn, &err);
     if (err) return err;
-    const Shape sh = make_shape(0, l->P, ctas);
-    zp.base = sh.base;
-    zp.chunk = sh.chunk;
+    const uint64_t nchunks = (l->P + kZ3Chunk - 1) / kZ3Chunk;
+    if (nchunks > 0xFFFFFFFFull - 65536ull) return ZERO_EOVERFLOW;  // claims stay below 2^32
+    Shape sh{0, kZ3Chunk, (unsigned)(nchunks < (uint64_t)ctas ? nchunks : (uint64_t)ctas)};
     return launch(fn, sh, &zp, static_cast<cudaStream_t>(stream));
 }
 

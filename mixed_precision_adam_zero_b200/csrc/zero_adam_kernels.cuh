@@ -80,6 +80,7 @@ struct Table {
     const void* const* grads;   // [T*R] gradients, tensor-major: grads[j*R + r]
     const uint32_t* flags;      // [T] bit 0: vector path allowed
     const uint64_t* tiles;      // [T+1] vector tiles of tensors 0..j-1 (whole-vector calls)
+    unsigned int* scratch;      // [4] ZeRO-3 gather: chunks claimed, CTAs finished (zero between calls)
     uint32_t T;
 };
 
@@ -646,13 +647,8 @@ struct Z3Params {
     uint32_t R;
 };
 
-template <class Pm>
-__global__ void __launch_bounds__(kThreads) z3_gather_kernel(const __grid_constant__ Z3Params p) {
-    uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
-    uint64_t b = a + p.chunk;
-    if (a < p.lo) a = p.lo;
-    if (b > p.hi) b = p.hi;
-    if (a >= b) return;
+// Elements [a, b) of the padded concatenation.
+__device__ __forceinline__ void z3_copy_range(const Z3Params& p, uint64_t a, uint64_t b) {
     uint32_t j = find_tensor(p.tab, a);
     uint64_t x = a;
     while (x < b) {
@@ -689,6 +685,31 @@ __global__ void __launch_bounds__(kThreads) z3_gather_kernel(const __grid_consta
             x = end;
         }
         ++j;
+    }
+}
+
+// Chunks of kZ3Chunk elements are handed out dynamically: CTA b starts on
+// chunk b, then claims chunks from gridDim.x on through the table's scratch
+// counter; the last CTA to finish clears the counters for the next call.
+constexpr uint64_t kZ3Chunk = 32768;
+
+template <class Pm>
+__global__ void __launch_bounds__(kThreads) z3_gather_kernel(const __grid_constant__ Z3Params p) {
+    __shared__ uint64_t s_next;
+    unsigned int* sc = p.tab.scratch;
+    const uint64_t nchunks = (p.hi + kZ3Chunk - 1) / kZ3Chunk;
+    uint64_t c = blockIdx.x;
+    while (c < nchunks) {
+        if (threadIdx.x == 0) s_next = (uint64_t)gridDim.x + atomicAdd(&sc[0], 1u);
+        const uint64_t a = c * kZ3Chunk;
+        z3_copy_range(p, a, a + kZ3Chunk < p.hi ? a + kZ3Chunk : p.hi);
+        __syncthreads();
+        c = s_next;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0 && atomicAdd(&sc[1], 1u) == gridDim.x - 1) {
+        sc[0] = 0u;
+        sc[1] = 0u;
     }
 }
 

@@ -207,7 +207,8 @@ def test_wait_timeout_selftest_argument_errors():
 
 def test_list_table_bytes():
     T, R = 292, 4
-    assert za.zero_list_table_bytes(T, R) == 8 * (T + 1) + 8 * T + 8 * T * R + ((4 * T + 15) // 16) * 16 + 8 * (T + 1)
+    assert za.zero_list_table_bytes(T, R) == 8 * (T + 1) + 8 * T + 8 * T * R + ((4 * T + 15) // 16) * 16 + \
+        8 * (T + 1) + 16
 
 
 def test_noalloc_step_refuses_a_caller_workspace():

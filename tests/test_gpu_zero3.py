@@ -80,3 +80,43 @@ def test_rank_steps_over_shards_equal_the_whole_step(R):
     full, _ = _gather(numels, R, shard_bufs, "bf16")
     for j, n in enumerate(numels):
         assert torch.equal(full[j][:n].view(torch.int16), whole.params16[j].view(torch.int16))
+
+
+def test_repeated_gathers_reuse_the_list_and_leave_its_scratch_zero():
+    # Work is handed out through counters in the table: every call must
+    # start from zero and leave them zero.  Sizes span many 32768-element
+    # chunks with ragged ends, and the shards change between calls.
+    R = 4
+    numels = [3 * 32768 * R + 11, 5, 32768 * R, 777_777]
+    shards = [[torch.zeros(-(-n // R), dtype=torch.bfloat16, device="cuda") for n in numels] for _ in range(R)]
+    full = [torch.zeros(R * -(-n // R), dtype=torch.bfloat16, device="cuda") for n in numels]
+    nb = za.zero_list_table_bytes(len(numels), R)
+    table = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    gl = za.zero3_gather_list_build(numels, full, shards, za.ZERO_BF16, table, nb)
+    before = table.clone()
+    for call in range(3):
+        for r in range(R):
+            for j in range(len(numels)):
+                shards[r][j].copy_(synth.normal(shards[r][j].numel(), 1.0, 7000 + 100 * call + 10 * r + j,
+                                                device="cuda", dtype=torch.bfloat16))
+        za.zero3_gather(gl)
+        torch.cuda.synchronize()
+        for j in range(len(numels)):
+            want = torch.cat([shards[r][j] for r in range(R)])
+            assert torch.equal(full[j].view(torch.int16), want.view(torch.int16)), (call, j)
+        assert torch.equal(table, before)                 # scratch counters back to zero
+
+
+def test_gather_of_the_gpt2_medium_list_in_the_benchmark_configuration():
+    # The benchmark's ZeRO-3 workload: the 292 GPT-2-medium tensors, R = 4,
+    # every padded element compared.
+    R = 4
+    numels = [n for _, n in synth.gpt2_medium_tensors()]
+    shards = [[torch.empty(-(-n // R), dtype=torch.bfloat16, device="cuda") for n in numels] for _ in range(R)]
+    for r in range(R):
+        for j, b in enumerate(shards[r]):      # small integers: exact in bf16, distinct along each shard
+            b.copy_((torch.arange(b.numel(), device="cuda") * 7 + 13 * r + j) % 201 - 100)
+    full, _ = _gather(numels, R, shards, "bf16")
+    for j in range(len(numels)):
+        want = torch.cat([shards[r][j] for r in range(R)])
+        assert torch.equal(full[j].view(torch.int16), want.view(torch.int16)), j
