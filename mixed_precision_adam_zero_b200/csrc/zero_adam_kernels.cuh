@@ -1,11 +1,15 @@
 // zero_adam_kernels.cuh -- sm_100a kernels of the fused ZeRO-2/3 Adam step.
 //
 // The step is HBM-bound (about 25 flops against 2R+26 bytes per parameter),
-// so it is written as streaming kernels, not as tensor-core work:
-//   * one CTA per slot of a persistent grid (SMs x resident CTAs), each CTA
-//     owning one contiguous range of the flat index space, so every CTA
-//     streams sequential addresses and the ranges balance to within 8
-//     elements;
+// so it is written as streaming kernels, not as tensor-core work.  This file
+// holds the shared arithmetic and the register-staged kernels (the step for
+// rank counts without a staged instance, the overflow scan, the 16-bit
+// cast, the ZeRO-3 gather, the accumulation); zero_adam_bulk.cuh holds the
+// shared-memory staged kernels that the common rank counts run.
+//   * register kernels: one CTA per slot of a persistent grid (SMs x
+//     resident CTAs), each CTA owning one contiguous range of the flat index
+//     space, so every CTA streams sequential addresses and the ranges
+//     balance to within 8 elements;
 //   * 128-bit loads and stores with the streaming (evict-first) cache hint;
 //     one vector is 8 elements: one 16-byte load per 16-bit gradient, two per
 //     fp32 array;
@@ -18,9 +22,10 @@
 //     even where the ranks' gradients nearly cancel.  The chain is the same
 //     in the vector and the scalar path, so results are bitwise reproducible;
 //   * grid-level results (the inf/NaN flag, the step counter) use a
-//     last-block-done epilogue: each CTA fences and bumps an arrival counter
-//     in the workspace, and the CTA that arrives last updates the control
-//     block and re-zeroes the workspace.  Nothing spins or waits.
+//     last-block-done epilogue: each CTA adds its packed arrival (count,
+//     inf/NaN, timeout) to one word of the workspace, and the CTA whose
+//     atomic completes the count updates the control block and re-zeroes
+//     the workspace.  No kernel here spins or waits.
 //
 // Sources of the arithmetic ("Deep dive: DeepSpeed", "Reduce first, then
 // update the owned slice"; AdamW of the "ZeRO" documentation page): see
