@@ -417,6 +417,8 @@ def run_gpu(args) -> None:
                 "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
                 "traffic": traffic,
+                # the ncu-measured DRAM bytes of one launch over the live launch time
+                "traffic_gbs": traffic / (per_launch_ms * 1e-3) / 1e9 if traffic else None,
                 "kernel": roofline_kernel(args.workload),
                 "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms,
             },
