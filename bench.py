@@ -334,7 +334,9 @@ def run_gpu(args) -> None:
         torch.cuda.synchronize()
     barrier()
     total_ms = starts[0].elapsed_time(ends[-1])
-    per_launch_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    per_launch = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    per_launch_ms = statistics.fmean(per_launch)
+    median_launch_ms = statistics.median(per_launch)
 
     # end to end: host (pinned) gradients copied in, 16-bit parameters read back, every step.
     # The read-back of step k runs on its own stream, on the device-to-host
@@ -377,7 +379,8 @@ def run_gpu(args) -> None:
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e0.elapsed_time(e1)
-    total_ms, per_launch_ms, e2e_ms = max_over_ranks([total_ms, per_launch_ms, e2e_ms], world, device)
+    total_ms, per_launch_ms, median_launch_ms, e2e_ms = max_over_ranks(
+        [total_ms, per_launch_ms, median_launch_ms, e2e_ms], world, device)
     ctrl = z.ctrl()
 
     if rank == 0:
@@ -420,7 +423,7 @@ def run_gpu(args) -> None:
                 # the ncu-measured DRAM bytes of one launch over the live launch time
                 "traffic_gbs": traffic / (per_launch_ms * 1e-3) / 1e9 if traffic else None,
                 "kernel": roofline_kernel(args.workload),
-                "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms,
+                "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms, "launch_ms_median": median_launch_ms,
             },
             "e2e": {
                 "value": job_throughput(world, P, K_e2e, e2e_ms), "unit": UNIT, "steps": K_e2e,

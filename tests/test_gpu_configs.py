@@ -138,3 +138,14 @@ def test_llama3b_list():
     assert z.P == 3_212_749_824 and len(tensors) == 254
     z.load_master(synth.normal(z.P, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device="cuda"))
     _sampled_run(z, gbufs, pbuf, 5, wl, "bf16")
+
+
+def test_flat_beyond_2_to_the_31():
+    """P = 2^31 + 13 flat, R = 2, bf16, 3 steps: 64-bit element indices in
+    the staged flat kernel (tile starts, owner bounds and the ragged tail all
+    beyond 2^31), sampled around 2^31 and at both ends."""
+    P, R, wl = 2**31 + 13, 2, synth.WORKLOADS["flat1p5b"]
+    z = FlatZero(P, R, "bf16", "bf16")
+    z.load_master(synth.normal(P, 0.02, synth.seed_for(wl, synth.KIND_MASTER, 1), device="cuda"))
+    near = [2**31 + d for d in range(-20, 13)] + [2**31 - 2048 * k for k in (1, 2, 3)]
+    _sampled_run(z, z.grads, z.params16, 3, wl, "bf16", extra=near, n_random=200_000)
