@@ -648,7 +648,7 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant_
 // concatenation [0, sum_j R*s_j).
 struct Z3Params {
     Table tab;
-    uint64_t lo, hi, base, chunk;
+    uint64_t lo, hi;  // the launch covers [lo, hi) of the padded concatenation (lo = 0)
     uint32_t R;
 };
 
