@@ -104,9 +104,10 @@ def test_emulated_ranks_equal_the_single_call_bitwise(R):
     _run(P=200_003, R=R)
 
 
+@pytest.mark.parametrize("R", [4, 8])
 @pytest.mark.parametrize("gdt,pdt", [("f32", "bf16"), ("bf16", "f16"), ("f16", "f16")])
-def test_emulated_ranks_dtypes_and_token_weights(gdt, pdt):
-    _run(P=100_019, R=4, gdt=gdt, pdt=pdt, token=True)
+def test_emulated_ranks_dtypes_and_token_weights(gdt, pdt, R):
+    _run(P=100_019, R=R, gdt=gdt, pdt=pdt, token=True)
 
 
 def test_emulated_ranks_share_the_skip_decision():
