@@ -175,6 +175,18 @@ typedef struct zero_step_args {
                                      stored there as well as into params16:
                                      the parameter all-gather, fused into the
                                      step. */
+    uint32_t n_grads;             /* 0: the R ranks' gradients; else this many
+                                     gradient buffers are reduced (e.g. 1: an
+                                     owner's already-reduced accumulation
+                                     slice), with rank_weights of n_grads
+                                     entries; R still sets the partition */
+    uint32_t reserved2;           /* zero */
+    uint64_t grad_offset;         /* the gradient buffers hold elements from
+                                     flat index grad_offset on (element i at
+                                     i - grad_offset): a multiple of 8, at
+                                     most lo; then check_nonfinite may not be
+                                     1 (scan with zero_scan_nonfinite and use
+                                     2).  0 for buffers of P elements. */
 } zero_step_args;
 
 /* Most push targets of one call (an NVLink domain's GPUs). */
@@ -384,6 +396,11 @@ typedef struct zero_accum_args {
                                     it is read or written) */
     int32_t path;                /* ZERO_PATH_AUTO (0), ZERO_PATH_REGISTER or
                                     ZERO_PATH_STAGED (see below) */
+    uint64_t accum_offset;       /* accum holds elements from flat index
+                                    accum_offset on (element i at
+                                    i - accum_offset), so an owner can keep
+                                    only its slice: a multiple of 8, at most
+                                    the slice's first element; 0 for [P] */
 } zero_accum_args;
 
 #define ZERO_PATH_AUTO 0

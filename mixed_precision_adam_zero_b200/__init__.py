@@ -85,7 +85,8 @@ class zero_step_args(ctypes.Structure):
                 ("check_nonfinite", ctypes.c_int32), ("growth_interval", ctypes.c_uint32),
                 ("ctrl", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
                 ("state_offset", ctypes.c_uint64), ("n_push", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
-                ("push_params16", ctypes.POINTER(ctypes.c_void_p))]
+                ("push_params16", ctypes.POINTER(ctypes.c_void_p)), ("n_grads", ctypes.c_uint32),
+                ("reserved2", ctypes.c_uint32), ("grad_offset", ctypes.c_uint64)]
 
 
 class zero_accum_args(ctypes.Structure):
@@ -94,7 +95,7 @@ class zero_accum_args(ctypes.Structure):
                 ("grads", ctypes.POINTER(ctypes.c_void_p)),
                 ("rank_weights", ctypes.POINTER(ctypes.c_double)), ("accum", ctypes.c_void_p),
                 ("scale", ctypes.c_double), ("workspace", ctypes.c_void_p), ("ctrl", ctypes.c_void_p),
-                ("path", ctypes.c_int32)]
+                ("path", ctypes.c_int32), ("accum_offset", ctypes.c_uint64)]
 
 
 class zero_tensor_list(ctypes.Structure):
@@ -252,7 +253,8 @@ def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master,
                    hp: Tuple[float, float, float, float, float] = (1e-3, 0.9, 0.999, 1e-8, 0.0),
                    check_nonfinite: int = 0, growth_interval: int = 0, reduced_out=None,
                    master2=None, exp_avg2=None, exp_avg_sq2=None, state_offset: int = 0,
-                   push_params16: Optional[Sequence] = None) -> zero_step_args:
+                   push_params16: Optional[Sequence] = None, n_grads: int = 0,
+                   grad_offset: int = 0) -> zero_step_args:
     """Fill a zero_step_args (the returned struct keeps its host arrays alive)."""
     a = zero_step_args()
     a.P, a.R, a.owner = P, R, owner
@@ -274,6 +276,7 @@ def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master,
     a.growth_interval = growth_interval
     a.ctrl, a.workspace = _ptr(ctrl), _ptr(workspace)
     a.state_offset = state_offset
+    a.n_grads, a.grad_offset = n_grads, grad_offset
     if push_params16:
         arr = (ctypes.c_void_p * len(push_params16))(*[_ptr(t) for t in push_params16])
         a._push_keep = arr
@@ -323,7 +326,7 @@ def zero_gather_params_list(master, lst: zero_tensor_list, stream=None) -> None:
 
 def make_accum_args(P: int, R: int, *, grad_dtype: int, grads: Sequence, accum, scale: float, first: bool,
                     rank_weights: Optional[Sequence[float]] = None, owner: int = -1, workspace=None,
-                    ctrl=None, path: int = ZERO_PATH_AUTO) -> zero_accum_args:
+                    ctrl=None, path: int = ZERO_PATH_AUTO, accum_offset: int = 0) -> zero_accum_args:
     """Fill a zero_accum_args (the returned struct keeps its host arrays alive)."""
     a = zero_accum_args()
     a.P, a.R, a.owner, a.grad_dtype, a.first = P, R, owner, grad_dtype, int(bool(first))
@@ -338,6 +341,7 @@ def make_accum_args(P: int, R: int, *, grad_dtype: int, grads: Sequence, accum, 
     a.scale = float(scale)
     a.workspace, a.ctrl = _ptr(workspace), _ptr(ctrl)
     a.path = path
+    a.accum_offset = accum_offset
     return a
 
 

@@ -210,6 +210,7 @@ int check_hparams(const zero_adam_hparams& h) {
 }
 
 bool is_grad_dtype(int32_t d) { return d == ZERO_F32 || d == ZERO_BF16 || d == ZERO_F16; }
+uint64_t grad_bytes(int32_t d) { return d == ZERO_F32 ? 4u : 2u; }
 bool is_param_dtype(int32_t d) { return d == ZERO_BF16 || d == ZERO_F16; }
 
 // Checks shared by the flat and the list step; fills the rank weights, the
@@ -223,7 +224,9 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     if (a->check_nonfinite < 0 || a->check_nonfinite > 2) return ZERO_EINVAL;
     if (a->n_push > ZERO_MAX_PUSH) return ZERO_ERANGE;
     if (a->reserved != 0u || (a->n_push > 0 && a->push_params16 == nullptr)) return ZERO_EINVAL;
-    if ((a->state_offset & 7u) != 0) return ZERO_EALIGN;
+    if ((a->state_offset & 7u) != 0 || (a->grad_offset & 7u) != 0) return ZERO_EALIGN;
+    if (a->n_grads > ZERO_MAX_RANKS) return ZERO_ERANGE;
+    if (a->reserved2 != 0u || (a->grad_offset != 0 && a->check_nonfinite == 1)) return ZERO_EINVAL;
     if (a->P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
     int rc = check_hparams(a->hp);
     if (rc) return rc;
@@ -240,16 +243,18 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     }
     if (!aligned16(a->reduced_out)) return ZERO_EALIGN;
 
-    // Rank weights as given (float64) and their sum, in rank order.
+    // Rank weights as given (float64) and their sum, in rank order, over the
+    // gradient buffers the call reduces (the R ranks', or n_grads of them).
+    const uint32_t ng = a->n_grads ? a->n_grads : a->R;
     double wsum = 0.0;
-    for (uint32_t r = 0; r < a->R; ++r) {
+    for (uint32_t r = 0; r < ng; ++r) {
         const double wr = a->rank_weights ? a->rank_weights[r] : 1.0;
         if (!finite_nonneg(wr)) return ZERO_EINVAL;
         wsum += wr;
     }
     if (!(wsum > 0.0) || !std::isfinite(wsum)) return ZERO_EINVAL;
     std::memset(kp, 0, sizeof(*kp));
-    for (uint32_t r = 0; r < a->R; ++r) kp->wt[r] = a->rank_weights ? a->rank_weights[r] : 1.0;
+    for (uint32_t r = 0; r < ng; ++r) kp->wt[r] = a->rank_weights ? a->rank_weights[r] : 1.0;
     kp->wsum = wsum;
 
     // State arrays that start at flat index state_offset: the kernels index
@@ -282,7 +287,7 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     kp->h.b2d = h.beta2;
     kp->ctrl = static_cast<zero_ctrl*>(a->ctrl);
     kp->ws = static_cast<Workspace*>(a->workspace);
-    kp->R = a->R;
+    kp->R = ng;  // the reduction's length; the partition is a->R (owner_range)
     kp->growth_interval = a->growth_interval;
     kp->two_set = two ? 1 : 0;
     return ZERO_OK;
@@ -301,7 +306,7 @@ template <bool LIST>
 int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
     uint64_t lo, hi;
     owner_range(a, &lo, &hi);
-    if (a->state_offset > lo && lo < hi) return ZERO_EINVAL;
+    if ((a->state_offset > lo || a->grad_offset > lo) && lo < hi) return ZERO_EINVAL;
     kp->lo = lo;
     kp->hi = hi;
     int err = ZERO_OK;
@@ -325,7 +330,7 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
     } else {
         kp->check = check ? 1 : 0;
     }
-    const Kern k = step_kern(LIST, kp->npush > 0, a->grad_dtype, a->param_dtype, a->R);
+    const Kern k = step_kern(LIST, kp->npush > 0, a->grad_dtype, a->param_dtype, kp->R);
     const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;
     const Shape sh = make_shape(lo, hi, ctas);
@@ -529,10 +534,14 @@ int zero_step_fused(const zero_step_args* a, void* stream) {
     if (a->grads == nullptr) return ZERO_EINVAL;
     if (a->P > 0 && a->params16 == nullptr) return ZERO_EINVAL;
     if (!aligned16(a->params16)) return ZERO_EALIGN;
-    for (uint32_t r = 0; r < a->R; ++r) {
+    // Gradient buffers that start at flat index grad_offset: moved back like
+    // the state arrays (only indices >= grad_offset are dereferenced).
+    const uintptr_t gback = (uintptr_t)(a->grad_offset * grad_bytes(a->grad_dtype));
+    for (uint32_t r = 0; r < kp.R; ++r) {
         if (a->P > 0 && a->grads[r] == nullptr) return ZERO_EINVAL;
         if (!aligned16(a->grads[r])) return ZERO_EALIGN;
-        kp.grads[r] = a->grads[r];
+        kp.grads[r] = a->grads[r] ? reinterpret_cast<const void*>(reinterpret_cast<uintptr_t>(a->grads[r]) - gback)
+                                  : nullptr;
     }
     kp.params16 = a->params16;
     return run_step<false>(a, &kp, static_cast<cudaStream_t>(stream));
@@ -544,7 +553,8 @@ int zero_step_fused_list(const zero_step_args* a, const zero_tensor_list* l, voi
     if (rc) return rc;
     if ((rc = check_list(l))) return rc;
     if (a->grads != nullptr || a->params16 != nullptr) return ZERO_EINVAL;
-    if (a->state_offset != 0 || a->n_push != 0) return ZERO_EINVAL;  // multi-GPU fields: flat calls only
+    if (a->state_offset != 0 || a->n_push != 0 || a->n_grads != 0 || a->grad_offset != 0)
+        return ZERO_EINVAL;  // multi-GPU fields: flat calls only
     if (a->P != l->P || a->R != l->R || a->grad_dtype != l->grad_dtype || a->param_dtype != l->param_dtype)
         return ZERO_EINVAL;
     kp.tab = device_table(l);
@@ -582,7 +592,11 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     if (!(wsum > 0.0) || !std::isfinite(wsum)) return ZERO_EINVAL;
     ap.inv_wsum = 1.0 / wsum;
     ap.scale = a->scale;
-    ap.acc = a->accum;
+    if ((a->accum_offset & 7u) != 0) return ZERO_EALIGN;
+    // An accumulator that starts at flat index accum_offset is moved back like
+    // the step's state arrays (only indices >= accum_offset are dereferenced).
+    ap.acc = a->accum ? reinterpret_cast<float*>(reinterpret_cast<uintptr_t>(a->accum) - a->accum_offset * 4u)
+                      : nullptr;
     ap.ws = static_cast<Workspace*>(a->workspace);
     ap.ctrl = static_cast<zero_ctrl*>(a->ctrl);
     ap.R = a->R;
@@ -596,6 +610,7 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
         ap.hi = (uint64_t)((P * ((uint32_t)a->owner + 1u)) / a->R);
     }
     if (ap.lo >= ap.hi) return ZERO_OK;
+    if (a->accum_offset > ap.lo) return ZERO_EINVAL;
     int err = ZERO_OK;
     const bool staged = a->path == ZERO_PATH_STAGED ||
                         (a->path == ZERO_PATH_AUTO && can_stage && ap.hi - ap.lo >= kStagedAccumMinElems);

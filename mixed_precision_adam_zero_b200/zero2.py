@@ -37,9 +37,10 @@ import torch
 import torch.distributed as dist
 from torch.multiprocessing.reductions import reduce_tensor
 
-from . import (ZERO_WORKSPACE_FOUND_OFFSET, make_step_args, zero_checkpoint_load, zero_checkpoint_save,
-               zero_ctrl_bytes, zero_ctrl_init, zero_ctrl_read, zero_gather_params, zero_partition_bounds,
-               zero_scan_nonfinite, zero_step_fused, zero_workspace_init)
+from . import (ZERO_F32, ZERO_WORKSPACE_FOUND_OFFSET, make_accum_args, make_step_args, zero_accumulate_grads,
+               zero_checkpoint_load, zero_checkpoint_save, zero_ctrl_bytes, zero_ctrl_init, zero_ctrl_read,
+               zero_gather_params, zero_partition_bounds, zero_scan_nonfinite, zero_step_fused,
+               zero_workspace_init)
 from .buffers import DTYPES
 
 
@@ -191,6 +192,42 @@ class Zero2Rank:
         else:
             self._barrier()
         zero_step_fused(self.step_args(hp, check, weights, growth_interval), self._s())
+        self._barrier()
+
+    # ------------------------------------------------------------ micro-steps
+
+    def accumulate(self, *, first: bool, scale: float, tokens: Optional[int] = None) -> None:
+        """Reduce this micro-batch's gradients (every rank's `grad`) into
+        this rank's fp32 accumulation slice: the reduce-scatter on every
+        backward call of ZeRO-2 ("Communication volume isn't elapsed time"),
+        keeping only the owned slice between calls.  `first` starts the
+        window; `scale` is typically 1 / micro-batches per update."""
+        if not hasattr(self, "accum"):
+            self.accum = torch.zeros_like(self.master)          # [state_offset, hi), like the state
+        weights = gather_weights(tokens, self.group, self.device)
+        self._barrier()                                         # every rank's micro-batch gradient is complete
+        zero_accumulate_grads(make_accum_args(
+            self.P, self.R, grad_dtype=self.gcode, grads=self.peer_grads, accum=self.accum, scale=scale,
+            first=first, rank_weights=weights, owner=self.r, workspace=self.workspace, ctrl=self.ctrl_buf,
+            accum_offset=self.state_offset), stream=self._s())
+        self._barrier()                                         # no rank still reads a gradient
+
+    def step_accumulated(self, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), *, check: bool = False,
+                         growth_interval: int = 0) -> None:
+        """The update over the accumulated slice: the owner's slice is already
+        reduced, so the step reads one fp32 buffer; the 16-bit results are
+        pushed into every replica as in `step`."""
+        if check:
+            zero_scan_nonfinite(self.accum, ZERO_F32, self.accum.numel(), self.workspace, self._s())
+            combine_found(self._found, self.group)
+        args = make_step_args(
+            self.P, self.R, grad_dtype=ZERO_F32, param_dtype=self.pcode, master=self.master,
+            exp_avg=self.exp_avg, exp_avg_sq=self.exp_avg_sq, ctrl=self.ctrl_buf, workspace=self.workspace,
+            grads=[self.accum], params16=self.params16, owner=self.r, hp=hp,
+            check_nonfinite=2 if check else 0, growth_interval=growth_interval, state_offset=self.state_offset,
+            push_params16=[t for j, t in enumerate(self.peer_params16) if j != self.r], n_grads=1,
+            grad_offset=self.state_offset)
+        zero_step_fused(args, self._s())
         self._barrier()
 
     def ctrl(self):

@@ -36,7 +36,7 @@ def test_struct_layouts_match_the_header():
     assert za.zero_workspace_bytes() == za.ZERO_WORKSPACE_BYTES == 256
     # zero_step_args: 5 ints + 2 host pointers + 8 device pointers + hparams + 2 ints + 2 pointers,
     # then state_offset, n_push, reserved and the push array
-    assert ctypes.sizeof(za.zero_step_args) == 8 + 4 * 4 + 8 * 2 + 8 * 8 + 40 + 8 + 16 + 8 + 4 + 4 + 8
+    assert ctypes.sizeof(za.zero_step_args) == 8 + 4 * 4 + 8 * 2 + 8 * 8 + 40 + 8 + 16 + 8 + 4 + 4 + 8 + 4 + 4 + 8
 
 
 def test_partition_bounds_match_the_oracle_bit_exactly():
@@ -129,6 +129,11 @@ def _args(**over):
     (dict(push_params16=[A] * 73), za.ZERO_ERANGE),
     (dict(push_params16=[A, A + 2]), za.ZERO_EALIGN),
     (dict(push_params16=[A, None]), za.ZERO_EINVAL),
+    (dict(n_grads=300), za.ZERO_ERANGE),
+    (dict(n_grads=2, rank_weights=[1, -1]), za.ZERO_EINVAL),      # weights over the n_grads buffers
+    (dict(grad_offset=4, owner=1), za.ZERO_EALIGN),
+    (dict(grad_offset=256, owner=1), za.ZERO_EINVAL),              # beyond owner 1's first element (250)
+    (dict(grad_offset=248, owner=1, check_nonfinite=1), za.ZERO_EINVAL),  # sliced gradients: scan first
 ])
 def test_step_argument_errors_are_rejected_on_the_host(over, status):
     a = _args(**over)
@@ -177,7 +182,8 @@ def test_multi_gpu_fields_are_flat_only():
     lst = za.zero_tensor_list()
     lst.table, lst.P, lst.T, lst.R, lst.grad_dtype, lst.param_dtype, lst.table_bytes = A, 1000, 1, 4, \
         za.ZERO_BF16, za.ZERO_BF16, 1 << 20
-    for over in (dict(push_params16=[A]), dict(state_offset=8, owner=1)):
+    for over in (dict(push_params16=[A]), dict(state_offset=8, owner=1), dict(n_grads=1),
+                 dict(grad_offset=8, owner=1)):
         a = _args(grads=None, params16=None, **over)
         with pytest.raises(za.ZeroError) as e:
             za.zero_step_fused_list(a, lst)
@@ -236,6 +242,8 @@ def test_noalloc_step_refuses_a_caller_workspace():
     (dict(path=3), za.ZERO_EINVAL),
     (dict(path=za.ZERO_PATH_STAGED), za.ZERO_EINVAL),                 # staged needs a workspace
     (dict(R=3, grads=[A] * 3, workspace=A, ctrl=A, path=za.ZERO_PATH_STAGED), za.ZERO_EINVAL),
+    (dict(accum_offset=4, owner=1), za.ZERO_EALIGN),
+    (dict(accum_offset=256, owner=1), za.ZERO_EINVAL),               # beyond owner 1's first element (250)
 ])
 def test_accumulate_argument_errors(kw, status):
     args = dict(P=1000, R=4, grad_dtype=za.ZERO_BF16, grads=[A] * 4, accum=A, scale=0.25, first=True)

@@ -158,6 +158,64 @@ def test_checkpoint_of_an_offset_slice_round_trips(tmp_path):
     assert not k.params16[:k.lo].view(torch.int16).any() and not k.params16[k.hi:].view(torch.int16).any()
 
 
+def _run_accumulated(P, R, gas=3, updates=2, check=False, S0=1.0, bad=None, token=False, staged=False, seed=87):
+    """Micro-batches reduced into each owner's own fp32 slice, then the
+    owners' steps over their slices (one gradient buffer each); against the
+    single-GPU accumulation over [0, P) and the step with R = 1."""
+    ref = FlatZero(P, 1, "f32", "bf16", loss_scale=S0, alloc_grads=False)
+    w0 = synth.normal(P, 0.02, seed, device="cuda")
+    ref.load_master(w0)
+    acc = torch.zeros(P, device="cuda")
+    ranks = _ranks(P, R, "bf16", "bf16", w0, S0)
+    for k in ranks:
+        k.acc = torch.full_like(k.master, 0.0)
+    micro = [torch.zeros(P, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    path = za.ZERO_PATH_STAGED if staged else za.ZERO_PATH_REGISTER
+    for u in range(1, updates + 1):
+        for mu in range(gas):
+            grads_for_step(seed, 100 * u + mu, micro, 1e-3, scale=ref.ctrl().loss_scale)
+            if bad is not None and (u, mu) == bad:
+                micro[mu % R][P // 3] = float("nan")
+            wts = [float(x) for x in synth.token_counts(R, seed, 100 * u + mu)] if token else None
+            za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=micro, accum=acc, scale=1.0 / gas,
+                                     first=(mu == 0), rank_weights=wts)
+            for r, k in enumerate(ranks):
+                za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=micro, accum=k.acc, scale=1.0 / gas,
+                                         first=(mu == 0), rank_weights=wts, owner=r, accum_offset=k.off,
+                                         workspace=k.ws, ctrl=k.ctrl, path=path)
+        torch.cuda.synchronize()
+        for k in ranks:                                  # each owner's slice equals the whole array's
+            assert torch.equal(k.acc[k.lo - k.off:k.hi - k.off].view(torch.int32), acc[k.lo:k.hi].view(torch.int32))
+        if check:
+            for k in ranks:
+                za.zero_scan_nonfinite(k.acc, za.ZERO_F32, k.acc.numel(), k.ws)
+            word = torch.stack([k.ws[FOUND].view(torch.int32) for k in ranks]).max()
+            for k in ranks:
+                k.ws[FOUND].view(torch.int32).fill_(int(word.item()))
+        for r, k in enumerate(ranks):
+            a = za.make_step_args(P, R, grad_dtype=za.ZERO_F32, param_dtype=za.ZERO_BF16, master=k.master,
+                                  exp_avg=k.exp_avg, exp_avg_sq=k.exp_avg_sq, ctrl=k.ctrl, workspace=k.ws,
+                                  grads=[k.acc], params16=k.params16, owner=r, hp=ADAMW_HP,
+                                  check_nonfinite=2 if check else 0, state_offset=k.off, n_grads=1,
+                                  grad_offset=k.off, push_params16=[o.params16 for j, o in enumerate(ranks) if j != r])
+            za.zero_step_fused(a)
+        ref.step(hp=ADAMW_HP, check=check, grads=[acc])
+    torch.cuda.synchronize()
+    _compare(ranks, ref)
+    return ref, ranks
+
+
+@pytest.mark.parametrize("R,staged", [(2, False), (4, True), (8, False), (3, False)])
+def test_emulated_accumulation_across_ranks_equals_the_single_gpu_window(R, staged):
+    _run_accumulated(P=120_011, R=R, staged=staged, token=True)
+
+
+def test_emulated_accumulation_shares_the_skip_decision():
+    ref, ranks = _run_accumulated(P=60_013, R=4, updates=3, check=True, S0=1024.0, bad=(2, 1))
+    c = ref.ctrl()
+    assert (c.step, c.skipped, c.loss_scale) == (2, 1, 512.0)
+
+
 # ---------------------------------------------------------------- two processes, one GPU, CUDA IPC
 
 def _free_port():
@@ -204,6 +262,29 @@ def _ipc_worker(rank, world, port, P, q):
         c = z.ctrl()
         if c.step != 3 or c.device_error != 0:
             status = f"ctrl {c.step} {c.device_error}"
+        # then two updates of two micro-batches each, reduced on every micro-batch
+        acc = torch.zeros(P, device="cuda")
+        ref_args = za.make_step_args(P, 1, grad_dtype=za.ZERO_F32, param_dtype=za.ZERO_BF16, master=ref.master[0],
+                                     exp_avg=ref.exp_avg[0], exp_avg_sq=ref.exp_avg_sq[0], ctrl=ref.ctrl_buf,
+                                     workspace=ref.workspace, grads=[acc], params16=ref.params16, hp=HP)
+        for u in (1, 2):
+            for mu in (0, 1):
+                fill(92, 10 * u + mu, everyone, 1e-3)
+                z.grad.copy_(everyone[rank])
+                z.accumulate(first=(mu == 0), scale=0.5)
+                za.zero_accumulate_grads(P, world, grad_dtype=za.ZERO_BF16, grads=everyone, accum=acc, scale=0.5,
+                                         first=(mu == 0))
+            z.step_accumulated(HP)
+            za.zero_step_fused(ref_args)
+        torch.cuda.synchronize()
+        w, m, v = ref.current()
+        if not torch.equal(z.params16.view(torch.int16), ref.params16.view(torch.int16)):
+            status = "params16 differ after accumulation"
+        for x, y in zip(z.owned(), (w, m, v)):
+            if not torch.equal(x.view(torch.int32), y[z.lo:z.hi].view(torch.int32)):
+                status = "state differs after accumulation"
+        if z.ctrl().step != 5:
+            status = f"ctrl after accumulation {z.ctrl().step}"
         dist.barrier()
         del z
     except Exception as e:                              # reported, then the process exits non-zero
