@@ -156,6 +156,16 @@ def test_checkpoint_of_an_offset_slice_round_trips(tmp_path):
     # exactly the slice is re-cast; nothing outside it is written
     assert torch.equal(k.params16[k.lo:k.hi].view(torch.int16), saved[3][k.lo:k.hi].view(torch.int16))
     assert not k.params16[:k.lo].view(torch.int16).any() and not k.params16[k.hi:].view(torch.int16).any()
+    # every rank's shard file: the consolidated fp32 weights are the single call's masters
+    paths = []
+    for r, o in enumerate(ranks):
+        b = za.make_step_args(P, R, grad_dtype=za.ZERO_BF16, param_dtype=za.ZERO_BF16, master=o.master,
+                              exp_avg=o.exp_avg, exp_avg_sq=o.exp_avg_sq, ctrl=o.ctrl, workspace=o.ws,
+                              grads=ref.grads, params16=o.params16, owner=r, hp=ADAMW_HP, state_offset=o.off)
+        paths.append(str(tmp_path / f"r{r}.zck"))
+        za.zero_checkpoint_save(paths[-1], b)
+    full = za.zero_checkpoint_consolidate(paths, P)
+    assert np.array_equal(np.asarray(full).view(np.int32), ref.current()[0].cpu().numpy().view(np.int32))
 
 
 def _run_accumulated(P, R, gas=3, updates=2, check=False, S0=1.0, bad=None, token=False, staged=False, seed=87):
@@ -224,7 +234,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _ipc_worker(rank, world, port, P, q):
+def _ipc_worker(rank, world, port, P, q, tmp):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -285,6 +295,23 @@ def _ipc_worker(rank, world, port, P, q):
                 status = "state differs after accumulation"
         if z.ctrl().step != 5:
             status = f"ctrl after accumulation {z.ctrl().step}"
+        # checkpoint: each rank saves its shard, loses its state and replica,
+        # and restores; the restored slices reach every replica again
+        path = os.path.join(tmp, f"rank{rank}.zck")
+        z.save(path, HP)
+        for x in (z.master, z.exp_avg, z.exp_avg_sq):
+            x.fill_(7.0)
+        z.params16.zero_()
+        torch.cuda.synchronize()
+        dist.barrier()
+        z.load(path, HP)
+        if not torch.equal(z.params16.view(torch.int16), ref.params16.view(torch.int16)):
+            status = "params16 differ after restore"
+        for x, y in zip(z.owned(), (w, m, v)):
+            if not torch.equal(x.view(torch.int32), y[z.lo:z.hi].view(torch.int32)):
+                status = "state differs after restore"
+        if z.ctrl().step != 5:
+            status = f"ctrl after restore {z.ctrl().step}"
         dist.barrier()
         del z
     except Exception as e:                              # reported, then the process exits non-zero
@@ -294,11 +321,11 @@ def _ipc_worker(rank, world, port, P, q):
         dist.destroy_process_group()
 
 
-def test_two_processes_share_one_gpu_through_cuda_ipc():
+def test_two_processes_share_one_gpu_through_cuda_ipc(tmp_path):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_ipc_worker, args=(r, 2, port, 100_003, q)) for r in range(2)]
+    procs = [ctx.Process(target=_ipc_worker, args=(r, 2, port, 100_003, q, str(tmp_path))) for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
