@@ -436,8 +436,8 @@ int noalloc_scratch(void** out) {
 int zadam_host::cast_slice(const float* master, uint64_t state_offset, void* params16, int32_t param_dtype,
                            uint64_t lo, uint64_t hi, void* stream) {
     if (!is_param_dtype(param_dtype) || master == nullptr || params16 == nullptr) return ZERO_EINVAL;
-    if ((state_offset & 7u) != 0 || state_offset > lo || !aligned16(master) || !aligned16(params16))
-        return ZERO_EALIGN;
+    if ((state_offset & 7u) != 0 || !aligned16(master) || !aligned16(params16)) return ZERO_EALIGN;
+    if (state_offset > lo) return ZERO_EINVAL;
     if (lo >= hi) return ZERO_OK;
     GatherParams gp;
     std::memset(&gp, 0, sizeof gp);

@@ -149,3 +149,45 @@ def test_flat_beyond_2_to_the_31():
     z.load_master(synth.normal(P, 0.02, synth.seed_for(wl, synth.KIND_MASTER, 1), device="cuda"))
     near = [2**31 + d for d in range(-20, 13)] + [2**31 - 2048 * k for k in (1, 2, 3)]
     _sampled_run(z, z.grads, z.params16, 3, wl, "bf16", extra=near, n_random=200_000)
+
+
+def test_gpt2m_list_fp16_in_place_two_pass():
+    """The GPT-2-medium list with one state set: the overflow scan runs as a
+    pass of its own before the in-place step (the benchmark's gpt2m_inplace
+    workload), inf planted at steps 3 and 7, 10 steps."""
+    wl = synth.WORKLOADS["gpt2m"]
+    tensors = synth.gpt2_medium_tensors()
+    z, gbufs, pbuf = _list_with_flat_buffers(tensors, 4, "f16", "f16", loss_scale=65536.0, two_set=False)
+    z.load_master(synth.normal(z.P, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device="cuda"))
+    sites = [synth.inf_site(wl, k, 4, z.P)[1] for k in (3, 7)]
+    _sampled_run(z, gbufs, pbuf, 10, wl, "f16", extra=sites, check=True, inf_steps=(3, 7), scale0=65536.0)
+    c = z.ctrl()
+    assert c.step == 8 and c.skipped == 2 and c.loss_scale == 16384.0
+
+
+def test_flat16m_four_micro_batches_per_update_full_oracle():
+    """The benchmark's accumulation workload at full size: 4 micro-batches of
+    8 bf16 rank gradients reduced into the fp32 accumulator (the staged
+    kernel, chosen automatically at this size), then the step over it,
+    2 updates; every element against the oracle."""
+    import mixed_precision_adam_zero_b200 as za
+    P, R, gas, wl = synth.FLAT16M_P, 8, 4, synth.WORKLOADS["flat16m"]
+    z = FlatZero(P, 1, "f32", "bf16", alloc_grads=False)
+    w0 = synth.normal(P, 0.02, synth.seed_for(wl, synth.KIND_MASTER, 2), device="cuda")
+    z.load_master(w0)
+    st = oracle.State.create(w0.double().cpu().numpy())
+    acc = torch.zeros(P, device="cuda")
+    oacc = np.zeros(P, dtype=np.float32)
+    micro = [torch.empty(P, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    for u in (1, 2):
+        for mu in range(gas):
+            _fill(wl, 1000 * u + mu, micro)
+            za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=micro, accum=acc, scale=1.0 / gas,
+                                     first=(mu == 0), workspace=z.workspace, ctrl=z.ctrl_buf)
+            oracle.accumulate(oacc, [host_grad(g) for g in micro], "bf16", 1.0 / gas, first=(mu == 0))
+        torch.cuda.synchronize()
+        assert_close(acc, oacc.astype(np.float64), f"accumulated gradient, update {u}")
+        z.step(hp=ADAMW_HP, grads=[acc])
+        oracle.step(st, [host_grad(acc)], "f32", ohp(ADAMW_HP))
+    torch.cuda.synchronize()
+    compare_full(z, st, z.params16)
