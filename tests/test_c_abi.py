@@ -1,0 +1,25 @@
+"""The C ABI from C: a plain C99 program compiled with gcc against
+include/zero_adam.h and linked with libzero_adam.so runs the host-only entry
+points (no GPU) and checks the pages' values and host-side argument errors."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+import mixed_precision_adam_zero_b200 as za
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_plain_c_program_against_the_header_and_library(tmp_path):
+    za._lib()                                             # built (fails loudly if not)
+    libdir = os.path.dirname(za.library_path())
+    exe = str(tmp_path / "abi_host_check")
+    src = os.path.join(ROOT, "tests", "c_abi", "abi_host_check.c")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"), src,
+                    "-o", exe, "-L", libdir, "-l:libzero_adam.so", f"-Wl,-rpath,{libdir}"], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "all checks passed" in r.stdout
