@@ -23,3 +23,20 @@ def test_plain_c_program_against_the_header_and_library(tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stderr
     assert "all checks passed" in r.stdout
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_plain_c_program_runs_the_step_with_cuda_runtime_memory(tmp_path):
+    za._lib()
+    libdir = os.path.dirname(za.library_path())
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    exe = str(tmp_path / "step_check")
+    src = os.path.join(ROOT, "tests", "c_abi", "step_check.c")
+    subprocess.run(["gcc", "-std=c99", "-O2", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(cuda, "include"), src, "-o", exe, "-L", libdir, "-l:libzero_adam.so",
+                    f"-Wl,-rpath,{libdir}", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                    f"-Wl,-rpath,{os.path.join(cuda, 'lib64')}", "-lm"], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert "matches its closed form" in r.stdout
