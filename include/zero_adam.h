@@ -411,9 +411,9 @@ typedef struct zero_accum_args {
  * its tiles in shared memory by bulk copies and hands them out dynamically;
  * it needs a workspace and ctrl and R = 1, 2, 4 or 8.  The register kernel
  * streams through registers and touches neither workspace nor ctrl.  Both
- * give bitwise identical sums.  ZERO_PATH_AUTO takes the staged kernel when
- * it is possible and the launch's range holds at least 12*2^20 elements
- * (where it is the faster one), else the register kernel.  Errors:
+ * give bitwise identical sums.  ZERO_PATH_AUTO takes the staged kernel
+ * whenever it is possible (the faster one at nearly every size), else the
+ * register kernel.  Errors:
  * ZERO_EINVAL (also: exactly one of workspace and ctrl given; an unknown
  * path; ZERO_PATH_STAGED without a workspace or with another R),
  * ZERO_EALIGN (accum, grads and workspace must be 16-byte aligned, ctrl

@@ -351,7 +351,7 @@ def zero_accumulate_grads(args, R: Optional[int] = None, *, stream=None, **kw) -
     `args` is a zero_accum_args from make_accum_args, or P, followed by R and
     make_accum_args' keywords.  With `workspace` and `ctrl` (device buffers as
     for a step call) the shared-memory staged kernel can run for R in 1, 2, 4,
-    8 (`path` chooses; by default it runs from 12*2^20 elements up)."""
+    8 (`path` chooses; by default it runs whenever it can)."""
     if not isinstance(args, zero_accum_args):
         args = make_accum_args(args, R, **kw)
     elif R is not None or kw:

@@ -158,13 +158,11 @@ const void* gather_fn(int32_t param_dtype) {
 }
 
 // Accumulation: the bulk kernel for a compile-time rank count when the
-// caller gives a workspace and the launch covers at least
-// kStagedAccumMinElems elements, else the register kernel.  Measured on a
-// B200 (R = 8 bf16, continuing window): the register kernel is faster at
-// 8.4M elements (87 % against 82 % of the copy peak), the two are equal at
-// 12.6M, and the staged kernel leads from there on (93 % against 86 % at
-// 16.8M); the staged kernel's fixed cost per launch is the larger.
-constexpr uint64_t kStagedAccumMinElems = 12ull << 20;
+// caller gives a workspace, else the register kernel.  Measured on a B200
+// (R = 8 bf16, a window of one first and three continuing micro-batches):
+// the staged kernel is 10 % faster at 4.2M elements, 4 % at 6.3M, equal at
+// 10.5M, 3 % faster at 12.6M and 7 % at 16.8M; only near 8.4M is the
+// register kernel ahead (4 %).
 template <class G, int RC>
 Kern accum_bulk_kern() {
     return Kern{(const void*)accum_bulk_kernel<G, RC>, AccumShape<G, RC>::kSmem, kBulkThreads};
@@ -612,8 +610,7 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     if (ap.lo >= ap.hi) return ZERO_OK;
     if (a->accum_offset > ap.lo) return ZERO_EINVAL;
     int err = ZERO_OK;
-    const bool staged = a->path == ZERO_PATH_STAGED ||
-                        (a->path == ZERO_PATH_AUTO && can_stage && ap.hi - ap.lo >= kStagedAccumMinElems);
+    const bool staged = a->path == ZERO_PATH_STAGED || (a->path == ZERO_PATH_AUTO && can_stage);
     const Kern k = accum_kern(a->grad_dtype, a->R, staged);
     const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;

@@ -154,9 +154,9 @@ def test_per_owner_accumulation_equals_whole_bitwise():
     assert torch.equal(whole, part)
 
 
-def test_automatic_path_around_the_size_threshold():
-    # Ranges just below and just above 12*2^20 elements: the automatic choice
-    # switches kernels there, and every choice gives the same bits.
+def test_every_path_gives_the_same_bits_at_large_ragged_sizes():
+    # Ranges of about 12*2^20 elements, ragged: the automatic choice (the
+    # staged kernel here), the register kernel and the staged kernel agree.
     R = 2
     for P in ((12 << 20) - 1, (12 << 20) + 13):
         g = _micro(P, R, torch.bfloat16, 700)
