@@ -225,23 +225,12 @@ int zero_checkpoint_load(const char* path, const zero_step_args* a, void* stream
     std::fclose(f);
     if (rc) return rc;
     if ((rc = zero_ctrl_set(a->ctrl, &h.ctrl, stream))) return rc;
-    if (a->params16 != nullptr && n > 0 && a->state_offset != 0) {
-        // Arrays of this rank's slice only: re-cast exactly [lo, hi) into
-        // the local 16-bit parameters (the other ranks' replicas receive
-        // the slice from the caller).
-        return zadam_host::cast_slice(a->master[0], a->state_offset, a->params16, a->param_dtype, lo, hi, stream);
-    }
     if (a->params16 != nullptr && n > 0) {
-        // The 16-bit parameters follow from the restored masters.  The cast
-        // runs over the slice widened to multiples of 8 elements (the cast's
-        // alignment); the extra elements get the cast of their own masters,
-        // which is their value whenever those are final, and every owner's
-        // restore re-casts its own slice last.
-        const uint64_t wlo = lo & ~7ull;
-        uint64_t whi = (hi + 7) & ~7ull;
-        if (whi > a->P) whi = a->P;
-        return zero_gather_params(a->master[0] + wlo, static_cast<unsigned char*>(a->params16) + wlo * 2,
-                                  a->param_dtype, whi - wlo, stream);
+        // The 16-bit parameters of exactly the slice follow from the restored
+        // masters; nothing outside [lo, hi) is read or written, so the arrays
+        // may hold only the slice (state_offset) and the other owners'
+        // elements of the replica are left to their own restores.
+        return zadam_host::cast_slice(a->master[0], a->state_offset, a->params16, a->param_dtype, lo, hi, stream);
     }
     return ZERO_OK;
 }
