@@ -34,6 +34,8 @@ class _Common:
         self.exp_avg_sq = [torch.zeros(P, **f32) for _ in range(sets)]
         self.ctrl_buf = torch.zeros(max(zero_ctrl_bytes(), 64), dtype=torch.uint8, device=self.device)
         self.workspace = torch.zeros(256, dtype=torch.uint8, device=self.device)
+        if self.stream is not None:       # the fills above ran on the current stream
+            self.stream.wait_stream(torch.cuda.current_stream(self.device))
         zero_workspace_init(self.workspace, self._s())
         zero_ctrl_init(self.ctrl_buf, loss_scale, self._s())
 
@@ -75,11 +77,15 @@ class FlatZero(_Common):
             [torch.zeros(P, dtype=self.gtorch, device=self.device) for _ in range(R)] if alloc_grads else None)
 
     def load_master(self, w0: torch.Tensor) -> None:
-        """Masters := w0, moments := 0 (set 0), params16 := RNE(w0)."""
-        self.master[0].copy_(w0)
-        self.exp_avg[0].zero_()
-        self.exp_avg_sq[0].zero_()
-        zero_gather_params(self.master[0], self.params16, self.pcode, self.P, self._s())
+        """Masters := w0, moments := 0 (set 0), params16 := RNE(w0), all on
+        the optimizer's stream (after the current stream's work on w0)."""
+        s = self._s()
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            self.master[0].copy_(w0)
+            self.exp_avg[0].zero_()
+            self.exp_avg_sq[0].zero_()
+        zero_gather_params(self.master[0], self.params16, self.pcode, self.P, s)
 
     def step_args(self, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), rank_weights=None, check=False, owner=-1,
                   growth_interval=0, reduced_out=None, grads: Optional[Sequence] = None):
@@ -107,14 +113,19 @@ class ListZero(_Common):
             [torch.zeros(n, dtype=self.gtorch, device=self.device) for n in self.numels] for _ in range(R)]
         nbytes = zero_list_table_bytes(len(self.numels), R)
         self.table = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
+        self._s().wait_stream(torch.cuda.current_stream(self.device))
         self.list = zero_list_table_build(self.numels, self.params16, self.grads, self.gcode, self.pcode,
                                           self.table, nbytes, self._s())
 
     def load_master(self, w0: torch.Tensor) -> None:
-        self.master[0].copy_(w0)
-        self.exp_avg[0].zero_()
-        self.exp_avg_sq[0].zero_()
-        zero_gather_params_list(self.master[0], self.list, self._s())
+        """As FlatZero.load_master, for the list's 16-bit tensors."""
+        s = self._s()
+        s.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(s):
+            self.master[0].copy_(w0)
+            self.exp_avg[0].zero_()
+            self.exp_avg_sq[0].zero_()
+        zero_gather_params_list(self.master[0], self.list, s)
 
     def step_args(self, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), rank_weights=None, check=False, owner=-1,
                   growth_interval=0, reduced_out=None):
