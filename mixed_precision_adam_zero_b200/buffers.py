@@ -11,7 +11,8 @@ import torch
 
 from . import (ZERO_BF16, ZERO_F16, ZERO_F32, make_step_args, zero_ctrl_bytes, zero_ctrl_init,
                zero_ctrl_read, zero_gather_params, zero_gather_params_list, zero_list_table_build,
-               zero_list_table_bytes, zero_step_fused, zero_step_fused_list, zero_workspace_init)
+               zero_list_table_bytes, zero_step_fused, zero_step_fused_list, zero_workspace_bytes,
+               zero_workspace_init)
 
 DTYPES = {"f32": (ZERO_F32, torch.float32), "bf16": (ZERO_BF16, torch.bfloat16), "f16": (ZERO_F16, torch.float16)}
 
@@ -33,7 +34,7 @@ class _Common:
         self.exp_avg = [torch.zeros(P, **f32) for _ in range(sets)]
         self.exp_avg_sq = [torch.zeros(P, **f32) for _ in range(sets)]
         self.ctrl_buf = torch.zeros(max(zero_ctrl_bytes(), 64), dtype=torch.uint8, device=self.device)
-        self.workspace = torch.zeros(256, dtype=torch.uint8, device=self.device)
+        self.workspace = torch.zeros(zero_workspace_bytes(), dtype=torch.uint8, device=self.device)
         if self.stream is not None:       # the fills above ran on the current stream
             self.stream.wait_stream(torch.cuda.current_stream(self.device))
         zero_workspace_init(self.workspace, self._s())

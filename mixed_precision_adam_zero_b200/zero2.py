@@ -40,7 +40,7 @@ from torch.multiprocessing.reductions import reduce_tensor
 from . import (ZERO_F32, ZERO_WORKSPACE_FOUND_OFFSET, make_accum_args, make_step_args, zero_accumulate_grads,
                zero_checkpoint_load, zero_checkpoint_save, zero_ctrl_bytes, zero_ctrl_init, zero_ctrl_read,
                zero_gather_params, zero_partition_bounds, zero_scan_nonfinite, zero_step_fused,
-               zero_workspace_init)
+               zero_workspace_bytes, zero_workspace_init)
 from .buffers import DTYPES
 
 
@@ -141,7 +141,7 @@ class Zero2Rank:
         self.grad = torch.zeros(P, device=self.device, dtype=self.gtorch)
         self.params16 = torch.zeros(P, device=self.device, dtype=self.ptorch)
         self.ctrl_buf = torch.zeros(max(zero_ctrl_bytes(), 64), dtype=torch.uint8, device=self.device)
-        self.workspace = torch.zeros(256, dtype=torch.uint8, device=self.device)
+        self.workspace = torch.zeros(zero_workspace_bytes(), dtype=torch.uint8, device=self.device)
         zero_workspace_init(self.workspace, self._s())
         zero_ctrl_init(self.ctrl_buf, loss_scale, self._s())
         self._found = self.workspace[ZERO_WORKSPACE_FOUND_OFFSET:ZERO_WORKSPACE_FOUND_OFFSET + 4].view(torch.int32)
