@@ -62,6 +62,10 @@ WORKLOADS["flat16m_gas4"] = ("flat", 16_777_259, 8, "bf16", "bf16", False)
 # ZeRO-3 module gather: full padded 16-bit views of every GPT-2-medium tensor
 # from R = 4 rank shards (2 bytes read and 2 written per padded element).
 WORKLOADS["gpt2m_z3gather"] = ("z3gather", "gpt2m", 4, "bf16", "bf16", False)
+# The ZeRO-2 step across GPUs, emulated on one GPU: R owner launches, each over
+# its own state slice, reading every rank's gradient slice and storing its
+# 16-bit results into all R replicas (the pushes land in this GPU's HBM).
+WORKLOADS["flat16m_zero2emu"] = ("zero2emu", 16_777_259, 8, "bf16", "bf16", False)
 
 
 def bytes_per_param(R: int, gdt: str, gas: int = 0) -> int:
@@ -73,6 +77,13 @@ def bytes_per_param(R: int, gdt: str, gas: int = 0) -> int:
     if gas:
         return gas * (GRAD_BYTES[gdt] * R + 4) + (gas - 1) * 4 + 4 + 24 + 2
     return GRAD_BYTES[gdt] * R + 24 + 2
+
+
+def zero2emu_bytes_per_param(R: int, gdt: str) -> int:
+    """The emulated multi-GPU step: every rank's gradient read once by its
+    owner, state read and written, and each 16-bit result stored into R
+    replicas."""
+    return GRAD_BYTES[gdt] * R + 24 + 2 * R
 
 
 def kernel_source_sha() -> str:
@@ -192,6 +203,39 @@ def build_workload(name: str, device):
         z.flat_p16 = fbuf
         z.ctrl = lambda: type("C", (), {"step": 0})()
         return z
+    if kind == "zero2emu":
+        from mixed_precision_adam_zero_b200 import make_step_args, zero_ctrl_init, zero_ctrl_read
+        from mixed_precision_adam_zero_b200.buffers import DTYPES
+        from mixed_precision_adam_zero_b200.zero2 import rank_slice
+        gcode, gt = DTYPES[gdt]
+        pcode, pt = DTYPES[pdt]
+        w0 = synth.normal(size, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device)
+        gbufs = [torch.empty(size, dtype=gt, device=device) for _ in range(R)]
+        for r, g in enumerate(gbufs):
+            synth.fill_normal_(g, 1e-3, synth.seed_for(wl, synth.KIND_GRAD, r, 1))
+        replicas = [w0.to(pt) for _ in range(R)]
+        ranks = []
+        for r in range(R):
+            lo, hi, off, n = rank_slice(size, R, r)
+            st = [torch.zeros(n, device=device) for _ in range(3)]
+            st[0][lo - off:hi - off].copy_(w0[lo:hi])
+            ctrl = torch.zeros(64, dtype=torch.uint8, device=device)
+            zero_ctrl_init(ctrl, 1.0)
+            ws = torch.zeros(256, dtype=torch.uint8, device=device)
+            ranks.append((st, ctrl, ws, off))
+
+        class Emu:
+            pass
+        z = Emu()
+        z.P, z.gbufs, z.check, z.flat_p16 = size, gbufs, False, replicas[0]
+        z.keep = (ranks, replicas)
+        z.owner_args = [make_step_args(size, R, grad_dtype=gcode, param_dtype=pcode, master=st[0], exp_avg=st[1],
+                                       exp_avg_sq=st[2], ctrl=ctrl, workspace=ws, grads=gbufs,
+                                       params16=replicas[r], owner=r, hp=ADAMW, state_offset=off,
+                                       push_params16=[t for j, t in enumerate(replicas) if j != r])
+                        for r, (st, ctrl, ws, off) in enumerate(ranks)]
+        z.ctrl = lambda: zero_ctrl_read(ranks[0][1])
+        return z
     if name in GAS:
         z = FlatZero(size, 1, "f32", pdt, device=device, loss_scale=S, alloc_grads=False)
         gt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt]
@@ -232,6 +276,8 @@ def roofline_kernel(workload: str) -> str:
     kind, size, R, gdt, pdt, scaled = WORKLOADS[workload]
     if kind == "z3gather":
         return "z3_gather_kernel"
+    if kind == "zero2emu":
+        return f"{R} x step_bulk_kernel (flat, push): the owners of an emulated {R}-rank ZeRO-2 step"
     step = ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") + (" (flat)" if kind == "flat" else " (list)")
     gas = GAS.get(workload, 0)
     if gas:
@@ -243,6 +289,8 @@ def roofline_kernel(workload: str) -> str:
 def launches_per_step(z) -> int:
     if hasattr(z, "gl"):
         return 1
+    if hasattr(z, "owner_args"):
+        return len(z.owner_args)
     if getattr(z, "gas", 0):
         return z.gas + 1
     if not z.check:
@@ -295,6 +343,10 @@ def run_gpu(args) -> None:
     if hasattr(z, "gl"):
         from mixed_precision_adam_zero_b200 import zero3_gather
         call = lambda: zero3_gather(z.gl, stream)
+    elif hasattr(z, "owner_args"):
+        def call():
+            for a in z.owner_args:
+                zero_step_fused(a, stream)
     elif getattr(z, "gas", 0):
         step_args = z.step_args(hp=ADAMW, check=z.check, grads=[z.accum])
         gcode = {"bf16": ZERO_BF16, "f16": ZERO_F16, "f32": ZERO_F32}[z.micro_gdt]
@@ -386,7 +438,8 @@ def run_gpu(args) -> None:
     if rank == 0:
         kind, size, R, gdt, pdt, scaled = WORKLOADS[args.workload]
         P = z.P
-        bpp = 4 if kind == "z3gather" else bytes_per_param(R, gdt, GAS.get(args.workload, 0))
+        bpp = 4 if kind == "z3gather" else (zero2emu_bytes_per_param(R, gdt) if kind == "zero2emu" else
+                                            bytes_per_param(R, gdt, GAS.get(args.workload, 0)))
         peaks = measured_peaks()
         peak = peaks.get("hbm_gbs")
         peak_src = "measured" if peak else "fallback"
