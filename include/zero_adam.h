@@ -125,13 +125,14 @@ typedef struct zero_step_args {
                                      slice, with that owner's own ctrl */
     int32_t grad_dtype;           /* ZERO_F32, ZERO_BF16 or ZERO_F16 */
     int32_t param_dtype;          /* ZERO_BF16 or ZERO_F16 */
-    const void *const *grads;     /* HOST array of R device pointers, rank r's
-                                     gradient [P] of grad_dtype (flat call);
-                                     NULL for the list call */
-    const double *rank_weights;   /* HOST array of R weights w_r (token counts:
-                                     finite, >= 0, sum > 0), or NULL for the
-                                     equal-weight mean w_r = 1; used in
-                                     float64 as given */
+    const void *const *grads;     /* HOST array of R device pointers (n_grads
+                                     if set), rank r's gradient [P] of
+                                     grad_dtype (flat call); NULL for the
+                                     list call */
+    const double *rank_weights;   /* HOST array of R (n_grads if set) weights
+                                     w_r (token counts: finite, >= 0, sum >
+                                     0), or NULL for the equal-weight mean
+                                     w_r = 1; used in float64 as given */
     float *master[2];             /* device [P] fp32 master weights */
     float *exp_avg[2];            /* device [P] fp32 first moment m */
     float *exp_avg_sq[2];         /* device [P] fp32 second moment v */
