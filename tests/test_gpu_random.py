@@ -80,3 +80,29 @@ def test_two_optimizers_step_concurrently_on_two_streams():
         for x, y in zip(a, b):
             assert torch.equal(x.view(torch.int16 if x.element_size() == 2 else torch.int32),
                                y.view(torch.int16 if y.element_size() == 2 else torch.int32))
+
+
+def _list_cases(n=10, seed=77):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        T = int(rng.integers(1, 40))
+        kinds = rng.integers(0, 4, size=T)
+        numels = [int(x) for x in np.where(kinds == 0, 0, np.where(kinds == 1, rng.integers(1, 9, size=T),
+                                                                    np.where(kinds == 2, rng.integers(9, 3000, size=T),
+                                                                             rng.integers(3000, 60_000, size=T))))]
+        R = int(rng.integers(1, 10))
+        gdt = ["f32", "bf16", "f16"][int(rng.integers(0, 3))]
+        pdt = ["bf16", "f16"][int(rng.integers(0, 2))]
+        out.append((i, numels, R, gdt, pdt, bool(rng.integers(0, 2)), bool(rng.integers(0, 2)),
+                    bool(rng.integers(0, 2))))
+    return out
+
+
+@pytest.mark.parametrize("case", _list_cases(), ids=lambda c: f"l{c[0]}-T{len(c[1])}-R{c[2]}-{c[3]}-{c[4]}")
+def test_random_tensor_list_against_the_oracle(case):
+    from test_gpu_parity import run_list
+    i, numels, R, gdt, pdt, token, two_set, misalign = case
+    if sum(numels) == 0:
+        numels = numels + [17]
+    run_list(numels, R, gdt, pdt, steps=2, token=token, two_set=two_set, misalign=misalign, seed=300 + i)
