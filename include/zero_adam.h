@@ -36,9 +36,11 @@
  *     the legacy default stream) unless stated otherwise.
  *   - The caller owns and allocates every buffer; the library allocates no
  *     device memory and keeps no state between calls apart from per-device
- *     launch-shape caches.
- *   - "device pointer" means memory of the current CUDA device; sizes are in
- *     elements unless named *_bytes.
+ *     launch-shape caches and the static scratch array behind
+ *     zero_step_fused_noalloc.
+ *   - "device pointer" means memory the current CUDA device can access: its
+ *     own, or another GPU's mapped into this process (the multi-GPU fields
+ *     of zero_step_args); sizes are in elements unless named *_bytes.
  */
 #ifndef ZERO_ADAM_H
 #define ZERO_ADAM_H
@@ -159,8 +161,13 @@ typedef struct zero_step_args {
                                      call leaves it all zero again.  Calls
                                      that may overlap on the GPU need separate
                                      workspaces. */
-    /* Data-parallel across GPUs (flat call only; 0 / NULL otherwise).  The
-     * call updates one owner's slice [lo, hi) as above; then: */
+    /* Data-parallel across GPUs (flat call only; 0 / NULL otherwise): the
+     * call updates one owner's slice [lo, hi) as above, and when every rank
+     * makes the call for its own slice, with the ranks' gradient buffers as
+     * grads and the other ranks' replicas as push targets, the calls
+     * together are the ZeRO-2 step of "Communication volume isn't elapsed
+     * time" (gradient reduce-scatter, local update, all-gather of the
+     * updated parameters).  Then: */
     uint64_t state_offset;        /* master, exp_avg, exp_avg_sq and
                                      reduced_out hold elements from flat index
                                      state_offset on (element i at index
@@ -271,8 +278,9 @@ int zero_ctrl_read(const void *ctrl, zero_ctrl *out, void *stream);
 /* Zero a workspace of ZERO_WORKSPACE_BYTES (cudaMemsetAsync). */
 int zero_workspace_init(void *workspace, void *stream);
 
-/* Overflow scan of one gradient buffer (the check of "Loss scaling", taken
- * ahead of a step with check_nonfinite = 2): sets the workspace's inf/NaN
+/* Overflow scan of one gradient buffer: the inf/NaN check of the step with
+ * loss scaling (given at the top of this file; the pages describe no loss
+ * scaling), taken ahead of a step with check_nonfinite = 2: sets the workspace's inf/NaN
  * word if any of grad[0, n) is inf or NaN, and otherwise leaves it as it
  * is, so several scans accumulate.  grad: device, 16-byte aligned, of
  * grad_dtype.  Asynchronous on `stream`.  Errors: ZERO_EINVAL, ZERO_EALIGN,
