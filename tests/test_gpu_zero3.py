@@ -120,3 +120,41 @@ def test_gather_of_the_gpt2_medium_list_in_the_benchmark_configuration():
     for j in range(len(numels)):
         want = torch.cat([shards[r][j] for r in range(R)])
         assert torch.equal(full[j].view(torch.int16), want.view(torch.int16)), j
+
+
+def test_a_zero3_rank_checkpoint_resumes_bitwise(tmp_path):
+    # A ZeRO-3 rank's state is a flat vector over its shard pieces (a list
+    # call over the whole local vector): the shard file restores it, the
+    # 16-bit shards follow from the masters, and the run continues as if
+    # never interrupted.
+    R, r = 4, 1
+    numels = [1000, 37, 4096 * 3 + 5, 2048, 9]
+    bounds = [za.zero3_shard_bounds(n, R, r) for n in numels]
+    sizes = [hi - lo for lo, hi, _ in bounds]
+
+    def rank():
+        z = ListZero(sizes, R, "bf16", "bf16")
+        z.load_master(synth.normal(z.P, 0.02, 93, device="cuda"))
+        return z
+    a, b = rank(), rank()
+    for k in (1, 2):
+        for z in (a, b):
+            grads_for_step(93, k, z.grads, 1e-3)
+            z.step(hp=ADAMW_HP)
+    path = str(tmp_path / "z3rank1.zck")
+    za.zero_checkpoint_save(path, a.step_args(hp=ADAMW_HP))
+    for x in a.current():
+        x.fill_(5.0)
+    for t in a.params16:
+        t.zero_()
+    za.zero_checkpoint_load(path, a.step_args(hp=ADAMW_HP))
+    za.zero_gather_params_list(a.master[0], a.list)
+    grads_for_step(93, 3, a.grads, 1e-3)
+    grads_for_step(93, 3, b.grads, 1e-3)
+    a.step(hp=ADAMW_HP)
+    b.step(hp=ADAMW_HP)
+    torch.cuda.synchronize()
+    for x, y in zip(a.current(), b.current()):
+        assert torch.equal(x.view(torch.int32), y.view(torch.int32))
+    assert torch.equal(a.flat_params16().view(torch.int16), b.flat_params16().view(torch.int16))
+    assert a.ctrl().step == b.ctrl().step == 3
