@@ -287,3 +287,13 @@ def test_parameter_storage_matches_the_oracle_and_the_pages():
         with pytest.raises(za.ZeroError) as e:
             za.zero_parameter_storage(*bad)
         assert e.value.status == za.ZERO_EINVAL
+
+
+def test_header_constants_match_the_binding():
+    import re
+    text = open(os.path.join(ROOT, "include", "zero_adam.h")).read()
+    defines = {m.group(1): int(m.group(2)) for m in
+               re.finditer(r"^#define (ZERO_[A-Z0-9_]+) \(?(-?\d+)\)?", text, flags=re.M)}
+    assert len(defines) >= 17
+    for name, value in defines.items():
+        assert getattr(za, name) == value, name
