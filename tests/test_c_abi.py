@@ -40,3 +40,25 @@ def test_plain_c_program_runs_the_step_with_cuda_runtime_memory(tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert "matches its closed form" in r.stdout
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_binding_struct_layouts_equal_the_c_compilers(tmp_path):
+    # sizeof and every field offset of the ABI structs, as gcc lays them out
+    # from the header, against the ctypes declarations of the binding
+    import ctypes
+    exe = str(tmp_path / "layout")
+    src = os.path.join(ROOT, "tests", "c_abi", "layout.c")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), src, "-o", exe],
+                   check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    seen = 0
+    for line in filter(None, out):
+        struct, field, value = line.split()
+        cls = getattr(za, struct)
+        if field == "sizeof":
+            assert ctypes.sizeof(cls) == int(value), struct
+        else:
+            assert getattr(cls, field).offset == int(value), (struct, field)
+        seen += 1
+    assert seen >= 50
