@@ -101,8 +101,13 @@ typedef struct zero_ctrl {
     uint32_t last_skipped;    /* 1 if the most recent step call skipped */
     uint32_t device_error;    /* nonzero: a bounded device-side wait of some
                                  step gave up (sticky until reset with
-                                 zero_ctrl_set); that step's results are
-                                 undefined.  Never expected in normal use. */
+                                 zero_ctrl_set).  That step counts as not
+                                 applied: t, parity, S and the growth count
+                                 stay and last_skipped is 1, so a two-set
+                                 optimizer keeps its last complete set; in
+                                 place, the elements the step did reach are
+                                 updated and the rest are not.  Never
+                                 expected in normal use. */
     uint32_t reserved;        /* zero */
 } zero_ctrl;
 
@@ -174,7 +179,8 @@ typedef struct zero_step_args {
                                      i - state_offset), so a rank allocates
                                      only [state_offset, hi).  A multiple of 8,
                                      at most lo; 0 for arrays of P elements. */
-    uint32_t n_push;              /* 0..ZERO_MAX_PUSH */
+    uint32_t n_push;              /* 0..ZERO_MAX_PUSH; nonzero needs
+                                     owner >= 0 (ZERO_EINVAL otherwise) */
     uint32_t reserved;            /* zero */
     void *const *push_params16;   /* HOST array of n_push device pointers,
                                      each [P] of param_dtype: the other ranks'
@@ -291,8 +297,11 @@ int zero_scan_nonfinite(const void *grad, int32_t grad_dtype, uint64_t n, void *
  * counterpart): launches one block whose thread waits, through the same
  * bounded wait as the staged kernels, on a shared-memory barrier that nothing
  * arrives at.  The wait gives up after its limit (about 2 s of GPU time) and
- * the kernel sets ctrl->device_error to 1, then exits normally: no trap, no
- * fault, the context stays usable.  Asynchronous on `stream`; read the
+ * the kernel records the outcome through the step epilogue's control-block
+ * update, as a two-set step with the overflow check on and growth_interval 1
+ * whose wait gave up: device_error = 1 and last_skipped = 1, with step,
+ * skipped, parity, loss_scale and growth_tracker unchanged.  It then exits
+ * normally: no trap, no fault, the context stays usable.  Asynchronous on `stream`; read the
  * result with zero_ctrl_read.  Errors: ZERO_EINVAL (NULL ctrl), ZERO_EALIGN
  * (ctrl not 8-byte aligned), ZERO_ECUDA. */
 int zero_selftest_wait_timeout(void *ctrl, void *stream);
@@ -365,7 +374,10 @@ int zero_list_table_build(uint32_t T, uint32_t R, const uint64_t *numel,
  * streams, other host threads) race on it and must be ordered by the caller.
  * The step needs ZERO_WORKSPACE_BYTES of scratch whatever P and R are; a
  * build whose step needed more than the array holds would be refused with
- * ZERO_ERANGE.  All other arguments, limits and errors are those of
+ * ZERO_ERANGE.  check_nonfinite may be 0 or 1 (1 runs the overflow scan into
+ * the library's array itself); 2 is ZERO_EINVAL, because no
+ * zero_scan_nonfinite call can write the inf/NaN word of an array the caller
+ * has no address for.  All other arguments, limits and errors are those of
  * zero_step_fused. */
 int zero_step_fused_noalloc(const zero_step_args *args, void *stream);
 

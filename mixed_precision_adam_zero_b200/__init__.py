@@ -62,6 +62,20 @@ class ZeroError(RuntimeError):
         self.status = status
 
 
+class ZeroDeviceError(RuntimeError):
+    """A step's bounded device-side wait gave up (zero_ctrl.device_error is
+    set): that step was not applied, and the flag stays set until the
+    control block is reset with zero_ctrl_set."""
+
+
+def check_ctrl(c: "zero_ctrl", where: str) -> "zero_ctrl":
+    """Return c, or raise ZeroDeviceError if its device_error is set."""
+    if c.device_error:
+        raise ZeroDeviceError(f"{where}: device_error {c.device_error} after {c.step} applied steps "
+                              f"(a bounded wait in a step kernel gave up; that step was not applied)")
+    return c
+
+
 class zero_adam_hparams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_double), ("beta1", ctypes.c_double), ("beta2", ctypes.c_double),
                 ("eps", ctypes.c_double), ("weight_decay", ctypes.c_double)]
@@ -242,8 +256,9 @@ def zero_scan_nonfinite(grad, grad_dtype: int, n: int, workspace, stream=None) -
 
 
 def zero_selftest_wait_timeout(ctrl, stream=None) -> None:
-    """Run the device-side timeout path once: sets ctrl.device_error to 1
-    after about 2 s of GPU time (see the C declaration)."""
+    """Run the device-side timeout path once: after about 2 s of GPU time it
+    records a step that was not applied, with ctrl.device_error = 1 (see the
+    C declaration)."""
     _check(_lib().zero_selftest_wait_timeout(_ptr(ctrl), _stream(stream)), "zero_selftest_wait_timeout")
 
 

@@ -9,7 +9,7 @@ from typing import List, Optional, Sequence
 
 import torch
 
-from . import (ZERO_BF16, ZERO_F16, ZERO_F32, make_step_args, zero_ctrl_bytes, zero_ctrl_init,
+from . import (ZERO_BF16, ZERO_F16, ZERO_F32, check_ctrl, make_step_args, zero_ctrl_bytes, zero_ctrl_init,
                zero_ctrl_read, zero_gather_params, zero_gather_params_list, zero_list_table_build,
                zero_list_table_bytes, zero_step_fused, zero_step_fused_list, zero_workspace_bytes,
                zero_workspace_init)
@@ -47,8 +47,12 @@ class _Common:
     def two_set(self) -> bool:
         return len(self.master) == 2
 
-    def ctrl(self):
-        return zero_ctrl_read(self.ctrl_buf, self._s())
+    def ctrl(self, raw: bool = False):
+        """The control block, read after this optimizer's stream has finished.
+        Raises ZeroDeviceError if a step's device-side wait gave up, unless
+        `raw`."""
+        c = zero_ctrl_read(self.ctrl_buf, self._s())
+        return c if raw else check_ctrl(c, type(self).__name__)
 
     def current(self):
         """(master, exp_avg, exp_avg_sq) of the set holding the state."""

@@ -273,6 +273,11 @@ int check_common(const zero_step_args* a, StepParams* kp) {
         kp->push[i] = a->push_params16[i];
     }
     kp->npush = a->n_push;
+    // Push targets hold the other ranks' replicas of one owner's slice.  An
+    // all-owner call may take its skip decision in the same pass that stores
+    // the 16-bit values (two-set mode), and only the local replica is
+    // restored after a skip; so pushes need an owner.
+    if (a->n_push > 0 && a->owner < 0) return ZERO_EINVAL;
     const zero_adam_hparams& h = a->hp;
     kp->h.b1 = (float)h.beta1;
     kp->h.b2 = (float)h.beta2;
@@ -622,6 +627,9 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
 
 int zero_step_fused_noalloc(const zero_step_args* a, void* stream) {
     if (a == nullptr || a->workspace != nullptr) return ZERO_EINVAL;
+    // Mode 2 reads an inf/NaN word that zero_scan_nonfinite calls wrote into
+    // the caller's workspace; no scan can write into the library's array.
+    if (a->check_nonfinite == 2) return ZERO_EINVAL;
     if (ZERO_WORKSPACE_BYTES > ZERO_NOALLOC_SCRATCH_BYTES) return ZERO_ERANGE;
     void* ws = nullptr;
     int rc = noalloc_scratch(&ws);

@@ -789,13 +789,17 @@ __global__ void __launch_bounds__(kBulkThreads, 1) accum_bulk_kernel(const __gri
 // ------------------------------------------------------------ timeout health check
 
 // One thread waits on a barrier that nothing arrives at; the bounded wait
-// gives up and the kernel records the timeout as the staged kernels do.
+// gives up and the kernel records the outcome through the step epilogue's
+// control-block update, as a two-set step with the overflow check on whose
+// wait gave up: device_error set, the step not applied.
 __global__ void wait_timeout_probe_kernel(zero_ctrl* c) {
     __shared__ __align__(8) uint64_t bar;
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1u);
         fence_mbar_init();
-        if (!mbar_wait_bounded(&bar, 0u)) c->device_error = 1u;
+        // growth_interval 1: a step wrongly counted as applied would also
+        // double the loss scale, which the health check's caller can see.
+        if (!mbar_wait_bounded(&bar, 0u)) ctrl_after_step(c, false, true, true, 1, 1u);
     }
 }
 

@@ -445,6 +445,40 @@ __device__ __forceinline__ uint32_t find_tensor_by_tile(const Table& t, uint64_t
     return lo;
 }
 
+// The control block after one step call (one thread, once per call).
+//   found:   an inf/NaN was seen -> skipped: S halves, t and the set stay;
+//   timeout: a bounded wait of some CTA gave up, so part of the output was
+//            never written -> not applied either (t and parity stay, so a
+//            two-set optimizer keeps its last complete set and the restore
+//            kernel re-casts the 16-bit parameters from it), S and the
+//            growth count stay as they were, and device_error is set;
+//   else:    applied: t += 1, the set flips (two-set mode), and with the
+//            check on S doubles after growth_interval applied steps in a row.
+__device__ __forceinline__ void ctrl_after_step(zero_ctrl* c, bool found, bool timeout, bool two_set, int check,
+                                                uint32_t growth_interval) {
+    if (timeout) {
+        c->device_error = 1u;
+        c->last_skipped = 1u;
+    } else if (found) {
+        c->loss_scale *= 0.5f;
+        c->growth_tracker = 0u;
+        c->skipped += 1ull;
+        c->last_skipped = 1u;
+    } else {
+        c->step += 1ull;
+        c->last_skipped = 0u;
+        if (two_set) c->parity ^= 1u;
+        if (check) {
+            uint32_t gt = c->growth_tracker + 1u;
+            if (growth_interval != 0u && gt >= growth_interval) {
+                c->loss_scale *= 2.0f;
+                gt = 0u;
+            }
+            c->growth_tracker = gt;
+        }
+    }
+}
+
 // Grid-level epilogue: the last CTA to finish updates the control block and
 // clears the workspace for the next launch.  Every other access to the
 // control block and the workspace in this launch happened before the
@@ -462,26 +496,7 @@ __device__ __forceinline__ void finish_step(const StepParams& p, bool bad, bool 
         const unsigned long long all = atomicAdd(&ws->arrive, mine) + mine;
         if (Arrival::count(all) == gridDim.x) {
             const bool found = p.check == 1 ? Arrival::any_found(all) : (p.check == 2 && ws->found != 0u);
-            zero_ctrl* c = p.ctrl;
-            if (found) {
-                c->loss_scale *= 0.5f;
-                c->growth_tracker = 0u;
-                c->skipped += 1ull;
-                c->last_skipped = 1u;
-            } else {
-                c->step += 1ull;
-                c->last_skipped = 0u;
-                if (p.two_set) c->parity ^= 1u;
-                if (p.check) {
-                    uint32_t gt = c->growth_tracker + 1u;
-                    if (p.growth_interval != 0u && gt >= p.growth_interval) {
-                        c->loss_scale *= 2.0f;
-                        gt = 0u;
-                    }
-                    c->growth_tracker = gt;
-                }
-            }
-            if (Arrival::any_timeout(all)) c->device_error = 1u;
+            ctrl_after_step(p.ctrl, found, Arrival::any_timeout(all), p.two_set != 0, p.check, p.growth_interval);
             ws->found = 0u;
             ws->next_tile = 0u;
             ws->arrive = 0ull;

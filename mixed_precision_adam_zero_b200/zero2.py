@@ -37,7 +37,7 @@ import torch
 import torch.distributed as dist
 from torch.multiprocessing.reductions import reduce_tensor
 
-from . import (ZERO_F32, ZERO_WORKSPACE_FOUND_OFFSET, make_accum_args, make_step_args, zero_accumulate_grads,
+from . import (ZERO_F32, ZERO_WORKSPACE_FOUND_OFFSET, check_ctrl, make_accum_args, make_step_args, zero_accumulate_grads,
                zero_checkpoint_load, zero_checkpoint_save, zero_ctrl_bytes, zero_ctrl_init, zero_ctrl_read,
                zero_gather_params, zero_partition_bounds, zero_scan_nonfinite, zero_step_fused,
                zero_workspace_bytes, zero_workspace_init)
@@ -230,8 +230,11 @@ class Zero2Rank:
         zero_step_fused(args, self._s())
         self._barrier()
 
-    def ctrl(self):
-        return zero_ctrl_read(self.ctrl_buf, self._s())
+    def ctrl(self, raw: bool = False):
+        """This rank's control block; raises ZeroDeviceError if a step's
+        device-side wait gave up, unless `raw`."""
+        c = zero_ctrl_read(self.ctrl_buf, self._s())
+        return c if raw else check_ctrl(c, f"Zero2Rank {self.r}")
 
     def owned(self):
         """(master, exp_avg, exp_avg_sq) of the owned slice [lo, hi)."""

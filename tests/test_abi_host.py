@@ -129,6 +129,7 @@ def _args(**over):
     (dict(push_params16=[A] * 73), za.ZERO_ERANGE),
     (dict(push_params16=[A, A + 2]), za.ZERO_EALIGN),
     (dict(push_params16=[A, None]), za.ZERO_EINVAL),
+    (dict(push_params16=[A]), za.ZERO_EINVAL),               # pushes need an owner
     (dict(n_grads=300), za.ZERO_ERANGE),
     (dict(n_grads=2, rank_weights=[1, -1]), za.ZERO_EINVAL),      # weights over the n_grads buffers
     (dict(grad_offset=4, owner=1), za.ZERO_EALIGN),
@@ -222,6 +223,23 @@ def test_noalloc_step_refuses_a_caller_workspace():
     with pytest.raises(za.ZeroError) as e:
         za.zero_step_fused_noalloc(a)
     assert e.value.status == za.ZERO_EINVAL
+
+
+def test_noalloc_step_refuses_mode_2():
+    # mode 2 reads an inf/NaN word that only zero_scan_nonfinite writes, and
+    # no scan can write into the library's array
+    a = _args(workspace=None, check_nonfinite=2)
+    with pytest.raises(za.ZeroError) as e:
+        za.zero_step_fused_noalloc(a)
+    assert e.value.status == za.ZERO_EINVAL
+
+
+def test_pushes_need_an_owner():
+    for check in (0, 1):
+        a = _args(push_params16=[A], owner=-1, check_nonfinite=check)
+        with pytest.raises(za.ZeroError) as e:
+            za.zero_step_fused(a)
+        assert e.value.status == za.ZERO_EINVAL
 
 
 @pytest.mark.parametrize("kw,status", [

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import synth
-from gpu_helpers import ADAMW_HP, assert_close, assert_params16, compare_full, host_grad, ohp
+from gpu_helpers import ADAMW_HP, assert_close, assert_params16, compare_full, host_grad, ohp, report_near_zero
 from mixed_precision_adam_zero_b200 import zero_partition_bounds
 from mixed_precision_adam_zero_b200.buffers import FlatZero, ListZero
 
@@ -72,7 +72,9 @@ def _sampled_run(z, flat_grad_bufs, flat_params16, steps, workload, gdt, extra=(
     assert_close(w.index_select(0, idx_dev), st.w, "master")
     assert_close(m.index_select(0, idx_dev), st.m, "exp_avg")
     assert_close(v.index_select(0, idx_dev), st.v, "exp_avg_sq")
-    assert_params16(flat_params16.index_select(0, idx_dev), w.index_select(0, idx_dev), st.w, z.param_dtype)
+    stats = assert_params16(flat_params16.index_select(0, idx_dev), w.index_select(0, idx_dev), st.w,
+                            z.param_dtype)
+    report_near_zero(stats, f"workload {workload} ({P} parameters, sampled)")
     _cast_check_full(flat_params16, w)
     c = z.ctrl()
     assert c.step == st.ctrl.t and c.skipped == st.ctrl.skipped and c.loss_scale == st.ctrl.loss_scale
@@ -103,7 +105,7 @@ def test_flat16m_full_oracle():
         z.step(hp=ADAMW_HP)
         oracle.step(st, [host_grad(g) for g in z.grads], "bf16", ohp(ADAMW_HP))
     torch.cuda.synchronize()
-    compare_full(z, st, z.params16)
+    report_near_zero(compare_full(z, st, z.params16), "flat16m (every element)")
 
 
 def test_gpt2m_list_fp16_loss_scale_skips():
@@ -190,4 +192,4 @@ def test_flat16m_four_micro_batches_per_update_full_oracle():
         z.step(hp=ADAMW_HP, grads=[acc])
         oracle.step(st, [host_grad(acc)], "f32", ohp(ADAMW_HP))
     torch.cuda.synchronize()
-    compare_full(z, st, z.params16)
+    report_near_zero(compare_full(z, st, z.params16), "flat16m, 4 micro-batches per update (every element)")

@@ -110,6 +110,53 @@ def test_emulated_ranks_dtypes_and_token_weights(gdt, pdt, R):
     _run(P=100_019, R=R, gdt=gdt, pdt=pdt, token=True)
 
 
+def test_push_targets_untouched_when_an_inf_skips_the_step():
+    """Owner calls with push targets and the overflow check in mode 1: each
+    call scans every rank's gradient before its step kernel runs, so a planted
+    inf skips the step before any 16-bit value reaches a peer's replica.  The
+    next step applies on every rank, bitwise like the single call.  An
+    all-owner call with push targets is refused."""
+    P, R, S0, seed = 60_013, 4, 1024.0, 91
+    pcode = DTYPES["f16"][0]
+    ref = FlatZero(P, R, "f16", "f16", loss_scale=S0)
+    w0 = synth.normal(P, 0.02, seed, device="cuda")
+    ref.load_master(w0)
+    ranks = _ranks(P, R, "f16", "f16", w0, S0)
+
+    def owner_calls():
+        for r, k in enumerate(ranks):
+            za.zero_step_fused(za.make_step_args(
+                P, R, grad_dtype=pcode, param_dtype=pcode, master=k.master, exp_avg=k.exp_avg,
+                exp_avg_sq=k.exp_avg_sq, ctrl=k.ctrl, workspace=k.ws, grads=ref.grads, params16=k.params16,
+                owner=r, hp=ADAMW_HP, check_nonfinite=1, state_offset=k.off,
+                push_params16=[o.params16 for j, o in enumerate(ranks) if j != r]))
+
+    grads_for_step(seed, 1, ref.grads, 1e-3, scale=S0)
+    ref.grads[2][P // 3] = float("inf")
+    before = [(k.params16.clone(), k.master.clone(), k.exp_avg.clone()) for k in ranks]
+    owner_calls()
+    ref.step(hp=ADAMW_HP, check=True)
+    torch.cuda.synchronize()
+    for r, (k, (p16, w, m)) in enumerate(zip(ranks, before)):
+        assert torch.equal(k.params16.view(torch.int16), p16.view(torch.int16)), f"replica of rank {r} written"
+        assert torch.equal(k.master.view(torch.int32), w.view(torch.int32)), f"master of rank {r} written"
+        assert torch.equal(k.exp_avg.view(torch.int32), m.view(torch.int32)), f"exp_avg of rank {r} written"
+        c = za.zero_ctrl_read(k.ctrl)
+        assert (c.step, c.skipped, c.last_skipped, c.loss_scale) == (0, 1, 1, S0 / 2)
+    grads_for_step(seed, 2, ref.grads, 1e-3, scale=S0 / 2)
+    owner_calls()
+    ref.step(hp=ADAMW_HP, check=True)
+    torch.cuda.synchronize()
+    _compare(ranks, ref)
+    k = ranks[0]
+    with pytest.raises(za.ZeroError) as e:
+        za.zero_step_fused(za.make_step_args(
+            P, R, grad_dtype=pcode, param_dtype=pcode, master=ref.master[0], exp_avg=ref.exp_avg[0],
+            exp_avg_sq=ref.exp_avg_sq[0], ctrl=ref.ctrl_buf, workspace=ref.workspace, grads=ref.grads,
+            params16=ref.params16, owner=-1, hp=ADAMW_HP, check_nonfinite=1, push_params16=[k.params16]))
+    assert e.value.status == za.ZERO_EINVAL
+
+
 def test_emulated_ranks_share_the_skip_decision():
     # fp16 gradients x 2^16; one rank's inf at step 2 skips the step on every
     # rank (scale halved everywhere), and the next steps apply again.

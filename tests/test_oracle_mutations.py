@@ -38,6 +38,15 @@ MUTANTS = [
     ("f16 subnormal off by one", "mag = ldexp((double)f, -24);", "mag = ldexp((double)f, -25);"),
     ("accumulation ignores first", "double prev = first ? 0.0 : (double)acc[k];", "double prev = (double)acc[k];"),
     ("accumulation drops the scale", "acc[k] = (float)(prev + scale * g);", "acc[k] = (float)(prev + g);"),
+    ("growth one step early", "c->growth_tracker == c->growth_interval)",
+     "c->growth_tracker + 1 == c->growth_interval)"),
+    ("growth count kept across a skip", "    c->loss_scale *= 0.5;\n    c->growth_tracker = 0;",
+     "    c->loss_scale *= 0.5;"),
+    ("growth with the check off", "    if (check) {\n        c->growth_tracker += 1;",
+     "    if (1) {\n        c->growth_tracker += 1;"),
+    ("growth count not restarted after growth", "c->loss_scale *= 2.0;\n            c->growth_tracker = 0;",
+     "c->loss_scale *= 2.0;"),
+    ("growth triples the scale", "c->loss_scale *= 2.0;", "c->loss_scale *= 3.0;"),
     ("overflow check misses NaN", "if (!isfinite(zo_load(gdtype, grads[r], k))) found |= 1;",
      "if (isinf(zo_load(gdtype, grads[r], k))) found |= 1;"),
 ]

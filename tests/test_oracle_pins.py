@@ -307,6 +307,44 @@ def test_nonfinite_gradient_skips_and_halves_the_scale(bad):
     assert st.ctrl.t == 2 and st.ctrl.last_skipped == 0
 
 
+def test_loss_scale_schedule_hand_derived():
+    """The growth and halving of S, the step count and the growth count,
+    call by call, against schedules derived by hand from the stated rule
+    (tests/golden/loss_scale_schedule.txt)."""
+    rng = np.random.default_rng(6)
+    P, R = 40, 2
+    hp = oracle.HP(lr=1e-3, beta1=0.8, beta2=0.999, eps=1e-8, weight_decay=3e-7)
+    schedules = {}
+    for row in golden_rows("loss_scale_schedule.txt"):
+        f = row.split()
+        schedules.setdefault(f[0], []).append([int(x) for x in f[1:]])
+    assert sorted(schedules) == ["A", "B", "C"]
+    for name, rows in schedules.items():
+        check, interval = rows[0][0], rows[0][1]
+        st = oracle.State.create(rng.normal(0, 0.02, P), loss_scale=65536.0, growth_interval=interval)
+        for check_r, interval_r, call, inf, skipped, S, t, growth in rows:
+            assert (check_r, interval_r) == (check, interval)
+            g = rng.normal(0, 1e-3, (R, P))
+            grads = [(g[r] * st.ctrl.loss_scale).astype(np.float32) for r in range(R)]
+            if inf:
+                grads[1][P // 2] = np.inf
+            before = st.copy()
+            got = oracle.step(st, grads, "f32", hp, check=bool(check))
+            where = f"schedule {name}, call {call}"
+            assert got == bool(skipped), where
+            assert (st.ctrl.loss_scale, st.ctrl.t, st.ctrl.growth_tracker) == (S, t, growth), where
+            assert st.ctrl.last_skipped == skipped, where
+            if skipped:
+                assert np.array_equal(st.w, before.w) and np.array_equal(st.v, before.v), where
+            else:
+                # the step divides by the scale the gradients were stored with
+                ref = before.copy()
+                ref.ctrl.loss_scale = 1.0
+                unscaled = [(grads[r].astype(np.float64) / before.ctrl.loss_scale) for r in range(R)]
+                oracle.step(ref, unscaled, "f64", hp)
+                assert np.array_equal(st.w, ref.w) and np.array_equal(st.m, ref.m), where
+
+
 def test_unscale_is_exact_division_by_the_scale():
     # Gradients stored times S = 2^k reduce to exactly the unscaled mean.
     vals = np.array([0.5, -0.25, 3.0], dtype=np.float32)
