@@ -15,9 +15,11 @@ Sources: the DeepSpeed "ZeRO" documentation page (zero3.rst); the Q&A page
 "How does DeepSpeed ZeRO stage 1, 2, and 3 partition optimizer states,
 gradients, and parameters?"; the "Deep dive: DeepSpeed" lesson.
 
-Parity unpinned: the growth of the loss scale after ``growth_interval``
-consecutive applied steps (the pages describe no loss scaling at all; only the
-halving on overflow is fixed, by the workload description of the fp16 case).
+Loss scaling: the pages describe none.  The halving on overflow is fixed by
+the workload description of the fp16 case; the growth after
+``growth_interval`` consecutive applied steps follows the stated reading and
+is pinned by a schedule derived by hand from it
+(tests/golden/loss_scale_schedule.txt), not by a value the pages print.
 """
 from __future__ import annotations
 

@@ -29,7 +29,9 @@
  *   - The overflow check covers every raw gradient of every rank; a skipped
  *     step changes no weight or moment, leaves t unchanged and halves S.
  *   - Growth of S (x2 after `growth_interval` consecutive applied steps when
- *     checking is on) is not described by the pages: parity unpinned.
+ *     checking is on) is not described by the pages; it follows the stated
+ *     loss-scaling reading and is pinned by a schedule derived by hand from
+ *     that reading (tests/golden/loss_scale_schedule.txt), not by the pages.
  *   - 16-bit parameters are the round-to-nearest-even of the float64 master,
  *     rounded once, directly to the 16-bit format.
  */
