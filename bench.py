@@ -5,13 +5,24 @@
 One step = one pass of the whole hot path (in-HBM reduce-scatter of the R
 rank gradients, Adam/AdamW on the fp32 masters and moments, round-to-nearest
 cast into the replicated 16-bit parameters) over one batch of synthetic
-gradients.  The default workload is the flat 16,777,259-parameter vector with
-R = 8 bf16 rank gradients (uneven owner slices), AdamW.  Prints one JSON line.
+gradients.  Prints one JSON line.
 
-Several GPUs (torchrun, one process per GPU) run independent replicas of the
-workload: the step has no exchange between GPUs in this configuration, so
-scaling is weak and no collective is on the data path; the only collectives
-are the barrier and the max-over-ranks reduction of the timings.
+Default on one GPU: the Llama-style 3.2B tensor list (254 tensors,
+3,212,749,824 parameters) with R = 8 bf16 rank gradients held in HBM, AdamW
+-- the largest workload that fits one GPU (about 96 GB resident).
+
+Several GPUs (torchrun, one process per GPU): by default the ZeRO-2 step
+across GPUs (`--workload zero2`): R = the number of GPUs, each process owns
+the slice floor(P r/R) .. floor(P (r+1)/R) of a flat 3.2B-parameter vector
+and its fp32 state, pulls the other ranks' gradients over its slice from
+their memory (the reduce-scatter as loads), and stores its 16-bit results
+into every rank's replica (the all-gather as stores), between two barriers.
+Any other workload under torchrun runs one independent replica per GPU
+(no collective on its data path).  Timings are CUDA events on the launching
+stream, the maximum over ranks.
+
+`--impl reference` times the float64 CPU oracle (the repository's checker)
+on a bounded sample of the same workload, on rank 0 only.
 """
 from __future__ import annotations
 
@@ -31,6 +42,18 @@ if ROOT not in sys.path:
 METRIC = "fused ZeRO step: params updated/sec and HBM GB/s (% of B200 peak), 1 GPU"
 UNIT = "params/s"
 ADAMW = (1e-3, 0.8, 0.999, 1e-8, 3e-7)
+OPTIMIZER = "AdamW lr=1e-3 betas=(0.8,0.999) eps=1e-8 wd=3e-7"
+L2_BYTES = 126 * 1000 * 1000
+DEFAULT_WORKLOAD = "llama3b"
+DEFAULT_WORKLOAD_MULTI = "zero2"
+# Parameters of the workload that the oracle steps over in the CPU baseline
+# and in the reference arm (the same sample in both).
+ORACLE_SAMPLE_P = 1 << 22
+# End-to-end: about this many bytes of host gradients per run by default.
+E2E_BUDGET_BYTES = 16 << 30
+# Peer copy bandwidth per direction measured on this machine's NVLink 5 (GB/s).
+NVLINK_GBS = 770.0
+LLAMA3B_P = 3_212_749_824
 
 # name -> (kind, P or tensor-list builder, R, grad dtype, param dtype, fp16 loss scaling)
 WORKLOADS = {
@@ -41,16 +64,21 @@ WORKLOADS = {
     "llama3b": ("list", "llama3b", 8, "bf16", "bf16", False),
     # the fp16 case with one state set: overflow scan first, then the step
     "gpt2m_inplace": ("list", "gpt2m", 4, "f16", "f16", True),
-    # GPT-2-medium's embeddings and first layer only (14 tensors, 65M
-    # parameters, about 2 GB on the device): a small case of the list kernel
+    # Small cases of the same kernel instances, a few GB on the device, for
+    # ncu captures: GPT-2-medium's embeddings and first layer (14 tensors,
+    # 65M parameters), one Llama decoder layer (9 tensors, 100.7M), and flat
+    # R = 4 vectors of 64M parameters with bf16 and fp32 gradients.
     "gpt2m_head": ("list", "gpt2m_head", 4, "f16", "f16", True),
+    "llama3b_layer": ("list", "llama3b_layer", 8, "bf16", "bf16", False),
+    "flat64m_r4": ("flat", 1 << 26, 4, "bf16", "bf16", False),
+    "flat64m_r4_f32": ("flat", 1 << 26, 4, "f32", "bf16", False),
     # bandwidth sweep of the flat kernel, R = 8 bf16
     "sweep1m": ("flat", 1 << 20, 8, "bf16", "bf16", False),
     "sweep4m": ("flat", 1 << 22, 8, "bf16", "bf16", False),
     "sweep64m": ("flat", 1 << 26, 8, "bf16", "bf16", False),
     "sweep256m": ("flat", 1 << 28, 8, "bf16", "bf16", False),
     "sweep1b": ("flat", 1 << 30, 8, "bf16", "bf16", False),
-    "sweep3p2b": ("flat", 3_212_749_824, 8, "bf16", "bf16", False),
+    "sweep3p2b": ("flat", LLAMA3B_P, 8, "bf16", "bf16", False),
 }
 GRAD_BYTES = {"bf16": 2, "f16": 2, "f32": 4}
 
@@ -66,6 +94,8 @@ WORKLOADS["gpt2m_z3gather"] = ("z3gather", "gpt2m", 4, "bf16", "bf16", False)
 # its own state slice, reading every rank's gradient slice and storing its
 # 16-bit results into all R replicas (the pushes land in this GPU's HBM).
 WORKLOADS["flat16m_zero2emu"] = ("zero2emu", 16_777_259, 8, "bf16", "bf16", False)
+# The ZeRO-2 step across GPUs, one process per GPU (R = 0: the world size).
+WORKLOADS["zero2"] = ("zero2", LLAMA3B_P, 0, "bf16", "bf16", False)
 
 
 def bytes_per_param(R: int, gdt: str, gas: int = 0) -> int:
@@ -84,6 +114,77 @@ def zero2emu_bytes_per_param(R: int, gdt: str) -> int:
     owner, state read and written, and each 16-bit result stored into R
     replicas."""
     return GRAD_BYTES[gdt] * R + 24 + 2 * R
+
+
+def nvlink_bytes_per_direction(P: int, R: int, gdt: str = "bf16") -> int:
+    """One rank of the ZeRO-2 step across R GPUs: the other ranks' gradients
+    over its slice come in, and its 16-bit results go out to the other
+    replicas, (R - 1)/R * P elements each way (2 bytes each for bf16)."""
+    return (R - 1) * P * GRAD_BYTES[gdt] // R
+
+
+def tensor_list(name: str):
+    import synth
+    if name == "gpt2m":
+        return synth.gpt2_medium_tensors()
+    if name == "gpt2m_head":
+        return synth.gpt2_medium_tensors()[:14]
+    if name == "llama3b":
+        return synth.llama_3b_tensors()
+    if name == "llama3b_layer":
+        return synth.llama_3b_tensors()[1:10]
+    raise KeyError(name)
+
+
+def workload_P(name: str, world: int = 1) -> int:
+    """Parameters one step updates (the padded elements for the ZeRO-3 gather)."""
+    kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
+    if kind == "list":
+        return sum(n for _, n in tensor_list(size))
+    if kind == "z3gather":
+        return sum(R * -(-n // R) for _, n in tensor_list(size))
+    return size
+
+
+def workload_R(name: str, world: int = 1) -> int:
+    R = WORKLOADS[name][2]
+    return R if R else world
+
+
+def workload_bpp(name: str, world: int = 1) -> int:
+    """Algorithmic HBM bytes per parameter of one step (on each GPU's share
+    for the ZeRO-2 step across GPUs: its slice's state, its own gradient read
+    by every owner and every owner's pushes into its replica)."""
+    kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
+    R = workload_R(name, world)
+    if kind == "z3gather":
+        return 4
+    if kind == "zero2emu":
+        return zero2emu_bytes_per_param(R, gdt)
+    if kind == "zero2":
+        # per parameter of the whole vector, summed over the R GPUs
+        return GRAD_BYTES[gdt] * R + 24 + 2 * R
+    return bytes_per_param(R, gdt, GAS.get(name, 0))
+
+
+def workload_config(name: str, world: int = 1) -> dict:
+    """The workload as both arms name it: static, no measured values."""
+    kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
+    P, R, bpp = workload_P(name, world), workload_R(name, world), workload_bpp(name, world)
+    touched = bpp * P // (world if kind == "zero2" else 1)
+    if touched > 3 * L2_BYTES:
+        l2 = f"inputs larger than L2 ({touched / 1e6:.0f} MB touched per step per GPU vs 126 MB L2), no flush"
+    else:
+        l2 = f"working set {touched / 1e6:.0f} MB per step, within 3x the 126 MB L2: partly L2-resident, no flush"
+    if kind == "zero2":
+        par = f"zero2 across {world} GPU(s): owner slices, peer gradient loads, parameter pushes"
+    else:
+        par = f"replicas x{world}" if world > 1 else "single GPU"
+    cfg = {"workload": name, "P": P, "R": R, "grad_dtype": gdt, "param_dtype": pdt, "optimizer": OPTIMIZER,
+           "loss_scale_check": bool(scaled), "bytes_per_param": bpp, "l2": l2, "parallelism": par}
+    if kind == "list":
+        cfg["tensors"] = len(tensor_list(size))
+    return cfg
 
 
 def kernel_source_sha() -> str:
@@ -116,6 +217,14 @@ def traffic_for(workload: str):
     if not e or e.get("kernel_source_sha") != kernel_source_sha():
         return None
     return e.get("dram_bytes_per_launch")
+
+
+def e2e_step_count(K: int, h2d_bytes: int, requested=None) -> int:
+    """Timed end-to-end steps: as requested, else enough for about
+    E2E_BUDGET_BYTES of host gradients, at least 2, at most K."""
+    if requested is not None:
+        return max(0, min(K, requested))
+    return min(K, max(2, E2E_BUDGET_BYTES // max(h2d_bytes, 1)))
 
 
 # ------------------------------------------------------------ clocks
@@ -174,41 +283,46 @@ class ClockSampler:
 
 # ------------------------------------------------------------ workload
 
-def build_workload(name: str, device):
+class Bench:
+    """A built workload: its step call, the device buffers a user would fill
+    from the host (gradients) and read back (16-bit parameters), the launches
+    per step and the control block."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def build_workload(name: str, device, stream, world: int = 1) -> Bench:
     import torch
     import synth
-    from mixed_precision_adam_zero_b200.buffers import FlatZero, ListZero
+    from mixed_precision_adam_zero_b200 import (ZERO_BF16, ZERO_F16, ZERO_F32, make_accum_args,
+                                                make_step_args, zero_accumulate_grads, zero_ctrl_init,
+                                                zero_ctrl_read, zero_step_fused, zero_step_fused_list)
+    from mixed_precision_adam_zero_b200.buffers import DTYPES, FlatZero, ListZero
     kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
     wl = synth.WORKLOADS.get(name.split("_")[0], 9)
     S = 65536.0 if scaled else 1.0
     two_set = scaled and not name.endswith("_inplace")
+    gcode, gt = DTYPES[gdt]
+    pcode, pt = DTYPES[pdt]
+
     if kind == "z3gather":
-        from mixed_precision_adam_zero_b200 import ZERO_BF16, zero3_gather_list_build, zero_list_table_bytes
-        numels = [n for _, n in synth.gpt2_medium_tensors()]
+        from mixed_precision_adam_zero_b200 import zero3_gather, zero3_gather_list_build, zero_list_table_bytes
+        numels = [n for _, n in tensor_list(size)]
         shard = [-(-n // R) for n in numels]
-        sbufs = [torch.empty(sum(shard), dtype=torch.bfloat16, device=device) for _ in range(R)]
+        sbufs = [torch.empty(sum(shard), dtype=pt, device=device) for _ in range(R)]
         for r, sb in enumerate(sbufs):
             synth.fill_normal_(sb, 0.02, synth.seed_for(wl, synth.KIND_MASTER, r))
-        fbuf = torch.empty(R * sum(shard), dtype=torch.bfloat16, device=device)
+        fbuf = torch.empty(R * sum(shard), dtype=pt, device=device)
         full = list(fbuf.split([R * s for s in shard]))
         nb = zero_list_table_bytes(len(numels), R)
         table = torch.zeros(nb, dtype=torch.uint8, device=device)
         gl = zero3_gather_list_build(numels, full, [list(sb.split(shard)) for sb in sbufs], ZERO_BF16, table, nb)
+        return Bench(P=R * sum(shard), call=lambda: zero3_gather(gl, stream), inputs=sbufs, output=fbuf,
+                     launches=1, ctrl=lambda: None, keep=(table, full))
 
-        class Z3:
-            pass
-        z = Z3()
-        z.P, z.gl, z.table, z.keep = R * sum(shard), gl, table, (sbufs, fbuf)
-        z.check, z.gbufs = False, sbufs
-        z.flat_p16 = fbuf
-        z.ctrl = lambda: type("C", (), {"step": 0})()
-        return z
     if kind == "zero2emu":
-        from mixed_precision_adam_zero_b200 import make_step_args, zero_ctrl_init, zero_ctrl_read
-        from mixed_precision_adam_zero_b200.buffers import DTYPES
         from mixed_precision_adam_zero_b200.zero2 import rank_slice
-        gcode, gt = DTYPES[gdt]
-        pcode, pt = DTYPES[pdt]
         w0 = synth.normal(size, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device)
         gbufs = [torch.empty(size, dtype=gt, device=device) for _ in range(R)]
         for r, g in enumerate(gbufs):
@@ -223,51 +337,67 @@ def build_workload(name: str, device):
             zero_ctrl_init(ctrl, 1.0)
             ws = torch.zeros(256, dtype=torch.uint8, device=device)
             ranks.append((st, ctrl, ws, off))
+        owner_args = [make_step_args(size, R, grad_dtype=gcode, param_dtype=pcode, master=st[0], exp_avg=st[1],
+                                     exp_avg_sq=st[2], ctrl=ctrl, workspace=ws, grads=gbufs,
+                                     params16=replicas[r], owner=r, hp=ADAMW, state_offset=off,
+                                     push_params16=[t for j, t in enumerate(replicas) if j != r])
+                      for r, (st, ctrl, ws, off) in enumerate(ranks)]
 
-        class Emu:
-            pass
-        z = Emu()
-        z.P, z.gbufs, z.check, z.flat_p16 = size, gbufs, False, replicas[0]
-        z.keep = (ranks, replicas)
-        z.owner_args = [make_step_args(size, R, grad_dtype=gcode, param_dtype=pcode, master=st[0], exp_avg=st[1],
-                                       exp_avg_sq=st[2], ctrl=ctrl, workspace=ws, grads=gbufs,
-                                       params16=replicas[r], owner=r, hp=ADAMW, state_offset=off,
-                                       push_params16=[t for j, t in enumerate(replicas) if j != r])
-                        for r, (st, ctrl, ws, off) in enumerate(ranks)]
-        z.ctrl = lambda: zero_ctrl_read(ranks[0][1])
-        return z
+        def call():
+            for a in owner_args:
+                zero_step_fused(a, stream)
+        return Bench(P=size, call=call, inputs=gbufs, output=replicas[0], launches=R,
+                     ctrl=lambda: zero_ctrl_read(ranks[0][1]), keep=(ranks, replicas, owner_args))
+
+    if kind == "zero2":
+        from mixed_precision_adam_zero_b200.zero2 import Zero2Rank
+        z2 = Zero2Rank(size, gdt, pdt, device=device)
+        z2.load_master(synth.normal(size, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device))
+        synth.fill_normal_(z2.grad, 1e-3, synth.seed_for(wl, synth.KIND_GRAD, z2.r, 1))
+        torch.cuda.synchronize(device)
+        return Bench(P=size, call=lambda: z2.step(ADAMW), inputs=[z2.grad], output=z2.params16, launches=1,
+                     ctrl=lambda: z2.ctrl(), keep=(z2,), zero2=z2)
+
     if name in GAS:
-        z = FlatZero(size, 1, "f32", pdt, device=device, loss_scale=S, alloc_grads=False)
-        gt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt]
-        z.micro = [torch.empty(size, dtype=gt, device=device) for _ in range(R)]
-        z.accum = torch.zeros(size, dtype=torch.float32, device=device)
+        z = FlatZero(size, 1, "f32", pdt, device=device, loss_scale=S, alloc_grads=False, stream=stream)
+        micro = [torch.empty(size, dtype=gt, device=device) for _ in range(R)]
+        accum = torch.zeros(size, dtype=torch.float32, device=device)
         z.load_master(synth.normal(z.P, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device))
-        for r, g in enumerate(z.micro):
+        for r, g in enumerate(micro):
             synth.fill_normal_(g, 1e-3, synth.seed_for(wl, synth.KIND_GRAD, r, 1), scale=S)
-        z.gbufs = z.micro
-        z.check = scaled
-        z.gas = GAS[name]
-        z.micro_R, z.micro_gdt = R, gdt
-        return z
+        gas = GAS[name]
+        step_args = z.step_args(hp=ADAMW, check=scaled, grads=[accum])
+        micro_args = [make_accum_args(z.P, R, grad_dtype=gcode, grads=micro, accum=accum, scale=1.0 / gas,
+                                      first=(mu == 0), workspace=z.workspace, ctrl=z.ctrl_buf)
+                      for mu in range(gas)]
+
+        def call():
+            for a in micro_args:
+                zero_accumulate_grads(a, stream=stream)
+            zero_step_fused(step_args, stream)
+        return Bench(P=size, call=call, inputs=micro, output=z.params16, launches=gas + 1, ctrl=z.ctrl,
+                     keep=(z, accum, step_args, micro_args))
+
     if kind == "flat":
-        z = FlatZero(size, R, gdt, pdt, device=device, loss_scale=S, two_set=two_set)
-        gbufs = z.grads
+        z = FlatZero(size, R, gdt, pdt, device=device, loss_scale=S, two_set=two_set, stream=stream)
+        gbufs, p16 = z.grads, z.params16
+        step_args = z.step_args(hp=ADAMW, check=scaled)
+        call = lambda: zero_step_fused(step_args, stream)
     else:
-        tensors = {"gpt2m": synth.gpt2_medium_tensors, "gpt2m_head": lambda: synth.gpt2_medium_tensors()[:14],
-                   "llama3b": synth.llama_3b_tensors}[size]()
-        numels = [n for _, n in tensors]
-        gt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}
-        gbufs = [torch.empty(sum(numels), dtype=gt[gdt], device=device) for _ in range(R)]
-        pbuf = torch.empty(sum(numels), dtype=gt[pdt], device=device)
-        z = ListZero(numels, R, gdt, pdt, device=device, loss_scale=S, two_set=two_set,
-                     params16=list(pbuf.split(numels)), grads=[list(g.split(numels)) for g in gbufs])
-        z.flat_p16 = pbuf
+        # each rank's gradients in one contiguous buffer, the tensors views into it
+        numels = [n for _, n in tensor_list(size)]
+        gbufs = [torch.empty(sum(numels), dtype=gt, device=device) for _ in range(R)]
+        p16 = torch.empty(sum(numels), dtype=pt, device=device)
+        z = ListZero(numels, R, gdt, pdt, device=device, loss_scale=S, two_set=two_set, stream=stream,
+                     params16=list(p16.split(numels)), grads=[list(g.split(numels)) for g in gbufs])
+        step_args = z.step_args(hp=ADAMW, check=scaled)
+        call = lambda: zero_step_fused_list(step_args, z.list, stream)
     z.load_master(synth.normal(z.P, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device))
     for r, g in enumerate(gbufs):
         synth.fill_normal_(g, 1e-3, synth.seed_for(wl, synth.KIND_GRAD, r, 1), scale=S)
-    z.gbufs = gbufs
-    z.check = scaled
-    return z
+    # two-set: the pass + a restore kernel (no-op unless skipped); one set: a scan + the pass
+    return Bench(P=z.P, call=call, inputs=gbufs, output=p16, launches=2 if scaled else 1, ctrl=z.ctrl,
+                 keep=(z, step_args))
 
 
 def roofline_kernel(workload: str) -> str:
@@ -278,6 +408,8 @@ def roofline_kernel(workload: str) -> str:
         return "z3_gather_kernel"
     if kind == "zero2emu":
         return f"{R} x step_bulk_kernel (flat, push): the owners of an emulated {R}-rank ZeRO-2 step"
+    if kind == "zero2":
+        return "step_bulk_kernel (flat, push): this GPU's owner kernel of the ZeRO-2 step across GPUs"
     step = ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") + (" (flat)" if kind == "flat" else " (list)")
     gas = GAS.get(workload, 0)
     if gas:
@@ -286,16 +418,30 @@ def roofline_kernel(workload: str) -> str:
     return step
 
 
-def launches_per_step(z) -> int:
-    if hasattr(z, "gl"):
-        return 1
-    if hasattr(z, "owner_args"):
-        return len(z.owner_args)
-    if getattr(z, "gas", 0):
-        return z.gas + 1
-    if not z.check:
-        return 1
-    return 2  # two-set: the pass + a restore kernel (no-op unless skipped); one set: a scan + the pass
+def roofline(workload: str, world: int, P: int, launch_ms: float, peaks: dict, traffic) -> dict:
+    """Roofline of the dominant kernel.  HBM-bound: algorithmic bytes per
+    launch over its mean duration against the measured copy peak.  The ZeRO-2
+    step across GPUs (R > 1): the bytes one GPU sends over NVLink per step,
+    against the machine's measured peer bandwidth per direction."""
+    kind = WORKLOADS[workload][0]
+    R = workload_R(workload, world)
+    if kind == "zero2" and R > 1:
+        b = nvlink_bytes_per_direction(P, R)
+        achieved = b / (launch_ms * 1e-3) / 1e9
+        return {"bound": "nvlink", "achieved": achieved, "peak": NVLINK_GBS, "unit": "GB/s",
+                "frac": achieved / NVLINK_GBS, "peak_source": "pool's measured peer copy per direction",
+                "traffic": None, "kernel": roofline_kernel(workload), "bytes_per_launch": b,
+                "launch_ms": launch_ms}
+    bpp = workload_bpp(workload, world) if kind != "zero2" else bytes_per_param(1, "bf16")
+    peak = peaks.get("hbm_gbs")
+    src = "measured" if peak else "fallback"
+    peak = peak or 6650.0
+    achieved = bpp * P / (launch_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "peak_source": f"{src} hbm_gbs", "traffic": traffic,
+            # the ncu-measured DRAM bytes of one launch over the live launch time
+            "traffic_gbs": traffic / (launch_ms * 1e-3) / 1e9 if traffic else None,
+            "kernel": roofline_kernel(workload), "bytes_per_launch": bpp * P, "launch_ms": launch_ms}
 
 
 # ------------------------------------------------------------ ranks
@@ -316,11 +462,26 @@ def max_over_ranks(values, world: int, device):
     return t.tolist()
 
 
+def agree_on(values, world: int, device) -> None:
+    """Every rank runs the same workload: the ranks' values (numbers) must be
+    equal, else every rank raises before any step."""
+    lo = max_over_ranks([-float(v) for v in values], world, device)
+    hi = max_over_ranks(values, world, device)
+    if [-x for x in lo] != hi:
+        raise RuntimeError(f"ranks disagree on the workload: min {[-x for x in lo]} max {hi}")
+
+
 def job_throughput(world: int, units_per_rank: int, steps: int, max_ms: float) -> float:
     """Whole-job units per second: every rank runs a replica of the workload,
     so the job processes world * units_per_rank per step, in the slowest
     rank's time."""
     return world * units_per_rank * steps / (max_ms * 1e-3)
+
+
+def zero2_throughput(P: int, steps: int, max_ms: float) -> float:
+    """The ZeRO-2 step across GPUs updates the P parameters once per step,
+    whatever the number of GPUs sharing it."""
+    return P * steps / (max_ms * 1e-3)
 
 
 # ------------------------------------------------------------ arms
@@ -333,44 +494,24 @@ def run_gpu(args) -> None:
     world, rank, local = rank_env()
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if world > 1:
+    kind = WORKLOADS[args.workload][0]
+    if world > 1 or kind == "zero2":
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29531")
+        os.environ.setdefault("RANK", "0")
+        os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    agree_on([len(args.workload), sum(map(ord, args.workload)), args.steps, args.warmup], world, device)
 
-    z = build_workload(args.workload, device)
     stream = torch.cuda.current_stream(device)
-    from mixed_precision_adam_zero_b200 import (ZERO_BF16, ZERO_F16, ZERO_F32, make_accum_args,
-                                                zero_accumulate_grads, zero_step_fused, zero_step_fused_list)
-    if hasattr(z, "gl"):
-        from mixed_precision_adam_zero_b200 import zero3_gather
-        call = lambda: zero3_gather(z.gl, stream)
-    elif hasattr(z, "owner_args"):
-        def call():
-            for a in z.owner_args:
-                zero_step_fused(a, stream)
-    elif getattr(z, "gas", 0):
-        step_args = z.step_args(hp=ADAMW, check=z.check, grads=[z.accum])
-        gcode = {"bf16": ZERO_BF16, "f16": ZERO_F16, "f32": ZERO_F32}[z.micro_gdt]
-        micro_args = [make_accum_args(z.P, z.micro_R, grad_dtype=gcode, grads=z.micro, accum=z.accum,
-                                      scale=1.0 / z.gas, first=(mu == 0), workspace=z.workspace,
-                                      ctrl=z.ctrl_buf) for mu in range(z.gas)]
-
-        def call():
-            for a in micro_args:
-                zero_accumulate_grads(a, stream=stream)
-            zero_step_fused(step_args, stream)
-    elif hasattr(z, "list"):
-        step_args = z.step_args(hp=ADAMW, check=z.check)
-        call = lambda: zero_step_fused_list(step_args, z.list, stream)
-    else:
-        step_args = z.step_args(hp=ADAMW, check=z.check)
-        call = lambda: zero_step_fused(step_args, stream)
+    b = build_workload(args.workload, device, stream, world)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
 
     for _ in range(args.warmup):
-        call()
+        b.call()
     torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
@@ -381,7 +522,7 @@ def run_gpu(args) -> None:
     with ClockSampler(local) as clocks:
         for i in range(K):
             starts[i].record(stream)
-            call()
+            b.call()
             ends[i].record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -390,116 +531,114 @@ def run_gpu(args) -> None:
     per_launch_ms = statistics.fmean(per_launch)
     median_launch_ms = statistics.median(per_launch)
 
-    # end to end: host (pinned) gradients copied in, 16-bit parameters read back, every step.
-    # The read-back of step k runs on its own stream, on the device-to-host
-    # copy engine, while step k+1's gradients come in; step k+1's kernel waits
-    # for it before it overwrites the 16-bit parameters.
-    K_e2e = min(K, args.e2e_steps)
-    h2d = sum(g.numel() * g.element_size() for g in z.gbufs)
-    if h2d > (8 << 30):
-        K_e2e = 0          # pinned host copies of this workload would not fit comfortably
-    host_grads = [g.cpu().pin_memory() for g in z.gbufs] if K_e2e else []
-    p16 = z.flat_p16 if hasattr(z, "flat_p16") else z.params16
-    host_p16 = torch.empty(p16.shape, dtype=p16.dtype).pin_memory() if K_e2e else None
+    # End to end: every step copies its gradients in from pinned host memory
+    # and reads the 16-bit parameters back.  The read-back of step k runs on
+    # its own stream (the device-to-host copy engine) while step k+1's
+    # gradients come in; step k+1's kernel waits for it before it overwrites
+    # the parameters.
+    h2d = sum(g.numel() * g.element_size() for g in b.inputs)
+    d2h = b.output.numel() * b.output.element_size()
+    K_e2e = e2e_step_count(K, h2d, args.e2e_steps)
+    if K_e2e:
+        host_in = torch.empty(sum(g.numel() for g in b.inputs), dtype=b.inputs[0].dtype, pin_memory=True)
+        host_grads = list(host_in.split([g.numel() for g in b.inputs]))
+        for hg, dg in zip(host_grads, b.inputs):
+            hg.copy_(dg.view(-1))
+        host_out = torch.empty(b.output.shape, dtype=b.output.dtype, pin_memory=True)
+        torch.cuda.synchronize()
     d2h_stream = torch.cuda.Stream(device)
 
     def e2e_steps(n):
         read_back = None
         for _ in range(n):
-            for hg, dg in zip(host_grads, z.gbufs):
-                dg.copy_(hg, non_blocking=True)
+            for hg, dg in zip(host_grads, b.inputs):
+                dg.view(-1).copy_(hg, non_blocking=True)
             if read_back is not None:
                 stream.wait_event(read_back)
-            call()
+            b.call()
             computed = torch.cuda.Event()
             computed.record(stream)
             d2h_stream.wait_event(computed)
             with torch.cuda.stream(d2h_stream):
-                host_p16.copy_(p16, non_blocking=True)
+                host_out.copy_(b.output, non_blocking=True)
             read_back = torch.cuda.Event()
             read_back.record(d2h_stream)
         if read_back is not None:
             stream.wait_event(read_back)
 
-    e2e_steps(2 if K_e2e else 0)
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    e2e_steps(K_e2e)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = 0.0
+    if K_e2e:
+        e2e_steps(1)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        e2e_steps(K_e2e)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
     total_ms, per_launch_ms, median_launch_ms, e2e_ms = max_over_ranks(
         [total_ms, per_launch_ms, median_launch_ms, e2e_ms], world, device)
-    ctrl = z.ctrl()
+    ctrl = b.ctrl()
 
     if rank == 0:
-        kind, size, R, gdt, pdt, scaled = WORKLOADS[args.workload]
-        P = z.P
-        bpp = 4 if kind == "z3gather" else (zero2emu_bytes_per_param(R, gdt) if kind == "zero2emu" else
-                                            bytes_per_param(R, gdt, GAS.get(args.workload, 0)))
-        peaks = measured_peaks()
-        peak = peaks.get("hbm_gbs")
-        peak_src = "measured" if peak else "fallback"
-        peak = peak or 6650.0
+        P = b.P
+        cfg = workload_config(args.workload, world)
+        assert cfg["P"] == P, (cfg["P"], P)
         ms_step = total_ms / K
-        achieved = bpp * P / (per_launch_ms * 1e-3) / 1e9
-        traffic = traffic_for(args.workload)
+        if kind == "zero2":
+            value, e2e_value = zero2_throughput(P, K, total_ms), zero2_throughput(P, K_e2e, e2e_ms or 1.0)
+        else:
+            value, e2e_value = job_throughput(world, P, K, total_ms), job_throughput(world, P, K_e2e, e2e_ms or 1.0)
+        rf = roofline(args.workload, world, P, per_launch_ms, measured_peaks(), traffic_for(args.workload))
+        rf["launch_ms_median"] = median_launch_ms
+        bpp = cfg["bytes_per_param"]
         line = {
             "metric": METRIC,
-            "value": job_throughput(world, P, K, total_ms),
+            "value": value,
             "unit": UNIT,
             "n_gpus": world,
             "steps": K,
             "warmup": args.warmup,
             "ms_per_step": ms_step,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if kind == "zero2" else "weak",
             "vs_baseline": None,
             "dtype": "f32",
             "data": "synthetic",
-            "config": {
-                "workload": args.workload, "P": P, "R": R, "grad_dtype": gdt, "param_dtype": pdt,
-                "optimizer": "AdamW lr=1e-3 betas=(0.8,0.999) eps=1e-8 wd=3e-7",
-                "loss_scale_check": bool(scaled), "bytes_per_param": bpp,
-                "hbm_gbs_algorithmic": bpp * P / (ms_step * 1e-3) / 1e9,
-                "l2": f"inputs larger than L2 ({bpp * P / 1e6:.0f} MB touched per step vs 126 MB L2), no flush",
-                "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                "applied_steps": int(ctrl.step),
-            },
-            "roofline": {
-                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_source": f"{peak_src} hbm_gbs",
-                "traffic": traffic,
-                # the ncu-measured DRAM bytes of one launch over the live launch time
-                "traffic_gbs": traffic / (per_launch_ms * 1e-3) / 1e9 if traffic else None,
-                "kernel": roofline_kernel(args.workload),
-                "bytes_per_launch": bpp * P, "launch_ms": per_launch_ms, "launch_ms_median": median_launch_ms,
-            },
+            "config": cfg,
+            "hbm_gbs_algorithmic": bpp * P / (ms_step * 1e-3) / 1e9 / (world if kind == "zero2" else 1),
+            "applied_steps": int(ctrl.step) if ctrl is not None else None,
+            "roofline": rf,
             "e2e": {
-                "value": job_throughput(world, P, K_e2e, e2e_ms), "unit": UNIT, "steps": K_e2e,
-                "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": p16.numel() * p16.element_size(),
+                "value": e2e_value, "unit": UNIT, "steps": K_e2e,
+                # the whole job: every GPU copies its own inputs in and its result out
+                "h2d_bytes_per_step": h2d * world,
+                "d2h_bytes_per_step": d2h * world,
             } if K_e2e else None,
-            "gpu_launches": K * launches_per_step(z),
+            "gpu_launches": K * b.launches,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if world > 1 or kind == "zero2":
+        del b
+        torch.cuda.synchronize()
         dist.destroy_process_group()
 
 
 def _oracle_sample(workload: str, n: int):
-    """Host inputs for the oracle: the first n parameters of the workload."""
+    """Host inputs for the oracle: the first n parameters of the workload,
+    drawn from the workload's distributions (masters N(0, 0.02), gradients
+    N(0, 1e-3) times the loss scale) with the workload's seeds on the host."""
     import numpy as np
     import torch
     import oracle
     import synth
     kind, size, R, gdt, pdt, scaled = WORKLOADS[workload]
+    R = R or 1
     wl = synth.WORKLOADS.get(workload.split("_")[0], 9)
     S = 65536.0 if scaled else 1.0
     tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt]
@@ -512,34 +651,56 @@ def _oracle_sample(workload: str, n: int):
     return st, grads, gdt, scaled
 
 
-def cpu_baseline(workload: str, seconds: float) -> dict:
-    """The float64 oracle, as it stands, on this host's cores: steps over a
-    bounded sample of the workload until `seconds` have passed."""
+def oracle_sample_size(workload: str) -> int:
+    return min(ORACLE_SAMPLE_P, workload_P(workload))
+
+
+def _oracle_rate(st, grads, gdt, scaled, n: int, threads: int, seconds: float, min_steps: int = 1):
+    """Steps of the oracle on `threads` threads until `seconds` have passed
+    (at least min_steps): (params/s, steps, elapsed s)."""
     import oracle
-    n = min(WORKLOADS[workload][1] if isinstance(WORKLOADS[workload][1], int) else 1 << 24, 1 << 24)
-    st, grads, gdt, scaled = _oracle_sample(workload, n)
     hp = oracle.HP(*ADAMW)
+    oracle.set_threads(threads)
     steps, t0 = 0, time.perf_counter()
     while True:
         oracle.step(st, grads, gdt, hp, check=scaled)
         steps += 1
         el = time.perf_counter() - t0
-        if el >= seconds:
+        if steps >= min_steps and el >= seconds:
             break
-    return {"value": n * steps / el, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": f"first {n} parameters of {workload}, {WORKLOADS[workload][2]} ranks, {steps} steps, "
-                      f"{el:.1f} s (float64 C loops, OpenMP)"}
+    return n * steps / el, steps, el
+
+
+def cpu_baseline(workload: str, seconds: float) -> dict:
+    """The float64 oracle, as it stands, on this host's cores, over the first
+    ORACLE_SAMPLE_P parameters of the workload: on every core for `seconds`,
+    then on one thread for about half as long."""
+    import oracle
+    n = oracle_sample_size(workload)
+    st, grads, gdt, scaled = _oracle_sample(workload, n)
+    cores = oracle.max_threads()
+    v_all, s_all, el_all = _oracle_rate(st, grads, gdt, scaled, n, cores, seconds)
+    v_one, s_one, el_one = _oracle_rate(st, grads, gdt, scaled, n, 1, seconds / 2)
+    oracle.set_threads(cores)
+    R = workload_R(workload)
+    return {"value": v_all, "unit": UNIT, "cores": cores, "kind": "oracle", "sample_P": n,
+            "sample": f"first {n} parameters of {workload}, {R} ranks, float64 C loops (OpenMP): "
+                      f"{s_all} steps in {el_all:.1f} s on {cores} threads, {s_one} steps in {el_one:.1f} s "
+                      f"on 1 thread",
+            "single_thread": {"value": v_one, "unit": UNIT, "cores": 1, "steps": s_one}}
 
 
 def run_reference(args) -> None:
-    """Reference arm: the float64 CPU oracle on the same workload, each step a
-    bounded sample of it; rank 0 alone runs it under torchrun."""
+    """Reference arm: the float64 CPU oracle on the same workload, each step
+    the first ORACLE_SAMPLE_P parameters of it (the cpu_baseline's sample), on
+    every host core; also its single-thread rate.  Rank 0 alone runs it."""
     if rank_env()[1] != 0:
         return
     import oracle
-    n = 1 << 20
+    n = oracle_sample_size(args.workload)
     st, grads, gdt, scaled = _oracle_sample(args.workload, n)
     hp = oracle.HP(*ADAMW)
+    cores = oracle.max_threads()
     for _ in range(args.warmup):
         oracle.step(st, grads, gdt, hp, check=scaled)
     t0 = time.perf_counter()
@@ -547,17 +708,20 @@ def run_reference(args) -> None:
         oracle.step(st, grads, gdt, hp, check=scaled)
     el = time.perf_counter() - t0
     value = n * args.steps / el
-    kind, size, R, g, p, sc = WORKLOADS[args.workload]
-    P = size if isinstance(size, int) else None
+    v_one, s_one, _ = _oracle_rate(st, grads, gdt, scaled, n, 1, args.cpu_seconds / 4)
+    oracle.set_threads(cores)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     line = {
         "impl": "reference",
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "P": P, "R": R, "grad_dtype": g, "param_dtype": p,
-                   "optimizer": "AdamW lr=1e-3 betas=(0.8,0.999) eps=1e-8 wd=3e-7"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
-                         "sample": f"first {n} parameters of {args.workload} per step"},
+        "higher_is_better": True, "scaling": "strong" if WORKLOADS[args.workload][0] == "zero2" else "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.workload, world),
+        "sample_P": n,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample_P": n,
+                         "sample": f"first {n} parameters of {args.workload} per step, {cores} threads",
+                         "single_thread": {"value": v_one, "unit": UNIT, "cores": 1, "steps": s_one}},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -566,16 +730,18 @@ def run_reference(args) -> None:
 def main() -> None:
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="flat16m", choices=sorted(WORKLOADS))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=50)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.workload is None:
+        args.workload = DEFAULT_WORKLOAD_MULTI if rank_env()[0] > 1 else DEFAULT_WORKLOAD
     if args.impl == "reference":
         run_reference(args)
     else:

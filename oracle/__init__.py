@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
         L.zo_accumulate.argtypes = [u64, u32, i32, pp, dp, ctypes.c_double, i32,
                                     ctypes.POINTER(ctypes.c_float)]
         L.zo_max_threads.restype = ctypes.c_int
+        L.zo_set_threads.argtypes = [ctypes.c_int]
+        L.zo_set_threads.restype = None
         _lib_handle = L
     return _lib_handle
 
@@ -109,6 +111,11 @@ def lib() -> ctypes.CDLL:
 def max_threads() -> int:
     """Threads the oracle's OpenMP loops use."""
     return int(lib().zo_max_threads())
+
+
+def set_threads(n: int) -> None:
+    """Threads for the oracle's next OpenMP loops (n >= 1)."""
+    lib().zo_set_threads(int(n))
 
 
 # ------------------------------------------------------------------ ownership

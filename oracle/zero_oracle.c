@@ -367,3 +367,15 @@ int zo_max_threads(void)
     return 1;
 #endif
 }
+
+/* Threads for the following OpenMP loops of this process (n >= 1); used to
+ * time the oracle single-threaded and on all cores. */
+void zo_set_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

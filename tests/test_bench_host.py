@@ -1,9 +1,12 @@
 """Host-side pieces of the benchmark: the workload table, the algorithmic
-bytes per parameter of each workload (the metric's formula), the kernel
+bytes per parameter of each workload (the metric's formula), the static
+workload description both arms print, the end-to-end step budget, the kernel
 label of each roofline, and the traffic record's keys."""
 import json
 import os
 import sys
+
+import pytest
 
 from conftest import ROOT
 
@@ -23,8 +26,9 @@ def test_bytes_per_parameter_follow_the_formula():
 
 def test_every_workload_has_a_kernel_label_and_valid_fields():
     for name, (kind, size, R, gdt, pdt, scaled) in bench.WORKLOADS.items():
-        assert kind in ("flat", "list", "z3gather", "zero2emu"), name
-        assert 1 <= R <= 256 and gdt in bench.GRAD_BYTES and pdt in ("bf16", "f16"), name
+        assert kind in ("flat", "list", "z3gather", "zero2emu", "zero2"), name
+        assert (kind == "zero2" and R == 0) or 1 <= R <= 256, name
+        assert gdt in bench.GRAD_BYTES and pdt in ("bf16", "f16"), name
         label = bench.roofline_kernel(name)
         assert "kernel" in label, name
         if scaled:
@@ -41,6 +45,66 @@ def test_traffic_record_names_known_workloads_and_current_format():
         assert os.path.exists(os.path.join(ROOT, e["summary"])), e["summary"]
 
 
-def test_default_workload_is_the_16m_flat_configuration():
-    kind, size, R, gdt, pdt, scaled = bench.WORKLOADS["flat16m"]
-    assert (kind, size, R, gdt, pdt, scaled) == ("flat", 16_777_259, 8, "bf16", "bf16", False)
+def test_default_workload_is_the_3p2b_llama_list():
+    assert bench.DEFAULT_WORKLOAD == "llama3b" and bench.DEFAULT_WORKLOAD_MULTI == "zero2"
+    cfg = bench.workload_config("llama3b")
+    assert (cfg["P"], cfg["R"], cfg["tensors"], cfg["grad_dtype"], cfg["param_dtype"]) == \
+        (3_212_749_824, 8, 254, "bf16", "bf16")
+    assert cfg["bytes_per_param"] == 42 and cfg["P"] >= 100_000_000
+    assert cfg["l2"].startswith("inputs larger than L2")
+
+
+def test_small_capture_cases_share_the_kernel_instances_of_the_large_workloads():
+    pairs = [("llama3b_layer", "llama3b"), ("gpt2m_head", "gpt2m"), ("flat64m_r4", "flat1p5b"),
+             ("flat64m_r4_f32", "flat1p5b_f32")]
+    for small, large in pairs:
+        ks, _, Rs, gs, ps, ss = bench.WORKLOADS[small]
+        kl, _, Rl, gl, pl, sl = bench.WORKLOADS[large]
+        assert (ks, Rs, gs, ps, ss) == (kl, Rl, gl, pl, sl), small
+        # a few GB on the device at most: R gradients, 12 bytes of state, the 16-bit parameters
+        P = bench.workload_P(small)
+        assert P * (bench.GRAD_BYTES[gs] * Rs + 14) < 4e9, small
+    assert bench.workload_P("llama3b_layer") == 3072 * 3072 * 2 + 3072 * 1024 * 2 + 3 * 3072 * 8192 + 2 * 3072
+
+
+def test_workload_config_is_static_and_complete():
+    for name in bench.WORKLOADS:
+        a, b = bench.workload_config(name), bench.workload_config(name)
+        assert a == b
+        assert {"workload", "P", "R", "grad_dtype", "param_dtype", "optimizer", "bytes_per_param", "l2",
+                "parallelism"} <= set(a)
+        assert a["P"] == bench.workload_P(name)
+
+
+def test_zero2_workload_scales_with_the_world():
+    for world in (1, 2, 8):
+        cfg = bench.workload_config("zero2", world)
+        assert cfg["R"] == world and cfg["P"] == bench.LLAMA3B_P
+        assert cfg["bytes_per_param"] == 2 * world + 24 + 2 * world
+    P = bench.LLAMA3B_P
+    assert bench.nvlink_bytes_per_direction(P, 1) == 0
+    assert bench.nvlink_bytes_per_direction(P, 8) == 7 * P * 2 // 8
+    rf = bench.roofline("zero2", 8, P, 10.0, {}, None)
+    assert rf["bound"] == "nvlink" and rf["peak"] == bench.NVLINK_GBS
+    assert rf["achieved"] == pytest.approx(7 * P * 2 / 8 / 1e-2 / 1e9)
+    rf1 = bench.roofline("zero2", 1, P, 10.0, {"hbm_gbs": 6546.6}, None)
+    assert rf1["bound"] == "hbm" and rf1["bytes_per_launch"] == 28 * P
+    assert bench.zero2_throughput(P, 4, 8.0) == pytest.approx(P * 4 / 8e-3)
+
+
+def test_e2e_step_budget():
+    assert bench.e2e_step_count(20, 268_436_144) == 20                  # small inputs: every timed step
+    assert bench.e2e_step_count(20, 8 * 2 * 3_212_749_824) == 2         # 51 GB per step: two steps
+    assert bench.e2e_step_count(1, 8 * 2 * 3_212_749_824) == 1          # never more than the timed steps
+    assert bench.e2e_step_count(20, 1 << 30, requested=5) == 5
+    assert bench.e2e_step_count(20, 1 << 30, requested=0) == 0
+
+
+def test_roofline_arithmetic():
+    rf = bench.roofline("llama3b", 1, 3_212_749_824, 20.0, {"hbm_gbs": 6546.6}, 1234)
+    assert rf["bound"] == "hbm" and rf["peak"] == 6546.6 and rf["peak_source"] == "measured hbm_gbs"
+    assert rf["achieved"] == pytest.approx(42 * 3_212_749_824 / 20e-3 / 1e9)
+    assert rf["frac"] == pytest.approx(rf["achieved"] / 6546.6)
+    assert rf["traffic"] == 1234
+    fb = bench.roofline("flat16m", 1, 16_777_259, 0.1, {}, None)
+    assert fb["peak_source"] == "fallback hbm_gbs" and fb["peak"] == 6650.0

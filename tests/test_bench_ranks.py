@@ -1,7 +1,8 @@
 """The benchmark's multi-rank plumbing on CPU: two gloo ranks run the same
 max-over-ranks reduction and throughput rule the GPU run uses (one replica of
-the workload per GPU, no collective on the data path), and the reference arm
-runs on rank 0 only."""
+the workload per GPU, no collective on the data path), the ranks' check that
+they run the same workload, the slices and NVLink bytes of the ZeRO-2 step
+across GPUs, and the reference arm on rank 0 only."""
 import json
 import os
 import socket
@@ -67,3 +68,55 @@ def test_reference_arm_runs_on_rank_zero_only():
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["n_gpus"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+def _zero2_worker(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    from mixed_precision_adam_zero_b200.zero2 import rank_slice
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        w, r, _ = bench.rank_env()
+        bench.agree_on([7, 11, 20], w, "cpu")                   # the same run on both ranks: no error
+        try:
+            bench.agree_on([7, 11 + r], w, "cpu")                # rank 1 asks for another workload
+            disagreed = False
+        except RuntimeError:
+            disagreed = True
+        P = bench.LLAMA3B_P
+        cfg = bench.workload_config("zero2", w)
+        lo, hi, off, n = rank_slice(P, w, r)
+        slices = [None] * w
+        dist.all_gather_object(slices, (lo, hi, off, n))
+        q.put((r, disagreed, cfg, slices))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_zero2_plumbing_with_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_zero2_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    out = sorted(q.get(timeout=10) for _ in range(2))
+    sys.path.insert(0, ROOT)
+    import bench
+    P = bench.LLAMA3B_P
+    for r, disagreed, cfg, slices in out:
+        assert disagreed                                        # both ranks refuse, before any step
+        assert cfg["R"] == 2 and cfg["P"] == P and cfg["workload"] == "zero2"
+        assert slices[0][0] == 0 and slices[0][1] == slices[1][0] and slices[1][1] == P   # they tile [0, P)
+        assert all(off % 8 == 0 and off <= lo and n >= hi - off for lo, hi, off, n in slices)
+        # each rank pulls the other's gradient over its own slice and pushes its results out
+        pulled = [(2 - 1) * (hi - lo) * 2 for lo, hi, _, _ in slices]
+        assert sum(pulled) == 2 * bench.nvlink_bytes_per_direction(P, 2)
