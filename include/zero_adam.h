@@ -111,6 +111,23 @@ typedef struct zero_ctrl {
     uint32_t reserved;        /* zero */
 } zero_ctrl;
 
+/* Kernel paths of the step and of the accumulation (field `path`):
+ *   ZERO_PATH_STAGED   one producer thread per CTA stages tiles of every
+ *                      input array into shared memory with 1-D bulk copies
+ *                      (cp.async.bulk, no tensor map, no multicast); compiled
+ *                      for 1, 2, 4 and 8 gradient buffers;
+ *   ZERO_PATH_REGISTER every thread reads its gradients with plain 16-byte
+ *                      global loads (ld.global) into registers; any count;
+ *   ZERO_PATH_AUTO     the staged kernel when one is compiled for the count
+ *                      (the faster one at nearly every size), else the
+ *                      register kernel.
+ * Both give bitwise identical results.  Across GPUs the gradient buffers are
+ * other GPUs' memory mapped into this process: ZERO_PATH_REGISTER then reads
+ * them with ordinary peer loads instead of bulk copies. */
+#define ZERO_PATH_AUTO 0
+#define ZERO_PATH_REGISTER 1
+#define ZERO_PATH_STAGED 2
+
 /* Arguments of one step over a FLAT parameter vector of P elements.
  *
  * Layout: every array is indexed by the flat parameter index i in [0, P);
@@ -181,7 +198,9 @@ typedef struct zero_step_args {
                                      at most lo; 0 for arrays of P elements. */
     uint32_t n_push;              /* 0..ZERO_MAX_PUSH; nonzero needs
                                      owner >= 0 (ZERO_EINVAL otherwise) */
-    uint32_t reserved;            /* zero */
+    uint32_t path;                /* which step kernel reads the gradients:
+                                     ZERO_PATH_AUTO (0), ZERO_PATH_REGISTER or
+                                     ZERO_PATH_STAGED (see below) */
     void *const *push_params16;   /* HOST array of n_push device pointers,
                                      each [P] of param_dtype: the other ranks'
                                      replicated 16-bit parameters (peer
@@ -326,6 +345,9 @@ int zero_selftest_wait_timeout(void *ctrl, void *stream);
  * (b) check on in two-set mode with owner == -1: one pass plus a restore
  * kernel that, only if the step was skipped, re-casts the 16-bit parameters
  * from the untouched master set.
+ * The step kernel is the one args->path selects; ZERO_PATH_STAGED with a
+ * gradient-buffer count other than 1, 2, 4 or 8, or an unknown path, is
+ * ZERO_EINVAL.
  * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ERANGE (R > ZERO_MAX_RANKS),
  * ZERO_EOVERFLOW (P*4 bytes overflow), ZERO_ECUDA. */
 int zero_step_fused(const zero_step_args *args, void *stream);
@@ -424,13 +446,9 @@ typedef struct zero_accum_args {
                                     the slice's first element; 0 for [P] */
 } zero_accum_args;
 
-#define ZERO_PATH_AUTO 0
-#define ZERO_PATH_REGISTER 1
-#define ZERO_PATH_STAGED 2
-
-/* Launches one kernel; asynchronous on `stream`.  The staged kernel stages
- * its tiles in shared memory by bulk copies and hands them out dynamically;
- * it needs a workspace and ctrl and R = 1, 2, 4 or 8.  The register kernel
+/* Launches one kernel; asynchronous on `stream`.  The staged kernel
+ * (ZERO_PATH_STAGED above) hands its tiles out dynamically; here it needs a
+ * workspace and ctrl and R = 1, 2, 4 or 8.  The register kernel
  * streams through registers and touches neither workspace nor ctrl.  Both
  * give bitwise identical sums.  ZERO_PATH_AUTO takes the staged kernel
  * whenever it is possible (the faster one at nearly every size), else the

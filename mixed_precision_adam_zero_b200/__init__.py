@@ -98,7 +98,7 @@ class zero_step_args(ctypes.Structure):
                 ("reduced_out", ctypes.c_void_p), ("hp", zero_adam_hparams),
                 ("check_nonfinite", ctypes.c_int32), ("growth_interval", ctypes.c_uint32),
                 ("ctrl", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-                ("state_offset", ctypes.c_uint64), ("n_push", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
+                ("state_offset", ctypes.c_uint64), ("n_push", ctypes.c_uint32), ("path", ctypes.c_uint32),
                 ("push_params16", ctypes.POINTER(ctypes.c_void_p)), ("n_grads", ctypes.c_uint32),
                 ("reserved2", ctypes.c_uint32), ("grad_offset", ctypes.c_uint64)]
 
@@ -269,7 +269,7 @@ def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master,
                    check_nonfinite: int = 0, growth_interval: int = 0, reduced_out=None,
                    master2=None, exp_avg2=None, exp_avg_sq2=None, state_offset: int = 0,
                    push_params16: Optional[Sequence] = None, n_grads: int = 0,
-                   grad_offset: int = 0) -> zero_step_args:
+                   grad_offset: int = 0, path: int = 0) -> zero_step_args:
     """Fill a zero_step_args (the returned struct keeps its host arrays alive)."""
     a = zero_step_args()
     a.P, a.R, a.owner = P, R, owner
@@ -292,6 +292,7 @@ def make_step_args(P: int, R: int, *, grad_dtype: int, param_dtype: int, master,
     a.ctrl, a.workspace = _ptr(ctrl), _ptr(workspace)
     a.state_offset = state_offset
     a.n_grads, a.grad_offset = n_grads, grad_offset
+    a.path = path
     if push_params16:
         arr = (ctypes.c_void_p * len(push_params16))(*[_ptr(t) for t in push_params16])
         a._push_keep = arr

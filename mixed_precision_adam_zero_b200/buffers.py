@@ -59,7 +59,7 @@ class _Common:
         k = self.ctrl().parity if self.two_set else 0
         return self.master[k], self.exp_avg[k], self.exp_avg_sq[k]
 
-    def _args(self, hp, rank_weights, check, owner, growth_interval, reduced_out, **kw):
+    def _args(self, hp, rank_weights, check, owner, growth_interval, reduced_out, path=0, **kw):
         two = self.two_set
         return make_step_args(
             self.P, self.R, grad_dtype=self.gcode, param_dtype=self.pcode,
@@ -67,7 +67,8 @@ class _Common:
             master2=self.master[1] if two else None, exp_avg2=self.exp_avg[1] if two else None,
             exp_avg_sq2=self.exp_avg_sq[1] if two else None,
             ctrl=self.ctrl_buf, workspace=self.workspace, rank_weights=rank_weights, owner=owner,
-            hp=hp, check_nonfinite=check, growth_interval=growth_interval, reduced_out=reduced_out, **kw)
+            hp=hp, check_nonfinite=check, growth_interval=growth_interval, reduced_out=reduced_out, path=path,
+            **kw)
 
 
 class FlatZero(_Common):
@@ -93,8 +94,8 @@ class FlatZero(_Common):
         zero_gather_params(self.master[0], self.params16, self.pcode, self.P, s)
 
     def step_args(self, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), rank_weights=None, check=False, owner=-1,
-                  growth_interval=0, reduced_out=None, grads: Optional[Sequence] = None):
-        return self._args(hp, rank_weights, check, owner, growth_interval, reduced_out,
+                  growth_interval=0, reduced_out=None, grads: Optional[Sequence] = None, path: int = 0):
+        return self._args(hp, rank_weights, check, owner, growth_interval, reduced_out, path=path,
                           grads=list(grads if grads is not None else self.grads), params16=self.params16)
 
     def step(self, **kw) -> None:
@@ -133,8 +134,8 @@ class ListZero(_Common):
         zero_gather_params_list(self.master[0], self.list, s)
 
     def step_args(self, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), rank_weights=None, check=False, owner=-1,
-                  growth_interval=0, reduced_out=None):
-        return self._args(hp, rank_weights, check, owner, growth_interval, reduced_out)
+                  growth_interval=0, reduced_out=None, path: int = 0):
+        return self._args(hp, rank_weights, check, owner, growth_interval, reduced_out, path=path)
 
     def step(self, **kw) -> None:
         zero_step_fused_list(self.step_args(**kw), self.list, self._s())

@@ -111,7 +111,8 @@ Kern bulk_kern() {
 }
 
 template <class G, class Pm, bool LIST, bool PUSH>
-Kern step_kern_rc(uint32_t R) {
+Kern step_kern_rc(uint32_t R, bool staged) {
+    if (!staged) return Kern{(const void*)step_kernel<G, Pm, 0, LIST, PUSH>, 0u, kThreads};
     switch (R) {
         case 1: return bulk_kern<G, Pm, 1, LIST, PUSH>();
         case 2: return bulk_kern<G, Pm, 2, LIST, PUSH>();
@@ -122,24 +123,29 @@ Kern step_kern_rc(uint32_t R) {
 }
 
 template <class G, bool LIST, bool PUSH>
-Kern step_kern_pm(int32_t param_dtype, uint32_t R) {
-    return param_dtype == ZERO_BF16 ? step_kern_rc<G, __nv_bfloat16, LIST, PUSH>(R)
-                                    : step_kern_rc<G, __half, LIST, PUSH>(R);
+Kern step_kern_pm(int32_t param_dtype, uint32_t R, bool staged) {
+    return param_dtype == ZERO_BF16 ? step_kern_rc<G, __nv_bfloat16, LIST, PUSH>(R, staged)
+                                    : step_kern_rc<G, __half, LIST, PUSH>(R, staged);
 }
 
 template <bool LIST, bool PUSH>
-Kern step_kern_gd(int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
+Kern step_kern_gd(int32_t grad_dtype, int32_t param_dtype, uint32_t R, bool staged) {
     switch (grad_dtype) {
-        case ZERO_F32: return step_kern_pm<float, LIST, PUSH>(param_dtype, R);
-        case ZERO_BF16: return step_kern_pm<__nv_bfloat16, LIST, PUSH>(param_dtype, R);
-        default: return step_kern_pm<__half, LIST, PUSH>(param_dtype, R);
+        case ZERO_F32: return step_kern_pm<float, LIST, PUSH>(param_dtype, R, staged);
+        case ZERO_BF16: return step_kern_pm<__nv_bfloat16, LIST, PUSH>(param_dtype, R, staged);
+        default: return step_kern_pm<__half, LIST, PUSH>(param_dtype, R, staged);
     }
 }
 
-Kern step_kern(bool list, bool push, int32_t grad_dtype, int32_t param_dtype, uint32_t R) {
-    if (list) return step_kern_gd<true, false>(grad_dtype, param_dtype, R);
-    return push ? step_kern_gd<false, true>(grad_dtype, param_dtype, R)
-                : step_kern_gd<false, false>(grad_dtype, param_dtype, R);
+bool has_staged(uint32_t R) { return R == 1 || R == 2 || R == 4 || R == 8; }
+
+// The step kernel for a path (ZERO_PATH_*): staged when asked for or, in
+// AUTO, when one is compiled for R; else the register kernel.
+Kern step_kern(bool list, bool push, int32_t grad_dtype, int32_t param_dtype, uint32_t R, uint32_t path) {
+    const bool staged = path != ZERO_PATH_REGISTER && has_staged(R);
+    if (list) return step_kern_gd<true, false>(grad_dtype, param_dtype, R, staged);
+    return push ? step_kern_gd<false, true>(grad_dtype, param_dtype, R, staged)
+                : step_kern_gd<false, false>(grad_dtype, param_dtype, R, staged);
 }
 
 template <bool LIST>
@@ -221,7 +227,9 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     if (!is_grad_dtype(a->grad_dtype) || !is_param_dtype(a->param_dtype)) return ZERO_EINVAL;
     if (a->check_nonfinite < 0 || a->check_nonfinite > 2) return ZERO_EINVAL;
     if (a->n_push > ZERO_MAX_PUSH) return ZERO_ERANGE;
-    if (a->reserved != 0u || (a->n_push > 0 && a->push_params16 == nullptr)) return ZERO_EINVAL;
+    if (a->n_push > 0 && a->push_params16 == nullptr) return ZERO_EINVAL;
+    if (a->path != ZERO_PATH_AUTO && a->path != ZERO_PATH_REGISTER && a->path != ZERO_PATH_STAGED)
+        return ZERO_EINVAL;
     if ((a->state_offset & 7u) != 0 || (a->grad_offset & 7u) != 0) return ZERO_EALIGN;
     if (a->n_grads > ZERO_MAX_RANKS) return ZERO_ERANGE;
     if (a->reserved2 != 0u || (a->grad_offset != 0 && a->check_nonfinite == 1)) return ZERO_EINVAL;
@@ -291,6 +299,7 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     kp->ctrl = static_cast<zero_ctrl*>(a->ctrl);
     kp->ws = static_cast<Workspace*>(a->workspace);
     kp->R = ng;  // the reduction's length; the partition is a->R (owner_range)
+    if (a->path == ZERO_PATH_STAGED && !has_staged(ng)) return ZERO_EINVAL;
     kp->growth_interval = a->growth_interval;
     kp->two_set = two ? 1 : 0;
     return ZERO_OK;
@@ -333,7 +342,7 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
     } else {
         kp->check = check ? 1 : 0;
     }
-    const Kern k = step_kern(LIST, kp->npush > 0, a->grad_dtype, a->param_dtype, kp->R);
+    const Kern k = step_kern(LIST, kp->npush > 0, a->grad_dtype, a->param_dtype, kp->R, a->path);
     const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;
     const Shape sh = make_shape(lo, hi, ctas);

@@ -125,8 +125,11 @@ class Zero2Rank:
     """One process's share of a ZeRO-2 optimizer over the group's R ranks."""
 
     def __init__(self, P: int, grad_dtype: str = "bf16", param_dtype: str = "bf16", *, group=None,
-                 loss_scale: float = 1.0, device=None, peers=None):
+                 loss_scale: float = 1.0, device=None, peers=None, path: int = 0):
+        """path: the step and accumulation kernels' ZERO_PATH_* (AUTO: staged
+        bulk copies from the peers' buffers; REGISTER: plain peer loads)."""
         self.group = group
+        self.path = path
         self.R = dist.get_world_size(group)
         self.r = dist.get_rank(group)
         self.P = P
@@ -178,7 +181,7 @@ class Zero2Rank:
             exp_avg=self.exp_avg, exp_avg_sq=self.exp_avg_sq, ctrl=self.ctrl_buf, workspace=self.workspace,
             grads=self.peer_grads, params16=self.params16, rank_weights=rank_weights, owner=self.r, hp=hp,
             check_nonfinite=2 if check else 0, growth_interval=growth_interval, state_offset=self.state_offset,
-            push_params16=[t for j, t in enumerate(self.peer_params16) if j != self.r])
+            push_params16=[t for j, t in enumerate(self.peer_params16) if j != self.r], path=self.path)
 
     def step(self, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), *, check: bool = False, tokens: Optional[int] = None,
              growth_interval: int = 0) -> None:
@@ -209,7 +212,7 @@ class Zero2Rank:
         zero_accumulate_grads(make_accum_args(
             self.P, self.R, grad_dtype=self.gcode, grads=self.peer_grads, accum=self.accum, scale=scale,
             first=first, rank_weights=weights, owner=self.r, workspace=self.workspace, ctrl=self.ctrl_buf,
-            accum_offset=self.state_offset), stream=self._s())
+            accum_offset=self.state_offset, path=self.path), stream=self._s())
         self._barrier()                                         # no rank still reads a gradient
 
     def step_accumulated(self, hp=(1e-3, 0.9, 0.999, 1e-8, 0.0), *, check: bool = False,
@@ -226,7 +229,7 @@ class Zero2Rank:
             grads=[self.accum], params16=self.params16, owner=self.r, hp=hp,
             check_nonfinite=2 if check else 0, growth_interval=growth_interval, state_offset=self.state_offset,
             push_params16=[t for j, t in enumerate(self.peer_params16) if j != self.r], n_grads=1,
-            grad_offset=self.state_offset)
+            grad_offset=self.state_offset, path=self.path)
         zero_step_fused(args, self._s())
         self._barrier()
 

@@ -42,7 +42,7 @@ int main(void) {
     printf("zero_step_args workspace %zu\n", offsetof(zero_step_args, workspace));
     printf("zero_step_args state_offset %zu\n", offsetof(zero_step_args, state_offset));
     printf("zero_step_args n_push %zu\n", offsetof(zero_step_args, n_push));
-    printf("zero_step_args reserved %zu\n", offsetof(zero_step_args, reserved));
+    printf("zero_step_args path %zu\n", offsetof(zero_step_args, path));
     printf("zero_step_args push_params16 %zu\n", offsetof(zero_step_args, push_params16));
     printf("zero_step_args n_grads %zu\n", offsetof(zero_step_args, n_grads));
     printf("zero_step_args reserved2 %zu\n", offsetof(zero_step_args, reserved2));

@@ -35,7 +35,7 @@ def test_struct_layouts_match_the_header():
     assert za.zero_ctrl_bytes() == ctypes.sizeof(za.zero_ctrl) == 40
     assert za.zero_workspace_bytes() == za.ZERO_WORKSPACE_BYTES == 256
     # zero_step_args: 5 ints + 2 host pointers + 8 device pointers + hparams + 2 ints + 2 pointers,
-    # then state_offset, n_push, reserved and the push array
+    # then state_offset, n_push, path and the push array
     assert ctypes.sizeof(za.zero_step_args) == 8 + 4 * 4 + 8 * 2 + 8 * 8 + 40 + 8 + 16 + 8 + 4 + 4 + 8 + 4 + 4 + 8
 
 
@@ -130,6 +130,9 @@ def _args(**over):
     (dict(push_params16=[A, A + 2]), za.ZERO_EALIGN),
     (dict(push_params16=[A, None]), za.ZERO_EINVAL),
     (dict(push_params16=[A]), za.ZERO_EINVAL),               # pushes need an owner
+    (dict(path=3), za.ZERO_EINVAL),                          # unknown kernel path
+    (dict(path=za.ZERO_PATH_STAGED, R=3, grads=[A] * 3), za.ZERO_EINVAL),   # no staged kernel for 3
+    (dict(path=za.ZERO_PATH_STAGED, n_grads=3), za.ZERO_EINVAL),
     (dict(n_grads=300), za.ZERO_ERANGE),
     (dict(n_grads=2, rank_weights=[1, -1]), za.ZERO_EINVAL),      # weights over the n_grads buffers
     (dict(grad_offset=4, owner=1), za.ZERO_EALIGN),

@@ -52,7 +52,7 @@ def _ranks(P, R, gdt, pdt, w0, S0):
     return out
 
 
-def _emulated_step(ranks, grads, P, R, gdt, pdt, check, wts):
+def _emulated_step(ranks, grads, P, R, gdt, pdt, check, wts, path=za.ZERO_PATH_AUTO):
     gcode, pcode = DTYPES[gdt][0], DTYPES[pdt][0]
     if check:
         for r, k in enumerate(ranks):
@@ -65,7 +65,7 @@ def _emulated_step(ranks, grads, P, R, gdt, pdt, check, wts):
                               exp_avg_sq=k.exp_avg_sq, ctrl=k.ctrl, workspace=k.ws, grads=grads,
                               params16=k.params16, rank_weights=wts, owner=r, hp=ADAMW_HP,
                               check_nonfinite=2 if check else 0, state_offset=k.off,
-                              push_params16=[o.params16 for j, o in enumerate(ranks) if j != r])
+                              push_params16=[o.params16 for j, o in enumerate(ranks) if j != r], path=path)
         za.zero_step_fused(a)
 
 
@@ -82,7 +82,8 @@ def _compare(ranks, ref):
         assert not k.ws.any()
 
 
-def _run(P, R, gdt="bf16", pdt="bf16", steps=3, check=False, S0=1.0, bad=(), token=False, seed=81):
+def _run(P, R, gdt="bf16", pdt="bf16", steps=3, check=False, S0=1.0, bad=(), token=False, seed=81,
+         path=za.ZERO_PATH_AUTO):
     ref = FlatZero(P, R, gdt, pdt, loss_scale=S0)
     w0 = synth.normal(P, 0.02, seed, device="cuda")
     ref.load_master(w0)
@@ -92,16 +93,22 @@ def _run(P, R, gdt="bf16", pdt="bf16", steps=3, check=False, S0=1.0, bad=(), tok
         if t in bad and P:
             ref.grads[t % R][(P * 2) // 3] = float("inf")
         wts = [float(x) for x in synth.token_counts(R, seed, t)] if token else None
-        _emulated_step(ranks, ref.grads, P, R, gdt, pdt, check, wts)
+        _emulated_step(ranks, ref.grads, P, R, gdt, pdt, check, wts, path)
         ref.step(hp=ADAMW_HP, check=check, rank_weights=wts)
     torch.cuda.synchronize()
     _compare(ranks, ref)
     return ref, ranks
 
 
+PATHS = [za.ZERO_PATH_AUTO, za.ZERO_PATH_REGISTER]
+
+
+@pytest.mark.parametrize("path", PATHS, ids=["staged", "plain-loads"])
 @pytest.mark.parametrize("R", [1, 2, 4, 8, 3])
-def test_emulated_ranks_equal_the_single_call_bitwise(R):
-    _run(P=200_003, R=R)
+def test_emulated_ranks_equal_the_single_call_bitwise(R, path):
+    # the owners' peer gradient reads by bulk copies (staged) or by plain
+    # loads (register kernel): both bitwise equal to the single staged call
+    _run(P=200_003, R=R, path=path)
 
 
 @pytest.mark.parametrize("R", [4, 8])
@@ -170,9 +177,10 @@ def test_emulated_ranks_small_and_empty_slices(P, R):
     _run(P=P, R=R, steps=2)
 
 
-def test_emulated_ranks_against_the_oracle():
+@pytest.mark.parametrize("path", PATHS, ids=["staged", "plain-loads"])
+def test_emulated_ranks_against_the_oracle(path):
     P, R = 30_011, 4
-    ref, ranks = _run(P=P, R=R, steps=2, seed=83)
+    ref, ranks = _run(P=P, R=R, steps=2, seed=83, path=path)
     # the single call was the reference above; pin the pair to the oracle too
     st = oracle.State.create(synth.normal(P, 0.02, 83, device="cuda").double().cpu().numpy())
     g = [torch.zeros(P, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
@@ -281,7 +289,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _ipc_worker(rank, world, port, P, q, tmp):
+def _ipc_worker(rank, world, port, P, q, tmp, path):
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -294,7 +302,7 @@ def _ipc_worker(rank, world, port, P, q, tmp):
                             timeout=datetime.timedelta(seconds=60))
     status = "ok"
     try:
-        z = Zero2Rank(P, "bf16", "bf16")
+        z = Zero2Rank(P, "bf16", "bf16", path=path)
         w0 = sy.normal(P, 0.02, 91, device="cuda")
         z.load_master(w0)
         everyone = [torch.zeros(P, dtype=torch.bfloat16, device="cuda") for _ in range(world)]
@@ -368,11 +376,13 @@ def _ipc_worker(rank, world, port, P, q, tmp):
         dist.destroy_process_group()
 
 
-def test_two_processes_share_one_gpu_through_cuda_ipc(tmp_path):
+@pytest.mark.parametrize("path", PATHS, ids=["staged", "plain-loads"])
+def test_two_processes_share_one_gpu_through_cuda_ipc(tmp_path, path):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_ipc_worker, args=(r, 2, port, 100_003, q, str(tmp_path))) for r in range(2)]
+    procs = [ctx.Process(target=_ipc_worker, args=(r, 2, port, 100_003, q, str(tmp_path), path))
+             for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
