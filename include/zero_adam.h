@@ -69,6 +69,11 @@ extern "C" {
 /* Largest number of logical ranks one step call accepts. */
 #define ZERO_MAX_RANKS 256
 
+/* Largest parameter count P of a step or accumulation call (2^40, far beyond
+ * one GPU's memory): beyond it the calls return ZERO_ERANGE, so the kernels'
+ * 32-bit tile numbers cannot wrap. */
+#define ZERO_MAX_ELEMENTS 1099511627776ull /* 2^40 */
+
 /* Bytes of the scratch workspace every step call needs (see zero_step_args). */
 #define ZERO_WORKSPACE_BYTES 256
 
@@ -348,8 +353,8 @@ int zero_selftest_wait_timeout(void *ctrl, void *stream);
  * The step kernel is the one args->path selects; ZERO_PATH_STAGED with a
  * gradient-buffer count other than 1, 2, 4 or 8, or an unknown path, is
  * ZERO_EINVAL.
- * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ERANGE (R > ZERO_MAX_RANKS),
- * ZERO_EOVERFLOW (P*4 bytes overflow), ZERO_ECUDA. */
+ * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ERANGE (R > ZERO_MAX_RANKS, or
+ * P > ZERO_MAX_ELEMENTS), ZERO_EOVERFLOW (P*8 bytes overflow), ZERO_ECUDA. */
 int zero_step_fused(const zero_step_args *args, void *stream);
 
 /* The same step over a tensor list: args->grads and args->params16 must be
@@ -456,7 +461,8 @@ typedef struct zero_accum_args {
  * ZERO_EINVAL (also: exactly one of workspace and ctrl given; an unknown
  * path; ZERO_PATH_STAGED without a workspace or with another R),
  * ZERO_EALIGN (accum, grads and workspace must be 16-byte aligned, ctrl
- * 8-byte aligned), ZERO_ERANGE, ZERO_EOVERFLOW, ZERO_ECUDA. */
+ * 8-byte aligned), ZERO_ERANGE (R > ZERO_MAX_RANKS, P > ZERO_MAX_ELEMENTS),
+ * ZERO_EOVERFLOW, ZERO_ECUDA. */
 int zero_accumulate_grads(const zero_accum_args *args, void *stream);
 
 /* ------------------------------------------------------------------ ZeRO-3 */

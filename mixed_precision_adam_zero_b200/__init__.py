@@ -33,6 +33,7 @@ ZERO_BF16 = 1
 ZERO_F16 = 2
 
 ZERO_MAX_RANKS = 256
+ZERO_MAX_ELEMENTS = 1 << 40
 ZERO_WORKSPACE_BYTES = 256
 ZERO_NOALLOC_SCRATCH_BYTES = 256
 ZERO_PATH_AUTO, ZERO_PATH_REGISTER, ZERO_PATH_STAGED = 0, 1, 2

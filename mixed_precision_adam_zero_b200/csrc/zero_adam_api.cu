@@ -92,10 +92,25 @@ Shape make_shape(uint64_t lo, uint64_t hi, int max_ctas) {
     return s;
 }
 
+// Every kernel is launched with programmatic stream serialization: it may
+// start while the kernel before it in the stream finishes, and waits for
+// that kernel's completion (griddepcontrol.wait) before it touches global
+// memory, so the launch latency and its prologue overlap the earlier
+// kernel's tail.
 int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st, unsigned smem = 0,
            int threads = kThreads) {
     void* args[] = {params};
-    const cudaError_t e = cudaLaunchKernel(fn, dim3(sh.grid), dim3(threads), args, smem, st);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sh.grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelExC(&cfg, fn, args);
     if (e != cudaSuccess) return zadam_record_cuda(e);
     return ZERO_OK;
 }
@@ -234,6 +249,7 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     if (a->n_grads > ZERO_MAX_RANKS) return ZERO_ERANGE;
     if (a->reserved2 != 0u || (a->grad_offset != 0 && a->check_nonfinite == 1)) return ZERO_EINVAL;
     if (a->P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
+    if (a->P > ZERO_MAX_ELEMENTS) return ZERO_ERANGE;
     int rc = check_hparams(a->hp);
     if (rc) return rc;
     if (a->ctrl == nullptr || a->workspace == nullptr) return ZERO_EINVAL;
@@ -581,6 +597,7 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     if (!is_grad_dtype(a->grad_dtype) || (a->first != 0 && a->first != 1)) return ZERO_EINVAL;
     if (!std::isfinite(a->scale)) return ZERO_EINVAL;
     if (a->P > (UINT64_MAX >> 3)) return ZERO_EOVERFLOW;
+    if (a->P > ZERO_MAX_ELEMENTS) return ZERO_ERANGE;
     if (a->P > 0 && a->accum == nullptr) return ZERO_EINVAL;
     if (!aligned16(a->accum)) return ZERO_EALIGN;
     if ((a->workspace == nullptr) != (a->ctrl == nullptr)) return ZERO_EINVAL;

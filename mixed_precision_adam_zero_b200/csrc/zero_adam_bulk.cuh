@@ -347,11 +347,13 @@ __device__ __forceinline__ StateIO state_io(const StepParams& p) {
 }
 
 // Flat calls: tiles are handed out dynamically.  The launch's vector body
-// [va, vb) is cut into kTile-element tiles.  CTA b starts on tile b without
-// asking anyone; after that each CTA's producer claims the next tile from a
-// counter in the workspace (claims number the tiles from gridDim.x on), one
-// claim ahead of use so the atomic's latency overlaps the copies.  All CTAs then finish within
-// about one tile of each other, whatever the speed of their SM.  The tile id
+// [va, vb) is cut into kTile-element tiles.  CTA b fills its ring with tiles
+// b, b + G, ..., b + (D-1) G (G CTAs, D stages) without asking anyone, so
+// every stage's copies are in flight at once from the start; after that each
+// CTA's producer claims the next tile from a counter in the workspace
+// (claims number the tiles from D*G on), one claim ahead of use so the
+// atomic's latency overlaps the copies.  All CTAs then finish within about
+// one tile of each other, whatever the speed of their SM.  The tile id
 // travels to the consumers in a per-stage slot, written before the stage's
 // barrier is armed; kEndTile marks the end.
 constexpr uint32_t kEndTile = 0xFFFFFFFFu;
@@ -366,7 +368,8 @@ template <int D, class Issue>
 __device__ __forceinline__ void flat_produce(Workspace* ws, uint64_t va, uint64_t vb, uint64_t* full,
                                              uint64_t* empty, uint32_t* slot, Issue&& issue) {
     const uint32_t ntiles = flat_tile_count(va, vb);
-    uint32_t next = blockIdx.x;
+    const uint32_t first_claimed = (uint32_t)D * gridDim.x;
+    uint32_t next = 0;
     uint32_t k = 0;
     bool ok = true;
     for (;; ++k) {
@@ -375,13 +378,14 @@ __device__ __forceinline__ void flat_produce(Workspace* ws, uint64_t va, uint64_
             ok = false;
             break;
         }
-        const uint32_t tile = next;
+        // ntiles <= 2^29 (the host refuses more than ZERO_MAX_ELEMENTS), so no tile id here wraps
+        const uint32_t tile = k < (uint32_t)D ? blockIdx.x + k * gridDim.x : next;
         if (tile >= ntiles) {
             slot[st] = kEndTile;
             mbar_arrive(&full[st]);
             break;
         }
-        next = gridDim.x + atomicAdd(&ws->next_tile, 1u);
+        if (k + 1u >= (uint32_t)D) next = first_claimed + atomicAdd(&ws->next_tile, 1u);
         slot[st] = tile;
         const uint64_t e0 = va + (uint64_t)tile * kTile;
         const uint32_t n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
@@ -416,6 +420,27 @@ __device__ __forceinline__ void flat_consume(Workspace* ws, uint64_t va, uint64_
     }
 }
 
+// The ragged ends of a flat launch, [lo, va) and [vb, hi) outside the vector
+// body (at most 7 elements each), one element per lane: lanes `lane` of
+// `nlanes` >= 14.
+template <class G, class Pm, int RC, bool PUSH>
+__device__ __forceinline__ void flat_ends(const StepParams& p, const Scal& s, const StateIO& io, uint32_t lane,
+                                          bool& bad) {
+    uint64_t va = (p.lo + 7) & ~7ull, vb = p.hi & ~7ull;
+    if (va > p.hi) va = p.hi;
+    if (vb < va) vb = va;
+    const uint64_t nhead = va - p.lo, ntail = p.hi - vb;
+    uint64_t e;
+    if (lane < nhead) e = p.lo + lane;
+    else if (lane - nhead < ntail) e = vb + (lane - nhead);
+    else return;
+    const GradPtrs<G, RC> gp(&p.grads[0]);
+    elem_step<G, Pm, RC, PUSH>(p, s, gp, static_cast<Pm*>(p.params16), e, e, io, bad);
+}
+
+// Flat step over [lo, hi): the producer thread, the consumer warps, and --
+// in the last CTA, while its ring fills -- the producer warp's other 31
+// lanes on the ragged ends, so they cost the launch no time at its end.
 template <class G, class Pm, int RC, bool PUSH = false>
 __device__ __forceinline__ void flat_dynamic(const StepParams& p, uint64_t* full, uint64_t* empty,
                                              uint32_t* slot, unsigned char* ring, bool& bad) {
@@ -440,6 +465,10 @@ __device__ __forceinline__ void flat_dynamic(const StepParams& p, uint64_t* full
             for (uint32_t q = 4u * threadIdx.x; q < n; q += 4u * kConsumers)
                 bulk_group<G, Pm, RC, PUSH>(p, s, stage, q, e0 + q, e0 + q, io.wo, io.mo, io.vo, pp, bad);
         });
+    } else if (blockIdx.x == gridDim.x - 1) {
+        const StateIO io = state_io(p);
+        const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
+        flat_ends<G, Pm, RC, PUSH>(p, s, io, threadIdx.x - kConsumers - 1u, bad);
     }
 }
 
@@ -457,9 +486,9 @@ struct TileDesc {
 // take the vector path) is [offs[j], round_down(offs[j+1], 8)); the bodies
 // are cut into kTile tiles, numbered across tensors (tab.tiles holds the
 // running count), and handed out dynamically like the flat call's tiles.
-// As for flat calls, CTA b starts on tile b and claims the rest.  Tile ids
-// a producer gets only grow, so it finds each tile's tensor by scanning
-// forward from the previous one.
+// As for flat calls, CTA b fills its ring with tiles b, b + G, ... and
+// claims the rest.  Tile ids a producer gets only grow, so it finds each
+// tile's tensor by scanning forward from the previous one.
 template <class G, class Pm, int RC>
 __device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full, uint64_t* empty,
                                              TileDesc* desc, unsigned char* ring, bool& bad) {
@@ -474,8 +503,9 @@ __device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full
         uint32_t jn = 0;           // scan position
         uint64_t t0 = 0, bb = 0, tfirst = 0;
         void* params = nullptr;
-        uint64_t next = blockIdx.x;
-        if (next < ntiles) jn = find_tensor_by_tile(t, next);
+        const uint64_t first_claimed = (uint64_t)D * gridDim.x;
+        uint64_t next = 0;
+        if (blockIdx.x < ntiles) jn = find_tensor_by_tile(t, blockIdx.x);
         uint32_t k = 0;
         bool ok = true;
         for (;; ++k) {
@@ -484,13 +514,13 @@ __device__ __forceinline__ void list_dynamic(const StepParams& p, uint64_t* full
                 ok = false;
                 break;
             }
-            const uint64_t tile = next;
+            const uint64_t tile = k < (uint32_t)D ? (uint64_t)blockIdx.x + (uint64_t)k * gridDim.x : next;
             if (tile >= ntiles) {
                 desc[st] = TileDesc{0ull, 0ull, nullptr, 0u, 0u};
                 mbar_arrive(&full[st]);
                 break;
             }
-            next = (uint64_t)gridDim.x + atomicAdd(&p.ws->next_tile, 1u);
+            if (k + 1u >= (uint32_t)D) next = first_claimed + atomicAdd(&p.ws->next_tile, 1u);
             while (t.tiles[jn + 1] <= tile) ++jn;
             if (jn != j) {
                 j = jn;
@@ -630,46 +660,51 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
     const void** s_gp = reinterpret_cast<const void**>(smem + kBarBytes);
     unsigned char* ring = smem + kBarBytes + kGpBytes;
 
+    __shared__ StepStart s_start;
     uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
     uint64_t b = a + p.chunk;
     if (a < p.lo) a = p.lo;
     if (b > p.hi) b = p.hi;
-    if (threadIdx.x == 0) s_timed_out = 0u;
-    bool skip = false;
-    if (p.check == 2) skip = *reinterpret_cast<volatile const unsigned*>(&p.ws->found) != 0u;
-    bool bad = false;
     const bool work = (LIST && !p.whole) ? a < b : p.lo < p.hi;
-    if (!skip && work) {
-        if (threadIdx.x == 0) {
+    // shared memory only until the wait: overlaps the earlier kernel's tail
+    if (threadIdx.x == 0) {
+        s_timed_out = 0u;
+        if (work) {
             for (int i = 0; i < D; ++i) {
                 mbar_init(&full[i], 1u);
                 mbar_init(&empty[i], kConsumerWarps);
             }
             fence_mbar_init();
         }
+    }
+    grid_dependency_wait();
+    allow_dependents();
+    bool skip = false;
+    if (p.check == 2) skip = *reinterpret_cast<volatile const unsigned*>(&p.ws->found) != 0u;
+    bool bad = false;
+    if (!skip && work) {
         __syncthreads();
+        // the epilogue's inputs, loaded while the first tiles are in flight
+        if (threadIdx.x == 0) s_start = StepStart{*p.ctrl, p.ws->found};
         if constexpr (LIST) {
             if (p.whole) list_dynamic<G, Pm, RC>(p, full, empty, reinterpret_cast<TileDesc*>(slot), ring, bad);
             else list_static<G, Pm, RC>(p, a, b, full, empty, ring, bad);
-        } else {
-            flat_dynamic<G, Pm, RC, PUSH>(p, full, empty, slot, ring, bad);
-        }
-        __syncthreads();
-        // Ragged heads and tails, and tensors that cannot take the vector path
-        // (flat: the launch's ragged ends, on the first CTA only).
-        const StateIO io = state_io(p);
-        const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
-        if constexpr (LIST) {
+            __syncthreads();
+            // Ragged heads and tails, and tensors that cannot take the vector path.
+            const StateIO io = state_io(p);
+            const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
             if (p.whole) {
                 if (a < b) list_scalar_whole<G, Pm, RC>(p, s, a, b, io, bad, s_gp);
             } else {
                 if (a < b) bulk_scalar_pass<G, Pm, RC, true>(p, s, a, b, io, bad, s_gp);
             }
-        } else if (blockIdx.x == 0) {
-            bulk_scalar_pass<G, Pm, RC, false, PUSH>(p, s, p.lo, p.hi, io, bad, s_gp);
+        } else {
+            flat_dynamic<G, Pm, RC, PUSH>(p, full, empty, slot, ring, bad);
         }
+    } else if (threadIdx.x == 0) {
+        s_start = StepStart{*p.ctrl, p.ws->found};
     }
-    finish_step<PUSH>(p, bad, s_timed_out != 0u);
+    finish_step<PUSH>(p, bad, s_timed_out != 0u, &s_start);
 }
 
 // ------------------------------------------------------------ micro-step accumulation
@@ -753,6 +788,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) accum_bulk_kernel(const __gri
         }
         fence_mbar_init();
     }
+    grid_dependency_wait();
+    allow_dependents();
     __syncthreads();
     const uint64_t va = (p.lo + 7) & ~7ull;
     const uint64_t vb = p.hi & ~7ull;
@@ -794,12 +831,17 @@ __global__ void __launch_bounds__(kBulkThreads, 1) accum_bulk_kernel(const __gri
 // wait gave up: device_error set, the step not applied.
 __global__ void wait_timeout_probe_kernel(zero_ctrl* c) {
     __shared__ __align__(8) uint64_t bar;
+    grid_dependency_wait();
+    allow_dependents();
     if (threadIdx.x == 0) {
         mbar_init(&bar, 1u);
         fence_mbar_init();
         // growth_interval 1: a step wrongly counted as applied would also
         // double the loss scale, which the health check's caller can see.
-        if (!mbar_wait_bounded(&bar, 0u)) ctrl_after_step(c, false, true, true, 1, 1u);
+        if (!mbar_wait_bounded(&bar, 0u)) {
+            const zero_ctrl c0 = *c;
+            ctrl_after_step(c0, c, false, true, true, 1, 1u);
+        }
     }
 }
 

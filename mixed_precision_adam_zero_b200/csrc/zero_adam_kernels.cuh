@@ -73,6 +73,15 @@ struct Arrival {
     }
 };
 
+// Programmatic dependent launch.  Every kernel the library launches is
+// launched so that it may start while the kernel before it in the stream is
+// still finishing (its CTAs take each SM as the earlier CTAs leave it), and
+// each kernel first waits, with grid_dependency_wait, until that kernel has
+// completed and its memory is visible, before its first access to global
+// memory; it then lets the kernel after it start early the same way.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 struct Hyper {
     float b1, b2, omb1, omb2, eps, lr_wd;  // float32 per-element constants
     double lr, b1d, b2d;                   // float64, for the bias corrections
@@ -445,7 +454,9 @@ __device__ __forceinline__ uint32_t find_tensor_by_tile(const Table& t, uint64_t
     return lo;
 }
 
-// The control block after one step call (one thread, once per call).
+// The control block after one step call (one thread, once per call), from
+// c0, its contents when the call started (no other code writes it during a
+// call).
 //   found:   an inf/NaN was seen -> skipped: S halves, t and the set stay;
 //   timeout: a bounded wait of some CTA gave up, so part of the output was
 //            never written -> not applied either (t and parity stay, so a
@@ -454,24 +465,24 @@ __device__ __forceinline__ uint32_t find_tensor_by_tile(const Table& t, uint64_t
 //            growth count stay as they were, and device_error is set;
 //   else:    applied: t += 1, the set flips (two-set mode), and with the
 //            check on S doubles after growth_interval applied steps in a row.
-__device__ __forceinline__ void ctrl_after_step(zero_ctrl* c, bool found, bool timeout, bool two_set, int check,
-                                                uint32_t growth_interval) {
+__device__ __forceinline__ void ctrl_after_step(const zero_ctrl& c0, zero_ctrl* c, bool found, bool timeout,
+                                                bool two_set, int check, uint32_t growth_interval) {
     if (timeout) {
         c->device_error = 1u;
         c->last_skipped = 1u;
     } else if (found) {
-        c->loss_scale *= 0.5f;
+        c->loss_scale = c0.loss_scale * 0.5f;
         c->growth_tracker = 0u;
-        c->skipped += 1ull;
+        c->skipped = c0.skipped + 1ull;
         c->last_skipped = 1u;
     } else {
-        c->step += 1ull;
+        c->step = c0.step + 1ull;
         c->last_skipped = 0u;
-        if (two_set) c->parity ^= 1u;
+        if (two_set) c->parity = c0.parity ^ 1u;
         if (check) {
-            uint32_t gt = c->growth_tracker + 1u;
+            uint32_t gt = c0.growth_tracker + 1u;
             if (growth_interval != 0u && gt >= growth_interval) {
-                c->loss_scale *= 2.0f;
+                c->loss_scale = c0.loss_scale * 2.0f;
                 gt = 0u;
             }
             c->growth_tracker = gt;
@@ -479,24 +490,44 @@ __device__ __forceinline__ void ctrl_after_step(zero_ctrl* c, bool found, bool t
     }
 }
 
+// What a step launch knew of its control block and workspace when it
+// started: the control block, and (mode 2) the inf/NaN word of the scans
+// that ran before it.
+struct StepStart {
+    zero_ctrl ctrl;
+    unsigned int found;
+};
+
 // Grid-level epilogue: the last CTA to finish updates the control block and
 // clears the workspace for the next launch.  Every other access to the
 // control block and the workspace in this launch happened before the
 // accessing CTA's arrival, and the next launch sees the writes at the kernel
-// boundary.  Only thread 0's `timed_out` is used.
-template <bool PUSH = false>
-__device__ __forceinline__ void finish_step(const StepParams& p, bool bad, bool timed_out = false) {
-    // Stores into other GPUs' parameter buffers are performed before the CTA
-    // completes, whatever orders the peers' next reads after this kernel.
-    if constexpr (PUSH) __threadfence_system();
+// boundary.  Only thread 0's `timed_out` is used.  `start`: the launch's
+// start record in shared memory (written before the CTA's first barrier), or
+// null to read the control block and the word here.
+template <bool PUSH>
+__device__ __forceinline__ void finish_step(const StepParams& p, bool bad, bool timed_out = false,
+                                            const StepStart* start = nullptr) {
+    // PUSH: no fence for the stores into other GPUs' replicas.  Nothing in
+    // the kernel signals a peer; the peers read their replicas only after
+    // this kernel has completed (its stores are then performed) and a
+    // collective barrier that follows it on the stream.
     const int any = __syncthreads_or(bad ? 1 : 0);
     if (threadIdx.x == 0) {
         Workspace* ws = p.ws;
         const unsigned long long mine = Arrival::mine(any != 0, timed_out);
         const unsigned long long all = atomicAdd(&ws->arrive, mine) + mine;
         if (Arrival::count(all) == gridDim.x) {
-            const bool found = p.check == 1 ? Arrival::any_found(all) : (p.check == 2 && ws->found != 0u);
-            ctrl_after_step(p.ctrl, found, Arrival::any_timeout(all), p.two_set != 0, p.check, p.growth_interval);
+            StepStart s0;
+            if (start != nullptr) {
+                s0 = *start;
+            } else {
+                s0.ctrl = *p.ctrl;
+                s0.found = ws->found;
+            }
+            const bool found = p.check == 1 ? Arrival::any_found(all) : (p.check == 2 && s0.found != 0u);
+            ctrl_after_step(s0.ctrl, p.ctrl, found, Arrival::any_timeout(all), p.two_set != 0, p.check,
+                            p.growth_interval);
             ws->found = 0u;
             ws->next_tile = 0u;
             ws->arrive = 0ull;
@@ -507,6 +538,8 @@ __device__ __forceinline__ void finish_step(const StepParams& p, bool bad, bool 
 template <class G, class Pm, int RC, bool LIST, bool PUSH = false>
 __global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ StepParams p) {
     __shared__ const void* s_gp[LIST ? ZERO_MAX_RANKS : 1];
+    grid_dependency_wait();
+    allow_dependents();
     const zero_ctrl* c = p.ctrl;
     const uint32_t par = p.two_set ? c->parity : 0u;
     const uint32_t out = par ^ (uint32_t)p.two_set;
@@ -574,6 +607,8 @@ __device__ __forceinline__ void scan_range(const G* g, uint64_t a, uint64_t b, b
 // Sets ws.found if any gradient of any rank in [lo, hi) is inf or NaN.
 template <class G, bool LIST>
 __global__ void __launch_bounds__(kThreads) scan_kernel(const __grid_constant__ StepParams p) {
+    grid_dependency_wait();
+    allow_dependents();
     uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
     uint64_t b = a + p.chunk;
     if (a < p.lo) a = p.lo;
@@ -631,6 +666,8 @@ __device__ __forceinline__ void cast_range(const float* w, Pm* pp, uint64_t toff
 
 template <class Pm, bool LIST>
 __global__ void __launch_bounds__(kThreads) gather_kernel(const __grid_constant__ GatherParams p) {
+    grid_dependency_wait();
+    allow_dependents();
     if (p.only_if_skipped && p.ctrl->last_skipped == 0u) return;
     const float* w = p.ctrl != nullptr ? p.w[p.ctrl->parity & 1u] : p.w[0];
     uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
@@ -716,6 +753,8 @@ constexpr uint64_t kZ3Chunk = 32768;
 template <class Pm>
 __global__ void __launch_bounds__(kThreads) z3_gather_kernel(const __grid_constant__ Z3Params p) {
     __shared__ uint64_t s_next;
+    grid_dependency_wait();
+    allow_dependents();
     unsigned int* sc = p.tab.scratch;
     const uint64_t nchunks = (p.hi + kZ3Chunk - 1) / kZ3Chunk;
     uint64_t c = blockIdx.x;
@@ -824,6 +863,8 @@ __device__ __forceinline__ void accum_elem(const AccumParams& p, const GradPtrs<
 
 template <class G, int RC>
 __global__ void __launch_bounds__(kThreads) accum_kernel(const __grid_constant__ AccumParams p) {
+    grid_dependency_wait();
+    allow_dependents();
     uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
     uint64_t b = a + p.chunk;
     if (a < p.lo) a = p.lo;

@@ -121,6 +121,7 @@ def _args(**over):
     (dict(rank_weights=[1, float("nan"), 1, 1]), za.ZERO_EINVAL),
     (dict(master2=A), za.ZERO_EINVAL),          # second set incomplete
     (dict(P=2**62), za.ZERO_EOVERFLOW),
+    (dict(P=2**40 + 1), za.ZERO_ERANGE),                     # beyond ZERO_MAX_ELEMENTS
     (dict(check_nonfinite=True, reduced_out=A + 4), za.ZERO_EALIGN),
     (dict(check_nonfinite=3), za.ZERO_EINVAL),
     (dict(state_offset=4, owner=1), za.ZERO_EALIGN),         # not a multiple of 8
@@ -256,6 +257,7 @@ def test_pushes_need_an_owner():
     (dict(grads=[A, A + 2, A, A]), za.ZERO_EALIGN),
     (dict(rank_weights=[1, 1, -1, 1]), za.ZERO_EINVAL),
     (dict(P=2**62), za.ZERO_EOVERFLOW),
+    (dict(P=2**40 + 1), za.ZERO_ERANGE),                     # beyond ZERO_MAX_ELEMENTS
     (dict(workspace=A), za.ZERO_EINVAL),            # a workspace needs a ctrl
     (dict(ctrl=A), za.ZERO_EINVAL),                 # and a ctrl a workspace
     (dict(workspace=A + 8, ctrl=A), za.ZERO_EALIGN),
