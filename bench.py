@@ -400,7 +400,7 @@ def build_workload(name: str, device, stream, world: int = 1) -> Bench:
                  keep=(z, step_args))
 
 
-def roofline_kernel(workload: str) -> str:
+def roofline_kernel(workload: str, world: int = 1) -> str:
     """The kernel (or, for accumulation, the launch sequence of one step) the
     roofline fraction is measured on."""
     kind, size, R, gdt, pdt, scaled = WORKLOADS[workload]
@@ -409,6 +409,8 @@ def roofline_kernel(workload: str) -> str:
     if kind == "zero2emu":
         return f"{R} x step_bulk_kernel (flat, push): the owners of an emulated {R}-rank ZeRO-2 step"
     if kind == "zero2":
+        if world == 1:
+            return "step_bulk_kernel (flat, owner 0 of 1, no peers): the ZeRO-2 step on one GPU"
         return "step_bulk_kernel (flat, push): this GPU's owner kernel of the ZeRO-2 step across GPUs"
     step = ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") + (" (flat)" if kind == "flat" else " (list)")
     gas = GAS.get(workload, 0)
@@ -430,7 +432,7 @@ def roofline(workload: str, world: int, P: int, launch_ms: float, peaks: dict, t
         achieved = b / (launch_ms * 1e-3) / 1e9
         return {"bound": "nvlink", "achieved": achieved, "peak": NVLINK_GBS, "unit": "GB/s",
                 "frac": achieved / NVLINK_GBS, "peak_source": "pool's measured peer copy per direction",
-                "traffic": None, "kernel": roofline_kernel(workload), "bytes_per_launch": b,
+                "traffic": None, "kernel": roofline_kernel(workload, world), "bytes_per_launch": b,
                 "launch_ms": launch_ms}
     bpp = workload_bpp(workload, world) if kind != "zero2" else bytes_per_param(1, "bf16")
     peak = peaks.get("hbm_gbs")
@@ -441,7 +443,7 @@ def roofline(workload: str, world: int, P: int, launch_ms: float, peaks: dict, t
             "peak_source": f"{src} hbm_gbs", "traffic": traffic,
             # the ncu-measured DRAM bytes of one launch over the live launch time
             "traffic_gbs": traffic / (launch_ms * 1e-3) / 1e9 if traffic else None,
-            "kernel": roofline_kernel(workload), "bytes_per_launch": bpp * P, "launch_ms": launch_ms}
+            "kernel": roofline_kernel(workload, world), "bytes_per_launch": bpp * P, "launch_ms": launch_ms}
 
 
 # ------------------------------------------------------------ ranks
@@ -486,7 +488,18 @@ def zero2_throughput(P: int, steps: int, max_ms: float) -> float:
 
 # ------------------------------------------------------------ arms
 
+def json_stdout():
+    """The process's stdout, reserved for the one JSON line: file descriptor
+    1 is pointed at stderr from here on, so that libraries which print to
+    stdout (NCCL's version banner, for one) cannot add lines to it."""
+    sys.stdout.flush()
+    out = os.fdopen(os.dup(1), "w")
+    os.dup2(2, 1)
+    return out
+
+
 def run_gpu(args) -> None:
+    out = json_stdout()
     import torch
     import torch.distributed as dist
     from datetime import timedelta
@@ -622,7 +635,7 @@ def run_gpu(args) -> None:
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
-        print(json.dumps(line), flush=True)
+        print(json.dumps(line), file=out, flush=True)
     if world > 1 or kind == "zero2":
         del b
         torch.cuda.synchronize()

@@ -108,3 +108,16 @@ def test_roofline_arithmetic():
     assert rf["traffic"] == 1234
     fb = bench.roofline("flat16m", 1, 16_777_259, 0.1, {}, None)
     assert fb["peak_source"] == "fallback hbm_gbs" and fb["peak"] == 6650.0
+
+
+def test_stdout_carries_only_the_json_line():
+    """What libraries print to file descriptor 1 (NCCL's banner, for one) goes
+    to stderr once the GPU arm has reserved stdout for its line."""
+    import subprocess
+    code = ("import os, sys; sys.path.insert(0, %r); import bench; out = bench.json_stdout(); "
+            "print('python noise'); os.write(1, b'library noise\\n'); print('{\"value\": 1}', file=out, flush=True)"
+            % ROOT)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout == '{"value": 1}\n'
+    assert "python noise" in r.stderr and "library noise" in r.stderr
