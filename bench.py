@@ -509,8 +509,12 @@ def run_gpu(args) -> None:
     device = torch.device("cuda", local)
     kind = WORKLOADS[args.workload][0]
     if world > 1 or kind == "zero2":
+        if world == 1 and "MASTER_PORT" not in os.environ:   # a one-process group: any free local port
+            import socket
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                os.environ["MASTER_PORT"] = str(sk.getsockname()[1])
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        os.environ.setdefault("MASTER_PORT", "29531")
         os.environ.setdefault("RANK", "0")
         os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
