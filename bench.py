@@ -94,8 +94,10 @@ WORKLOADS["gpt2m_z3gather"] = ("z3gather", "gpt2m", 4, "bf16", "bf16", False)
 # its own state slice, reading every rank's gradient slice and storing its
 # 16-bit results into all R replicas (the pushes land in this GPU's HBM).
 WORKLOADS["flat16m_zero2emu"] = ("zero2emu", 16_777_259, 8, "bf16", "bf16", False)
-# The ZeRO-2 step across GPUs, one process per GPU (R = 0: the world size).
+# The ZeRO-2 step across GPUs, one process per GPU (R = 0: the world size),
+# over the 3.2B flat vector, and a 16.8M-parameter case of the same path.
 WORKLOADS["zero2"] = ("zero2", LLAMA3B_P, 0, "bf16", "bf16", False)
+WORKLOADS["zero2_16m"] = ("zero2", 16_777_259, 0, "bf16", "bf16", False)
 
 
 def bytes_per_param(R: int, gdt: str, gas: int = 0) -> int:

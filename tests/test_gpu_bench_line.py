@@ -63,3 +63,26 @@ def test_bench_line_default_is_the_3p2b_llama_list():
     d = _run("--steps", "5", "--warmup", "3", "--cpu-seconds", "1")
     _check_line(d, "llama3b", 3_212_749_824, 8, 5, 3, 2)
     assert d["config"]["tensors"] == 254
+
+
+def test_bench_line_zero2_mode_on_one_gpu():
+    """The path bench.py takes under torchrun (the ZeRO-2 step across GPUs,
+    one Zero2Rank per process, an NCCL group), here with one process: R = 1,
+    owner 0 of 1; stdout carries exactly the one JSON line although NCCL
+    initialises."""
+    torch.cuda.empty_cache()
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "zero2_16m", "--steps", "10",
+                        "--warmup", "3", "--e2e-steps", "1", "--cpu-seconds", "1"], capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = r.stdout.strip().splitlines()
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    P = 16_777_259
+    assert d["config"]["workload"] == "zero2_16m" and d["config"]["R"] == 1 and d["config"]["P"] == P
+    assert d["scaling"] == "strong" and d["n_gpus"] == 1
+    assert d["value"] == pytest.approx(P / (d["ms_per_step"] * 1e-3), rel=1e-9)
+    rf = d["roofline"]
+    assert rf["bound"] == "hbm" and rf["bytes_per_launch"] == 28 * P and "no peers" in rf["kernel"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 2 * P and d["e2e"]["d2h_bytes_per_step"] == 2 * P
+    assert d["applied_steps"] == 10 + 3 + 1 + 1 and d["gpu_launches"] == 10
