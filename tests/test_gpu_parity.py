@@ -198,3 +198,58 @@ def test_gather_params_is_rne_of_the_masters(pdt):
     assert torch.equal(out.view(torch.int16), w.to(dt).view(torch.int16))
     ob = oracle.rne16(w.double().cpu().numpy(), pdt)
     assert np.array_equal(out.view(torch.int16).cpu().numpy().view(np.uint16), ob)
+
+
+def _same_bits(a: torch.Tensor, b: torch.Tensor) -> bool:
+    return torch.equal(a.view(torch.int32 if a.element_size() == 4 else torch.int16),
+                       b.view(torch.int32 if b.element_size() == 4 else torch.int16))
+
+
+@pytest.mark.parametrize("gdt,pdt", [("bf16", "bf16"), ("f16", "f16"), ("f32", "bf16"), ("bf16", "f16")])
+@pytest.mark.parametrize("R", [1, 2, 4, 8])
+def test_register_and_staged_kernels_agree_bitwise_flat(gdt, pdt, R):
+    """The two step kernels of a compile-time rank count -- bulk copies into
+    shared memory (ZERO_PATH_STAGED) and plain loads into registers
+    (ZERO_PATH_REGISTER) -- give the same bits, token weights and the
+    in-pass overflow check included, on a size with ragged ends."""
+    import mixed_precision_adam_zero_b200 as za
+    P = 100_003
+    zs, zr = FlatZero(P, R, gdt, pdt, two_set=True), FlatZero(P, R, gdt, pdt, two_set=True)
+    w0 = synth.normal(P, 0.02, 61, device="cuda")
+    zs.load_master(w0)
+    zr.load_master(w0)
+    for k in range(1, 4):
+        grads_for_step(61, k, zs.grads, 1e-3)
+        for a, b in zip(zr.grads, zs.grads):
+            a.copy_(b)
+        wts = _weights(R, k, token=True)
+        zs.step(hp=ADAMW_HP, rank_weights=wts, check=True, path=za.ZERO_PATH_STAGED)
+        zr.step(hp=ADAMW_HP, rank_weights=wts, check=True, path=za.ZERO_PATH_REGISTER)
+    torch.cuda.synchronize()
+    for a, b in zip(zs.current(), zr.current()):
+        assert _same_bits(a, b)
+    assert _same_bits(zs.params16, zr.params16)
+    assert zs.ctrl().step == zr.ctrl().step == 3
+
+
+@pytest.mark.parametrize("R", [4, 8])
+def test_register_and_staged_kernels_agree_bitwise_list(R):
+    """The same for tensor lists (ragged and misaligned tensors included)."""
+    import mixed_precision_adam_zero_b200 as za
+    numels = [4096, 1000, 37, 8192 * 3 + 5, 1024, 9]
+    zs, zr = ListZero(numels, R, "bf16", "bf16"), ListZero(numels, R, "bf16", "bf16")
+    w0 = synth.normal(sum(numels), 0.02, 63, device="cuda")
+    zs.load_master(w0)
+    zr.load_master(w0)
+    for k in range(1, 4):
+        grads_for_step(63, k, zs.grads, 1e-3)
+        for a, b in zip(zr.grads, zs.grads):
+            for x, y in zip(a, b):
+                x.copy_(y)
+        zs.step(hp=ADAMW_HP, path=za.ZERO_PATH_STAGED)
+        zr.step(hp=ADAMW_HP, path=za.ZERO_PATH_REGISTER)
+    torch.cuda.synchronize()
+    for a, b in zip(zs.current(), zr.current()):
+        assert _same_bits(a, b)
+    for a, b in zip(zs.params16, zr.params16):
+        assert _same_bits(a, b)
