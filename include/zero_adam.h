@@ -26,7 +26,10 @@
  *                                             16-bit parameter buffer)
  * with t the 1-based count of applied steps.  With the overflow check on, a
  * step whose gradients hold any inf or NaN changes no weight or moment, keeps
- * t, and halves S.
+ * t, and halves S.  The reduction is exact up to one final rounding; m, v
+ * and w are updated in float32, the square root and the division of the
+ * step term with the hardware's approximate forms (a few units in the last
+ * place of a term of size about lr). 
  *
  * Conventions for every entry point:
  *   - Return 0 (ZERO_OK) or a negative ZERO_E* code; arguments are checked on
