@@ -30,6 +30,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -189,13 +190,23 @@ def workload_config(name: str, world: int = 1) -> dict:
     return cfg
 
 
+def source_code_only(text: str) -> str:
+    """C/C++ source with its comments removed and its whitespace collapsed:
+    what the compiler sees of the code, so that an edited comment does not
+    count as a changed kernel."""
+    text = re.sub(r"//[^\n]*|/\*.*?\*/", " ", text, flags=re.S)
+    return " ".join(text.split())
+
+
 def kernel_source_sha() -> str:
+    """Hash of the kernels' code (comments and layout ignored), the key under
+    which profiles/traffic.json records its counters."""
     h = hashlib.sha256()
     for rel in ("mixed_precision_adam_zero_b200/csrc/zero_adam_kernels.cuh",
                 "mixed_precision_adam_zero_b200/csrc/zero_adam_bulk.cuh",
                 "mixed_precision_adam_zero_b200/csrc/zero_adam_api.cu"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            h.update(source_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

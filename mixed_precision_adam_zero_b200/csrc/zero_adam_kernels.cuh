@@ -25,7 +25,8 @@
 //     last-block-done epilogue: each CTA adds its packed arrival (count,
 //     inf/NaN, timeout) to one word of the workspace, and the CTA whose
 //     atomic completes the count updates the control block and re-zeroes
-//     the workspace.  No kernel here spins or waits.
+//     the workspace.  No kernel here spins; the only wait is the grid
+//     dependency wait of the programmatic launch (grid_dependency_wait).
 //
 // Sources of the arithmetic ("Deep dive: DeepSpeed", "Reduce first, then
 // update the owned slice"; AdamW of the "ZeRO" documentation page): see

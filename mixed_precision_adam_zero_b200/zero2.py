@@ -19,7 +19,8 @@ all-gather sequence of stage 2):
      ranks' 16-bit buffers: the reduce-scatter (loads from the peers), the
      update and the parameter all-gather (stores into the peers) are one
      kernel;
-  4. a barrier: every push has landed, and no rank still reads a gradient
+  4. a barrier: every push has landed (the step kernel has completed before
+     the barrier's collective starts on the stream), and no rank still reads a gradient
      that the next backward pass may overwrite.
 
 Only steps 1, 2 and 4 use torch.distributed; with NCCL they are ordered on

@@ -121,3 +121,10 @@ def test_stdout_carries_only_the_json_line():
     assert r.returncode == 0, r.stderr
     assert r.stdout == '{"value": 1}\n'
     assert "python noise" in r.stderr and "library noise" in r.stderr
+
+
+def test_kernel_hash_ignores_comments_and_layout():
+    a = "int f(int x) {  // the answer\n    return x + 1; /* plus\n one */\n}\n"
+    b = "int f(int x) {\n  return x + 1;\n}"
+    c = "int f(int x) { return x + 2; }"
+    assert bench.source_code_only(a) == bench.source_code_only(b) != bench.source_code_only(c)
