@@ -49,7 +49,7 @@ DEFAULT_WORKLOAD = "llama3b"
 DEFAULT_WORKLOAD_MULTI = "zero2"
 # Parameters of the workload that the oracle steps over in the CPU baseline
 # and in the reference arm (the same sample in both).
-ORACLE_SAMPLE_P = 1 << 22
+ORACLE_SAMPLE_P = 1 << 24
 # End-to-end: about this many bytes of host gradients per run by default.
 E2E_BUDGET_BYTES = 16 << 30
 # Peer copy bandwidth per direction measured on this machine's NVLink 5 (GB/s).

@@ -51,7 +51,7 @@ def _check_line(d, workload, P, R, steps, warmup, e2e_steps):
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(c)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0 and cb["sample"]
-    assert cb["sample_P"] == min(P, 1 << 22) and cb["single_thread"]["value"] > 0
+    assert cb["sample_P"] == min(P, 1 << 24) and cb["single_thread"]["value"] > 0
 
 
 def test_bench_line_flat16m():
