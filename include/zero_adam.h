@@ -36,7 +36,11 @@
  *     the host before anything is launched, and a rejected call launches
  *     nothing.  No error is signalled from the device by trapping.
  *   - Device-side calls are asynchronous on the given stream (a NULL stream is
- *     the legacy default stream) unless stated otherwise.
+ *     the legacy default stream) unless stated otherwise.  Their kernels are
+ *     launched with programmatic stream serialization: a kernel may start
+ *     while the kernel before it in the stream finishes, but waits for that
+ *     kernel's completion before it reads or writes any memory, so stream
+ *     order is kept exactly as with a plain launch.
  *   - The caller owns and allocates every buffer; the library allocates no
  *     device memory and keeps no state between calls apart from per-device
  *     launch-shape caches and the static scratch array behind
