@@ -576,6 +576,10 @@ def run_gpu(args) -> None:
             host_out = torch.empty(b.output.shape, dtype=b.output.dtype, pin_memory=True)
         except RuntimeError as e:          # the host cannot pin this much memory: no end-to-end number
             K_e2e, e2e_note = 0, f"pinned host copies of {(h2d + d2h) / 1e9:.1f} GB not available: {e}"[:300]
+    if world > 1:                          # every rank takes the same collective steps: the fewest e2e steps
+        K_e2e = int(-max_over_ranks([-K_e2e], world, device)[0])
+        if K_e2e == 0 and e2e_note is None and e2e_step_count(K, h2d, args.e2e_steps):
+            e2e_note = "another rank could not pin its host copies"
     if K_e2e:
         host_grads = list(host_in.split([g.numel() for g in b.inputs]))
         for hg, dg in zip(host_grads, b.inputs):
