@@ -120,10 +120,12 @@ def zero2emu_bytes_per_param(R: int, gdt: str) -> int:
 
 
 def nvlink_bytes_per_direction(P: int, R: int, gdt: str = "bf16") -> int:
-    """One rank of the ZeRO-2 step across R GPUs: the other ranks' gradients
-    over its slice come in, and its 16-bit results go out to the other
-    replicas, (R - 1)/R * P elements each way (2 bytes each for bf16)."""
-    return (R - 1) * P * GRAD_BYTES[gdt] // R
+    """One rank of the ZeRO-2 step across R GPUs, each way.  In: the other
+    ranks' gradients over its slice, and their 16-bit results into its
+    replica.  Out: its gradient over their slices, and its 16-bit results
+    into their replicas.  (R - 1)/R * P gradient elements and as many 16-bit
+    parameters each way (a reduce-scatter plus an all-gather)."""
+    return (R - 1) * P * (GRAD_BYTES[gdt] + 2) // R
 
 
 def tensor_list(name: str):
@@ -436,8 +438,8 @@ def roofline_kernel(workload: str, world: int = 1) -> str:
 def roofline(workload: str, world: int, P: int, launch_ms: float, peaks: dict, traffic) -> dict:
     """Roofline of the dominant kernel.  HBM-bound: algorithmic bytes per
     launch over its mean duration against the measured copy peak.  The ZeRO-2
-    step across GPUs (R > 1): the bytes one GPU sends over NVLink per step,
-    against the machine's measured peer bandwidth per direction."""
+    step across GPUs (R > 1): the bytes one GPU moves over NVLink each way
+    per step, against the machine's measured peer bandwidth per direction."""
     kind = WORKLOADS[workload][0]
     R = workload_R(workload, world)
     if kind == "zero2" and R > 1:

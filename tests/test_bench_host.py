@@ -83,10 +83,10 @@ def test_zero2_workload_scales_with_the_world():
         assert cfg["bytes_per_param"] == 2 * world + 24 + 2 * world
     P = bench.LLAMA3B_P
     assert bench.nvlink_bytes_per_direction(P, 1) == 0
-    assert bench.nvlink_bytes_per_direction(P, 8) == 7 * P * 2 // 8
+    assert bench.nvlink_bytes_per_direction(P, 8) == 7 * P * 4 // 8
     rf = bench.roofline("zero2", 8, P, 10.0, {}, None)
     assert rf["bound"] == "nvlink" and rf["peak"] == bench.NVLINK_GBS
-    assert rf["achieved"] == pytest.approx(7 * P * 2 / 8 / 1e-2 / 1e9)
+    assert rf["achieved"] == pytest.approx(7 * P * 4 / 8 / 1e-2 / 1e9)
     rf1 = bench.roofline("zero2", 1, P, 10.0, {"hbm_gbs": 6546.6}, None)
     assert rf1["bound"] == "hbm" and rf1["bytes_per_launch"] == 28 * P
     assert bench.zero2_throughput(P, 4, 8.0) == pytest.approx(P * 4 / 8e-3)

@@ -117,6 +117,7 @@ def test_zero2_plumbing_with_two_gloo_ranks():
         assert cfg["R"] == 2 and cfg["P"] == P and cfg["workload"] == "zero2"
         assert slices[0][0] == 0 and slices[0][1] == slices[1][0] and slices[1][1] == P   # they tile [0, P)
         assert all(off % 8 == 0 and off <= lo and n >= hi - off for lo, hi, off, n in slices)
-        # each rank pulls the other's gradient over its own slice and pushes its results out
-        pulled = [(2 - 1) * (hi - lo) * 2 for lo, hi, _, _ in slices]
-        assert sum(pulled) == 2 * bench.nvlink_bytes_per_direction(P, 2)
+        # into each rank: the other's gradient over its own slice, and the other's results
+        n = [hi - lo for lo, hi, _, _ in slices]
+        into = [n[r] * 2 + n[1 - r] * 2 for r in range(2)]
+        assert into[0] == into[1] == bench.nvlink_bytes_per_direction(P, 2)
