@@ -51,7 +51,7 @@ DEFAULT_WORKLOAD_MULTI = "zero2"
 # and in the reference arm (the same sample in both).
 ORACLE_SAMPLE_P = 1 << 24
 # End-to-end: about this many bytes of host gradients per run by default.
-E2E_BUDGET_BYTES = 16 << 30
+E2E_BUDGET_BYTES = 256 << 30
 # Peer copy bandwidth per direction measured on this machine's NVLink 5 (GB/s).
 NVLINK_GBS = 770.0
 LLAMA3B_P = 3_212_749_824

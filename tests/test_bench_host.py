@@ -94,7 +94,7 @@ def test_zero2_workload_scales_with_the_world():
 
 def test_e2e_step_budget():
     assert bench.e2e_step_count(20, 268_436_144) == 20                  # small inputs: every timed step
-    assert bench.e2e_step_count(20, 8 * 2 * 3_212_749_824) == 2         # 51 GB per step: two steps
+    assert bench.e2e_step_count(20, 8 * 2 * 3_212_749_824) == 5         # 51 GB per step: five steps
     assert bench.e2e_step_count(1, 8 * 2 * 3_212_749_824) == 1          # never more than the timed steps
     assert bench.e2e_step_count(20, 1 << 30, requested=5) == 5
     assert bench.e2e_step_count(20, 1 << 30, requested=0) == 0

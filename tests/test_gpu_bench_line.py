@@ -12,6 +12,9 @@ import torch
 
 from conftest import ROOT
 
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
 pytestmark = pytest.mark.gpu
 
 
@@ -61,7 +64,8 @@ def test_bench_line_flat16m():
 
 def test_bench_line_default_is_the_3p2b_llama_list():
     d = _run("--steps", "5", "--warmup", "3", "--cpu-seconds", "1")
-    _check_line(d, "llama3b", 3_212_749_824, 8, 5, 3, 2)
+    P = 3_212_749_824
+    _check_line(d, "llama3b", P, 8, 5, 3, bench.e2e_step_count(5, 8 * 2 * P))   # the default e2e window
     assert d["config"]["tensors"] == 254
 
 
