@@ -10,6 +10,7 @@ import torch
 import oracle
 import synth
 from gpu_helpers import ADAMW_HP, assert_close, assert_params16, compare_full, host_grad, ohp, report_near_zero
+import mixed_precision_adam_zero_b200 as za
 from mixed_precision_adam_zero_b200 import zero_partition_bounds
 from mixed_precision_adam_zero_b200.buffers import FlatZero, ListZero
 
@@ -49,7 +50,9 @@ def _cast_check_full(params16: torch.Tensor, master: torch.Tensor):
 
 
 def _sampled_run(z, flat_grad_bufs, flat_params16, steps, workload, gdt, extra=(), token=False,
-                 check=False, inf_steps=(), scale0=1.0, n_random=1_000_000):
+                 check=False, inf_steps=(), scale0=1.0, n_random=1_000_000, path=0, inf_at=None):
+    """`path`: the step kernel (ZERO_PATH_*); `inf_at`: the (rank, index) of
+    every planted inf, else a seeded site per step."""
     P, R = z.P, z.R
     idx = synth.sample_indices(P, n_random, workload, extra=list(extra) + _boundaries(P, R, getattr(z, "numels", ())))
     idx_dev = idx.cuda()
@@ -59,10 +62,10 @@ def _sampled_run(z, flat_grad_bufs, flat_params16, steps, workload, gdt, extra=(
         S = st.ctrl.loss_scale
         _fill(workload, k, flat_grad_bufs, scale=S)
         if k in inf_steps:
-            rank, i = synth.inf_site(workload, k, R, P)
+            rank, i = inf_at if inf_at is not None else synth.inf_site(workload, k, R, P)
             flat_grad_bufs[rank][i] = float("inf")
         wts = [float(x) for x in synth.token_counts(R, workload, k)] if token else None
-        z.step(hp=ADAMW_HP, rank_weights=wts, check=check)
+        z.step(hp=ADAMW_HP, rank_weights=wts, check=check, path=path)
         sample = [host_grad(b.index_select(0, idx_dev)) for b in flat_grad_bufs]
         skipped = oracle.step(st, sample, gdt, ohp(ADAMW_HP), weights=wts, check=check,
                               sharded=True, P=P, idx=idx.numpy().astype(np.uint64))
@@ -153,6 +156,64 @@ def test_flat_beyond_2_to_the_31():
     _sampled_run(z, z.grads, z.params16, 3, wl, "bf16", extra=near, n_random=200_000)
 
 
+NEAR_2_31 = [2**31 + d for d in range(-20, 13)] + [2**31 - 2048 * k for k in (1, 2, 3)]
+
+
+def test_flat_beyond_2_to_the_31_register_kernel_and_scan():
+    """P = 2^31 + 13 flat, R = 2, fp16 x 2^16 with one state set: the
+    overflow scan pass and the register step kernel (plain loads) with 64-bit
+    element indices, an inf planted at index 2^31 + 5 at step 2 (found only
+    if the scan reaches past 2^31); the initial 16-bit cast of the masters
+    over the whole vector as well."""
+    P, R, wl = 2**31 + 13, 2, synth.WORKLOADS["flat1p5b"]
+    z = FlatZero(P, R, "f16", "f16", loss_scale=65536.0)
+    z.load_master(synth.normal(P, 0.02, synth.seed_for(wl, synth.KIND_MASTER, 3), device="cuda"))
+    _cast_check_full(z.params16, z.master[0])
+    _sampled_run(z, z.grads, z.params16, 3, wl, "f16", extra=NEAR_2_31, check=True, inf_steps=(2,),
+                 scale0=65536.0, n_random=200_000, path=za.ZERO_PATH_REGISTER, inf_at=(1, 2**31 + 5))
+    c = z.ctrl()
+    assert (c.step, c.skipped, c.loss_scale) == (2, 1, 32768.0)
+
+
+@pytest.mark.parametrize("path", [za.ZERO_PATH_STAGED, za.ZERO_PATH_REGISTER])
+def test_list_tensor_beyond_2_to_the_31(path):
+    """A tensor list whose middle tensor has 2^31 + 77 elements (tensor-local
+    offsets beyond 2^31), R = 2 bf16, 3 steps, staged and register kernels;
+    sampled around every tensor boundary and around local offset 2^31."""
+    wl = synth.WORKLOADS["flat1p5b"]
+    tensors = [("head", 1000), ("big", 2**31 + 77), ("tail", 999)]
+    z, gbufs, pbuf = _list_with_flat_buffers(tensors, 2, "bf16", "bf16")
+    z.load_master(synth.normal(z.P, 0.02, synth.seed_for(wl, synth.KIND_MASTER, 4), device="cuda"))
+    _cast_check_full(pbuf, z.master[0])
+    near = [1000 + x for x in NEAR_2_31] + [1000 + 2**31 + 77 + d for d in range(-9, 9)]
+    _sampled_run(z, gbufs, pbuf, 3, wl, "bf16", extra=near, n_random=200_000, path=path)
+
+
+@pytest.mark.parametrize("path", [za.ZERO_PATH_STAGED, za.ZERO_PATH_REGISTER])
+def test_accumulate_beyond_2_to_the_31(path):
+    """Micro-step accumulation over P = 2^31 + 13 (R = 2 bf16, token
+    weights, two micro-batches): the staged and register accumulation
+    kernels' 64-bit indices, sampled against the oracle."""
+    P, R, wl = 2**31 + 13, 2, synth.WORKLOADS["flat1p5b"]
+    z = FlatZero(64, 1, "f32", "bf16", alloc_grads=False)       # only its workspace and control block
+    acc = torch.empty(P, dtype=torch.float32, device="cuda")
+    micro = [torch.empty(P, dtype=torch.bfloat16, device="cuda") for _ in range(R)]
+    idx = synth.sample_indices(P, 200_000, wl, extra=NEAR_2_31 + _boundaries(P, R))
+    idx_dev = idx.cuda()
+    oacc = np.zeros(idx.numel(), dtype=np.float32)
+    for mu in range(2):
+        _fill(wl, 500 + mu, micro)
+        wts = [float(x) for x in synth.token_counts(R, wl, 500 + mu)]
+        za.zero_accumulate_grads(P, R, grad_dtype=za.ZERO_BF16, grads=micro, accum=acc, scale=0.5,
+                                 first=(mu == 0), rank_weights=wts, workspace=z.workspace, ctrl=z.ctrl_buf,
+                                 path=path)
+        oracle.accumulate(oacc, [host_grad(g.index_select(0, idx_dev)) for g in micro], "bf16", 0.5,
+                          first=(mu == 0), weights=wts)
+    torch.cuda.synchronize()
+    assert_close(acc.index_select(0, idx_dev), oacc.astype(np.float64), "accumulated gradient")
+    assert z.ctrl().device_error == 0 and not z.workspace.any()
+
+
 def test_gpt2m_list_fp16_in_place_two_pass():
     """The GPT-2-medium list with one state set: the overflow scan runs as a
     pass of its own before the in-place step (the benchmark's gpt2m_inplace
@@ -172,7 +233,6 @@ def test_flat16m_four_micro_batches_per_update_full_oracle():
     8 bf16 rank gradients reduced into the fp32 accumulator (the staged
     kernel, chosen automatically at this size), then the step over it,
     2 updates; every element against the oracle."""
-    import mixed_precision_adam_zero_b200 as za
     P, R, gas, wl = synth.FLAT16M_P, 8, 4, synth.WORKLOADS["flat16m"]
     z = FlatZero(P, 1, "f32", "bf16", alloc_grads=False)
     w0 = synth.normal(P, 0.02, synth.seed_for(wl, synth.KIND_MASTER, 2), device="cuda")
