@@ -41,6 +41,15 @@
  *     while the kernel before it in the stream finishes, but waits for that
  *     kernel's completion before it reads or writes any memory, so stream
  *     order is kept exactly as with a plain launch.
+ *   - The step calls (zero_step_fused, zero_step_fused_list,
+ *     zero_step_fused_noalloc, with their scan and restore kernels),
+ *     zero_accumulate_grads and zero_gather_params[_list] only enqueue work
+ *     on the stream, so stream capture can record them into a CUDA graph.
+ *     Capture a call after one eager call of the same kind on the device (the
+ *     first launch of each kernel on a device fills its launch-shape cache).
+ *     A replay reuses the values the arguments had at capture time (pointers,
+ *     sizes, hyperparameters, rank weights); the step count, loss scale and
+ *     skip record live in the control block and advance on every replay.
  *   - The caller owns and allocates every buffer; the library allocates no
  *     device memory and keeps no state between calls apart from per-device
  *     launch-shape caches and the static scratch array behind
