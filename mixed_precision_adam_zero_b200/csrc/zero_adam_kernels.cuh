@@ -545,8 +545,11 @@ __device__ __forceinline__ void finish_step(const StepParams& p, bool bad, bool 
     }
 }
 
+// Two 256-thread CTAs per SM: at most 128 registers a thread.  Without the
+// bound the list instances with fp32 gradients took 131 (one CTA per SM);
+// with it they spill 16 bytes, and every other instance fits without a spill.
 template <class G, class Pm, int RC, bool LIST, bool PUSH = false>
-__global__ void __launch_bounds__(kThreads) step_kernel(const __grid_constant__ StepParams p) {
+__global__ void __launch_bounds__(kThreads, 2) step_kernel(const __grid_constant__ StepParams p) {
     __shared__ const void* s_gp[LIST ? ZERO_MAX_RANKS : 1];
     grid_dependency_wait();
     allow_dependents();
