@@ -427,10 +427,11 @@ def roofline_kernel(workload: str, world: int = 1) -> str:
         if world == 1:
             return "step_bulk_kernel (flat, owner 0 of 1, no peers): the ZeRO-2 step on one GPU"
         return "step_bulk_kernel (flat, push): this GPU's owner kernel of the ZeRO-2 step across GPUs"
-    step = ("step_bulk_kernel" if R in (1, 2, 4, 8) else "step_kernel") + (" (flat)" if kind == "flat" else " (list)")
+    staged = R in (1, 2, 4, 8) or (R == 16 and gdt != "f32")
+    step = ("step_bulk_kernel" if staged else "step_kernel") + (" (flat)" if kind == "flat" else " (list)")
     gas = GAS.get(workload, 0)
     if gas:
-        acc = "accum_bulk_kernel" if R in (1, 2, 4, 8) else "accum_kernel"
+        acc = "accum_bulk_kernel" if staged else "accum_kernel"
         return f"{gas} x {acc} + step_bulk_kernel (flat, R = 1 f32)"
     return step
 

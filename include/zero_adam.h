@@ -136,7 +136,8 @@ typedef struct zero_ctrl {
  *   ZERO_PATH_STAGED   one producer thread per CTA stages tiles of every
  *                      input array into shared memory with 1-D bulk copies
  *                      (cp.async.bulk, no tensor map, no multicast); compiled
- *                      for 1, 2, 4 and 8 gradient buffers;
+ *                      for 1, 2, 4 and 8 gradient buffers, and for 16 with
+ *                      16-bit gradients;
  *   ZERO_PATH_REGISTER every thread reads its gradients with plain 16-byte
  *                      global loads (ld.global) into registers; any count;
  *   ZERO_PATH_AUTO     the staged kernel when one is compiled for the count
@@ -367,8 +368,8 @@ int zero_selftest_wait_timeout(void *ctrl, void *stream);
  * kernel that, only if the step was skipped, re-casts the 16-bit parameters
  * from the untouched master set.
  * The step kernel is the one args->path selects; ZERO_PATH_STAGED with a
- * gradient-buffer count other than 1, 2, 4 or 8, or an unknown path, is
- * ZERO_EINVAL.
+ * gradient-buffer count other than 1, 2, 4, 8 or (16-bit gradients) 16, or
+ * an unknown path, is ZERO_EINVAL.
  * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ERANGE (R > ZERO_MAX_RANKS, or
  * P > ZERO_MAX_ELEMENTS), ZERO_EOVERFLOW (P*8 bytes overflow), ZERO_ECUDA. */
 int zero_step_fused(const zero_step_args *args, void *stream);
@@ -469,7 +470,8 @@ typedef struct zero_accum_args {
 
 /* Launches one kernel; asynchronous on `stream`.  The staged kernel
  * (ZERO_PATH_STAGED above) hands its tiles out dynamically; here it needs a
- * workspace and ctrl and R = 1, 2, 4 or 8.  The register kernel
+ * workspace and ctrl and R = 1, 2, 4, 8 or (16-bit gradients) 16.  The
+ * register kernel
  * streams through registers and touches neither workspace nor ctrl.  Both
  * give bitwise identical sums.  ZERO_PATH_AUTO takes the staged kernel
  * whenever it is possible (the faster one at nearly every size), else the

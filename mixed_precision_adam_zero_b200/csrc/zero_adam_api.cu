@@ -117,9 +117,9 @@ int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st, unsig
 
 // ------------------------------------------------------------ kernel tables
 
-// Calls with a compile-time rank count stage their tiles through shared
-// memory with bulk copies; other rank counts use the register path.  PUSH:
-// flat calls that also store the 16-bit values into other replicas.
+// Calls with a compiled rank count stage their tiles through shared memory
+// with bulk copies; other rank counts use the register path.  PUSH: flat
+// calls that also store the 16-bit values into other replicas.
 template <class G, class Pm, int RC, bool LIST, bool PUSH>
 Kern bulk_kern() {
     return Kern{(const void*)step_bulk_kernel<G, Pm, RC, LIST, PUSH>, BulkShape<G, RC>::kSmem, kBulkThreads};
@@ -133,6 +133,9 @@ Kern step_kern_rc(uint32_t R, bool staged) {
         case 2: return bulk_kern<G, Pm, 2, LIST, PUSH>();
         case 4: return bulk_kern<G, Pm, 4, LIST, PUSH>();
         case 8: return bulk_kern<G, Pm, 8, LIST, PUSH>();
+        case 16:
+            if constexpr (sizeof(G) == 2) return bulk_kern<G, Pm, 16, LIST, PUSH>();
+            else return Kern{(const void*)step_kernel<G, Pm, 0, LIST, PUSH>, 0u, kThreads};
         default: return Kern{(const void*)step_kernel<G, Pm, 0, LIST, PUSH>, 0u, kThreads};
     }
 }
@@ -152,12 +155,17 @@ Kern step_kern_gd(int32_t grad_dtype, int32_t param_dtype, uint32_t R, bool stag
     }
 }
 
-bool has_staged(uint32_t R) { return R == 1 || R == 2 || R == 4 || R == 8; }
+// Rank counts with a staged instance: 1, 2, 4 and 8, and 16 for 16-bit
+// gradients (two 88 KB stages; with fp32 gradients one stage would not leave
+// room for a second).
+bool has_staged(uint32_t R, int32_t grad_dtype) {
+    return R == 1 || R == 2 || R == 4 || R == 8 || (R == 16 && grad_dtype != ZERO_F32);
+}
 
 // The step kernel for a path (ZERO_PATH_*): staged when asked for or, in
 // AUTO, when one is compiled for R; else the register kernel.
 Kern step_kern(bool list, bool push, int32_t grad_dtype, int32_t param_dtype, uint32_t R, uint32_t path) {
-    const bool staged = path != ZERO_PATH_REGISTER && has_staged(R);
+    const bool staged = path != ZERO_PATH_REGISTER && has_staged(R, grad_dtype);
     if (list) return step_kern_gd<true, false>(grad_dtype, param_dtype, R, staged);
     return push ? step_kern_gd<false, true>(grad_dtype, param_dtype, R, staged)
                 : step_kern_gd<false, false>(grad_dtype, param_dtype, R, staged);
@@ -197,6 +205,9 @@ Kern accum_kern_rc(uint32_t R, bool bulk) {
             case 2: return accum_bulk_kern<G, 2>();
             case 4: return accum_bulk_kern<G, 4>();
             case 8: return accum_bulk_kern<G, 8>();
+            case 16:
+                if constexpr (sizeof(G) == 2) return accum_bulk_kern<G, 16>();
+                break;
             default: break;
         }
     }
@@ -315,7 +326,7 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     kp->ctrl = static_cast<zero_ctrl*>(a->ctrl);
     kp->ws = static_cast<Workspace*>(a->workspace);
     kp->R = ng;  // the reduction's length; the partition is a->R (owner_range)
-    if (a->path == ZERO_PATH_STAGED && !has_staged(ng)) return ZERO_EINVAL;
+    if (a->path == ZERO_PATH_STAGED && !has_staged(ng, a->grad_dtype)) return ZERO_EINVAL;
     kp->growth_interval = a->growth_interval;
     kp->two_set = two ? 1 : 0;
     return ZERO_OK;
@@ -603,7 +614,7 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     if ((a->workspace == nullptr) != (a->ctrl == nullptr)) return ZERO_EINVAL;
     if (a->path != ZERO_PATH_AUTO && a->path != ZERO_PATH_REGISTER && a->path != ZERO_PATH_STAGED)
         return ZERO_EINVAL;
-    const bool can_stage = a->workspace != nullptr && (a->R == 1 || a->R == 2 || a->R == 4 || a->R == 8);
+    const bool can_stage = a->workspace != nullptr && has_staged(a->R, a->grad_dtype);
     if (a->path == ZERO_PATH_STAGED && !can_stage) return ZERO_EINVAL;
     if (!aligned16(a->workspace) || (reinterpret_cast<uintptr_t>(a->ctrl) & 7u) != 0) return ZERO_EALIGN;
     AccumParams ap;

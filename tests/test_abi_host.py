@@ -133,6 +133,7 @@ def _args(**over):
     (dict(push_params16=[A]), za.ZERO_EINVAL),               # pushes need an owner
     (dict(path=3), za.ZERO_EINVAL),                          # unknown kernel path
     (dict(path=za.ZERO_PATH_STAGED, R=3, grads=[A] * 3), za.ZERO_EINVAL),   # no staged kernel for 3
+    (dict(path=za.ZERO_PATH_STAGED, R=16, grads=[A] * 16, grad_dtype=za.ZERO_F32), za.ZERO_EINVAL),  # 16 x fp32
     (dict(path=za.ZERO_PATH_STAGED, n_grads=3), za.ZERO_EINVAL),
     (dict(n_grads=300), za.ZERO_ERANGE),
     (dict(n_grads=2, rank_weights=[1, -1]), za.ZERO_EINVAL),      # weights over the n_grads buffers
@@ -265,6 +266,8 @@ def test_pushes_need_an_owner():
     (dict(path=3), za.ZERO_EINVAL),
     (dict(path=za.ZERO_PATH_STAGED), za.ZERO_EINVAL),                 # staged needs a workspace
     (dict(R=3, grads=[A] * 3, workspace=A, ctrl=A, path=za.ZERO_PATH_STAGED), za.ZERO_EINVAL),
+    (dict(R=16, grads=[A] * 16, grad_dtype=za.ZERO_F32, workspace=A, ctrl=A, path=za.ZERO_PATH_STAGED),
+     za.ZERO_EINVAL),
     (dict(accum_offset=4, owner=1), za.ZERO_EALIGN),
     (dict(accum_offset=256, owner=1), za.ZERO_EINVAL),               # beyond owner 1's first element (250)
 ])

@@ -24,7 +24,8 @@ def _run(P, R, gdt, gas, updates, token=True, S0=1.0, check=False, bad=None, two
     accumulation gets the step's workspace and ctrl (shared-memory staged
     kernel for R in 1, 2, 4, 8), else none (register kernel)."""
     z = FlatZero(P, 1, "f32", "bf16", two_set=two_set, loss_scale=S0, alloc_grads=False)
-    ws = dict(workspace=z.workspace, ctrl=z.ctrl_buf, path=STAGED if R in (1, 2, 4, 8) else za.ZERO_PATH_AUTO) \
+    ws = dict(workspace=z.workspace, ctrl=z.ctrl_buf,
+              path=STAGED if R in (1, 2, 4, 8) or (R == 16 and gdt != "f32") else za.ZERO_PATH_AUTO) \
         if staged else dict(path=za.ZERO_PATH_REGISTER)
     acc = torch.zeros(P, dtype=torch.float32, device="cuda")
     micro = [torch.zeros(P, dtype={"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt],
@@ -56,7 +57,7 @@ def _run(P, R, gdt, gas, updates, token=True, S0=1.0, check=False, bad=None, two
 
 @pytest.mark.parametrize("staged", [True, False])
 @pytest.mark.parametrize("gdt,R", [("bf16", 8), ("bf16", 4), ("f16", 4), ("f32", 4), ("f32", 8), ("bf16", 3),
-                                   ("bf16", 2), ("bf16", 1)])
+                                   ("bf16", 16), ("f16", 16), ("bf16", 2), ("bf16", 1)])
 def test_accumulate_then_step(gdt, R, staged):
     _run(P=60_013, R=R, gdt=gdt, gas=4, updates=3, staged=staged)
 
@@ -73,8 +74,8 @@ def _micro(P, R, dt, seed):
     return [synth.normal(P, 1e-3, seed + r, device="cuda", dtype=dt) for r in range(R)]
 
 
-@pytest.mark.parametrize("gdt", ["bf16", "f16", "f32"])
-@pytest.mark.parametrize("R", [1, 2, 4, 8])
+@pytest.mark.parametrize("gdt,R", [(g, r) for g in ("bf16", "f16", "f32") for r in (1, 2, 4, 8, 16)
+                                   if not (g == "f32" and r == 16)])
 def test_staged_and_register_kernels_agree_bitwise(gdt, R):
     tdt = {"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[gdt]
     P = 37 * 2048 + 5
