@@ -418,17 +418,19 @@ def build_workload(name: str, device, stream, world: int = 1) -> Bench:
 def roofline_kernel(workload: str, world: int = 1) -> str:
     """The kernel (or, for accumulation, the launch sequence of one step) the
     roofline fraction is measured on."""
-    kind, size, R, gdt, pdt, scaled = WORKLOADS[workload]
+    kind, size, _, gdt, pdt, scaled = WORKLOADS[workload]
+    R = workload_R(workload, world)          # zero2: one rank per GPU
     if kind == "z3gather":
         return "z3_gather_kernel"
     if kind == "zero2emu":
         return f"{R} x step_bulk_kernel (flat, push): the owners of an emulated {R}-rank ZeRO-2 step"
+    staged = R in (1, 2, 4, 8) or (R == 16 and gdt != "f32")
+    name = "step_bulk_kernel" if staged else "step_chunked_kernel"   # flat and whole-list calls: always staged
     if kind == "zero2":
         if world == 1:
-            return "step_bulk_kernel (flat, owner 0 of 1, no peers): the ZeRO-2 step on one GPU"
-        return "step_bulk_kernel (flat, push): this GPU's owner kernel of the ZeRO-2 step across GPUs"
-    staged = R in (1, 2, 4, 8) or (R == 16 and gdt != "f32")
-    step = ("step_bulk_kernel" if staged else "step_kernel") + (" (flat)" if kind == "flat" else " (list)")
+            return f"{name} (flat, owner 0 of 1, no peers): the ZeRO-2 step on one GPU"
+        return f"{name} (flat, push): this GPU's owner kernel of the ZeRO-2 step across GPUs"
+    step = name + (" (flat)" if kind == "flat" else " (list)")
     gas = GAS.get(workload, 0)
     if gas:
         acc = "accum_bulk_kernel" if staged else "accum_kernel"

@@ -135,14 +135,16 @@ typedef struct zero_ctrl {
 /* Kernel paths of the step and of the accumulation (field `path`):
  *   ZERO_PATH_STAGED   one producer thread per CTA stages tiles of every
  *                      input array into shared memory with 1-D bulk copies
- *                      (cp.async.bulk, no tensor map, no multicast); compiled
- *                      for 1, 2, 4 and 8 gradient buffers, and for 16 with
- *                      16-bit gradients;
+ *                      (cp.async.bulk, no tensor map, no multicast); an
+ *                      instance is compiled for 1, 2, 4 and 8 gradient
+ *                      buffers, and for 16 with 16-bit gradients; for any
+ *                      other count the step streams each tile's ranks through
+ *                      the stages eight at a time (flat calls and list calls
+ *                      over the whole vector; not a list call for one owner);
  *   ZERO_PATH_REGISTER every thread reads its gradients with plain 16-byte
  *                      global loads (ld.global) into registers; any count;
- *   ZERO_PATH_AUTO     the staged kernel when one is compiled for the count
- *                      (the faster one at nearly every size), else the
- *                      register kernel.
+ *   ZERO_PATH_AUTO     the staged kernel wherever it can run (the faster one
+ *                      at nearly every size), else the register kernel.
  * Both give bitwise identical results.  Across GPUs the gradient buffers are
  * other GPUs' memory mapped into this process: ZERO_PATH_REGISTER then reads
  * them with ordinary peer loads instead of bulk copies. */
@@ -367,9 +369,9 @@ int zero_selftest_wait_timeout(void *ctrl, void *stream);
  * (b) check on in two-set mode with owner == -1: one pass plus a restore
  * kernel that, only if the step was skipped, re-casts the 16-bit parameters
  * from the untouched master set.
- * The step kernel is the one args->path selects; ZERO_PATH_STAGED with a
- * gradient-buffer count other than 1, 2, 4, 8 or (16-bit gradients) 16, or
- * an unknown path, is ZERO_EINVAL.
+ * The step kernel is the one args->path selects; an unknown path is
+ * ZERO_EINVAL, and so is ZERO_PATH_STAGED for a list call for one owner with
+ * a gradient-buffer count other than 1, 2, 4, 8 or (16-bit gradients) 16.
  * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ERANGE (R > ZERO_MAX_RANKS, or
  * P > ZERO_MAX_ELEMENTS), ZERO_EOVERFLOW (P*8 bytes overflow), ZERO_ECUDA. */
 int zero_step_fused(const zero_step_args *args, void *stream);

@@ -118,57 +118,73 @@ int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st, unsig
 // ------------------------------------------------------------ kernel tables
 
 // Calls with a compiled rank count stage their tiles through shared memory
-// with bulk copies; other rank counts use the register path.  PUSH: flat
-// calls that also store the 16-bit values into other replicas.
+// with bulk copies (step_bulk_kernel); flat calls and whole-list calls with
+// any other count stream each tile's ranks through the same kind of ring,
+// eight at a time (step_chunked_kernel); the register kernel takes the rest
+// and every call that asks for it.  PUSH: flat calls that also store the
+// 16-bit values into other replicas.
+enum class StepKind { Register, Staged, Chunked };
+
 template <class G, class Pm, int RC, bool LIST, bool PUSH>
 Kern bulk_kern() {
     return Kern{(const void*)step_bulk_kernel<G, Pm, RC, LIST, PUSH>, BulkShape<G, RC>::kSmem, kBulkThreads};
 }
 
 template <class G, class Pm, bool LIST, bool PUSH>
-Kern step_kern_rc(uint32_t R, bool staged) {
-    if (!staged) return Kern{(const void*)step_kernel<G, Pm, 0, LIST, PUSH>, 0u, kThreads};
-    switch (R) {
-        case 1: return bulk_kern<G, Pm, 1, LIST, PUSH>();
-        case 2: return bulk_kern<G, Pm, 2, LIST, PUSH>();
-        case 4: return bulk_kern<G, Pm, 4, LIST, PUSH>();
-        case 8: return bulk_kern<G, Pm, 8, LIST, PUSH>();
-        case 16:
-            if constexpr (sizeof(G) == 2) return bulk_kern<G, Pm, 16, LIST, PUSH>();
-            else return Kern{(const void*)step_kernel<G, Pm, 0, LIST, PUSH>, 0u, kThreads};
-        default: return Kern{(const void*)step_kernel<G, Pm, 0, LIST, PUSH>, 0u, kThreads};
+Kern step_kern_rc(uint32_t R, StepKind kind) {
+    if (kind == StepKind::Chunked)
+        return Kern{(const void*)step_chunked_kernel<G, Pm, LIST, PUSH>, ChunkShape<G>::kSmem, kBulkThreads};
+    if (kind == StepKind::Staged) {
+        switch (R) {
+            case 1: return bulk_kern<G, Pm, 1, LIST, PUSH>();
+            case 2: return bulk_kern<G, Pm, 2, LIST, PUSH>();
+            case 4: return bulk_kern<G, Pm, 4, LIST, PUSH>();
+            case 8: return bulk_kern<G, Pm, 8, LIST, PUSH>();
+            case 16:
+                if constexpr (sizeof(G) == 2) return bulk_kern<G, Pm, 16, LIST, PUSH>();
+                break;
+            default: break;
+        }
     }
+    return Kern{(const void*)step_kernel<G, Pm, 0, LIST, PUSH>, 0u, kThreads};
 }
 
 template <class G, bool LIST, bool PUSH>
-Kern step_kern_pm(int32_t param_dtype, uint32_t R, bool staged) {
-    return param_dtype == ZERO_BF16 ? step_kern_rc<G, __nv_bfloat16, LIST, PUSH>(R, staged)
-                                    : step_kern_rc<G, __half, LIST, PUSH>(R, staged);
+Kern step_kern_pm(int32_t param_dtype, uint32_t R, StepKind kind) {
+    return param_dtype == ZERO_BF16 ? step_kern_rc<G, __nv_bfloat16, LIST, PUSH>(R, kind)
+                                    : step_kern_rc<G, __half, LIST, PUSH>(R, kind);
 }
 
 template <bool LIST, bool PUSH>
-Kern step_kern_gd(int32_t grad_dtype, int32_t param_dtype, uint32_t R, bool staged) {
+Kern step_kern_gd(int32_t grad_dtype, int32_t param_dtype, uint32_t R, StepKind kind) {
     switch (grad_dtype) {
-        case ZERO_F32: return step_kern_pm<float, LIST, PUSH>(param_dtype, R, staged);
-        case ZERO_BF16: return step_kern_pm<__nv_bfloat16, LIST, PUSH>(param_dtype, R, staged);
-        default: return step_kern_pm<__half, LIST, PUSH>(param_dtype, R, staged);
+        case ZERO_F32: return step_kern_pm<float, LIST, PUSH>(param_dtype, R, kind);
+        case ZERO_BF16: return step_kern_pm<__nv_bfloat16, LIST, PUSH>(param_dtype, R, kind);
+        default: return step_kern_pm<__half, LIST, PUSH>(param_dtype, R, kind);
     }
 }
 
-// Rank counts with a staged instance: 1, 2, 4 and 8, and 16 for 16-bit
-// gradients (two 88 KB stages; with fp32 gradients one stage would not leave
-// room for a second).
+// Rank counts with a compiled staged instance: 1, 2, 4 and 8, and 16 for
+// 16-bit gradients (two 88 KB stages; with fp32 gradients one stage would not
+// leave room for a second).
 bool has_staged(uint32_t R, int32_t grad_dtype) {
     return R == 1 || R == 2 || R == 4 || R == 8 || (R == 16 && grad_dtype != ZERO_F32);
 }
 
-// The step kernel for a path (ZERO_PATH_*): staged when asked for or, in
-// AUTO, when one is compiled for R; else the register kernel.
-Kern step_kern(bool list, bool push, int32_t grad_dtype, int32_t param_dtype, uint32_t R, uint32_t path) {
-    const bool staged = path != ZERO_PATH_REGISTER && has_staged(R, grad_dtype);
-    if (list) return step_kern_gd<true, false>(grad_dtype, param_dtype, R, staged);
-    return push ? step_kern_gd<false, true>(grad_dtype, param_dtype, R, staged)
-                : step_kern_gd<false, false>(grad_dtype, param_dtype, R, staged);
+// The step kernel for a path (ZERO_PATH_*): AUTO and STAGED take the staged
+// instance compiled for R, else (flat calls, whole-list calls) the chunked
+// kernel; a list call for one owner with another R, and REGISTER, take the
+// register kernel.
+Kern step_kern(bool list, bool whole, bool push, int32_t grad_dtype, int32_t param_dtype, uint32_t R,
+               uint32_t path) {
+    StepKind kind = StepKind::Register;
+    if (path != ZERO_PATH_REGISTER) {
+        if (has_staged(R, grad_dtype)) kind = StepKind::Staged;
+        else if (!list || whole) kind = StepKind::Chunked;
+    }
+    if (list) return step_kern_gd<true, false>(grad_dtype, param_dtype, R, kind);
+    return push ? step_kern_gd<false, true>(grad_dtype, param_dtype, R, kind)
+                : step_kern_gd<false, false>(grad_dtype, param_dtype, R, kind);
 }
 
 template <bool LIST>
@@ -326,7 +342,6 @@ int check_common(const zero_step_args* a, StepParams* kp) {
     kp->ctrl = static_cast<zero_ctrl*>(a->ctrl);
     kp->ws = static_cast<Workspace*>(a->workspace);
     kp->R = ng;  // the reduction's length; the partition is a->R (owner_range)
-    if (a->path == ZERO_PATH_STAGED && !has_staged(ng, a->grad_dtype)) return ZERO_EINVAL;
     kp->growth_interval = a->growth_interval;
     kp->two_set = two ? 1 : 0;
     return ZERO_OK;
@@ -369,7 +384,7 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
     } else {
         kp->check = check ? 1 : 0;
     }
-    const Kern k = step_kern(LIST, kp->npush > 0, a->grad_dtype, a->param_dtype, kp->R, a->path);
+    const Kern k = step_kern(LIST, kp->whole != 0, kp->npush > 0, a->grad_dtype, a->param_dtype, kp->R, a->path);
     const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;
     const Shape sh = make_shape(lo, hi, ctas);
@@ -596,6 +611,8 @@ int zero_step_fused_list(const zero_step_args* a, const zero_tensor_list* l, voi
         return ZERO_EINVAL;  // multi-GPU fields: flat calls only
     if (a->P != l->P || a->R != l->R || a->grad_dtype != l->grad_dtype || a->param_dtype != l->param_dtype)
         return ZERO_EINVAL;
+    // A list call for one owner has no chunked kernel: STAGED needs a compiled R.
+    if (a->path == ZERO_PATH_STAGED && a->owner >= 0 && !has_staged(a->R, a->grad_dtype)) return ZERO_EINVAL;
     kp.tab = device_table(l);
     kp.whole = a->owner < 0 ? 1 : 0;
     return run_step<true>(a, &kp, static_cast<cudaStream_t>(stream));

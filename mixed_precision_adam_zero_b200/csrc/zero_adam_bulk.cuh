@@ -578,8 +578,9 @@ __device__ __forceinline__ void list_scalar_whole(const StepParams& p, const Sca
             const uint64_t be = vec ? (t1 & ~7ull) : t0;  // body [t0, be)
             const uint64_t from = be > x ? be : x;
             if (from < sb) {
+                const uint32_t nr = RC > 0 ? (uint32_t)RC : p.R;  // RC == 0: the chunked kernel, any R
                 __syncthreads();
-                for (uint32_t r = threadIdx.x; r < RC; r += kBulkThreads) s_gp[r] = p.tab.grads[(uint64_t)j * RC + r];
+                for (uint32_t r = threadIdx.x; r < nr; r += kBulkThreads) s_gp[r] = p.tab.grads[(uint64_t)j * nr + r];
                 __syncthreads();
                 const GradPtrs<G, RC> gp(s_gp);
                 Pm* pp = static_cast<Pm*>(p.tab.params[j]);
@@ -700,6 +701,265 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
             }
         } else {
             flat_dynamic<G, Pm, RC, PUSH>(p, full, empty, slot, ring, bad);
+        }
+    } else if (threadIdx.x == 0) {
+        s_start = StepStart{*p.ctrl, p.ws->found};
+    }
+    finish_step<PUSH>(p, bad, s_timed_out != 0u, &s_start);
+}
+
+// ------------------------------------------------------------ any rank count
+
+// Rank counts without a compiled staged instance (3, 5-7, 9-15, 17-256, and
+// 16 with fp32 gradients) stream each tile through the ring in chunks of
+// kChunkRanks ranks: the stage of chunk c holds the tile's gradient slices of
+// ranks [8c, 8c + 8), and the tile's last chunk also its master, m and v.  A
+// consumer thread handles the same four elements in every chunk of a tile and
+// keeps their float64 sums in registers from the first chunk to the last, so
+// the ranks are added in the order 0..R-1 as in the other kernels (the
+// results are bitwise theirs); the last chunk applies Adam.  Flat calls and
+// list calls over the whole vector (a list call for one owner takes the
+// register kernel).  Tiles are handed out as in flat_dynamic and
+// list_dynamic: CTA b starts on tile b and claims the rest from the
+// workspace counter one tile ahead.
+constexpr uint32_t kChunkRanks = 8;
+static_assert(4 * kConsumers == kTile, "one 4-element group per consumer thread per tile");
+
+template <class G>
+using ChunkShape = BulkShape<G, (int)kChunkRanks>;
+
+// Stage descriptor of the chunked kernel, written before the stage's
+// barrier is armed.
+struct ChunkDesc {
+    uint64_t e0;      // flat index of the tile's first element
+    uint64_t toff;    // flat index of the tensor's first element (0: flat)
+    void* params;     // the tensor's 16-bit parameters
+    uint32_t n;       // elements (a multiple of 8); 0: no more tiles
+    uint32_t chunk;   // ranks [8 chunk, 8 chunk + 8) of the tile
+};
+static_assert(sizeof(ChunkDesc) * 8 <= kBarBytes - 128, "stage descriptors must fit the barrier header");
+
+// Copies of one chunk into `stage`: ranks [r0, r0 + rn) of the gradient bases
+// `gp` (the tile's tensor), and the state when `last`.
+template <class G>
+__device__ __forceinline__ void chunk_issue(const StateIO& io, const void* const* gp, uint32_t r0, uint32_t rn,
+                                            bool last, unsigned char* stage, uint64_t* bar, uint64_t e0,
+                                            uint64_t le0, uint32_t n) {
+    using Sh = ChunkShape<G>;
+    const uint32_t gbytes = n * (uint32_t)sizeof(G), sbytes = n * 4u;
+    mbar_expect_tx(bar, rn * gbytes + (last ? 3u * sbytes : 0u));
+    for (uint32_t r = 0; r < rn; ++r)
+        bulk_g2s(stage + r * Sh::kGradSlice, static_cast<const G*>(gp[r0 + r]) + le0, gbytes, bar);
+    if (last) {
+        unsigned char* st = stage + kChunkRanks * Sh::kGradSlice;
+        bulk_g2s(st, io.wi + e0, sbytes, bar);
+        bulk_g2s(st + kTile * 4u, io.mi + e0, sbytes, bar);
+        bulk_g2s(st + 2u * kTile * 4u, io.vi + e0, sbytes, bar);
+    }
+}
+
+// The producer thread of the chunked kernel.  Flat: tile i is [va + i kTile,
+// ...) of the vector body [va, vb).  List: tiles are numbered across the
+// tensors' vector bodies (tab.tiles).  Every tile takes ceil(R/8) stages.
+template <class G, bool LIST>
+__device__ __forceinline__ void chunk_produce(const StepParams& p, uint64_t va, uint64_t vb, uint64_t* full,
+                                              uint64_t* empty, ChunkDesc* desc, unsigned char* ring) {
+    using Sh = ChunkShape<G>;
+    constexpr uint32_t D = (uint32_t)Sh::kStages;
+    const StateIO io = state_io(p);
+    const Table& t = p.tab;
+    const uint32_t C = (p.R + kChunkRanks - 1u) / kChunkRanks;
+    const uint64_t ntiles = LIST ? t.tiles[t.T] : (uint64_t)flat_tile_count(va, vb);
+    const void* const* gp = &p.grads[0];
+    void* params = p.params16;
+    uint64_t t0 = 0, bb = vb, tfirst = 0;
+    uint32_t j = 0xFFFFFFFFu, jn = 0;
+    uint64_t tile = blockIdx.x;
+    if (LIST && tile < ntiles) jn = find_tensor_by_tile(t, tile);
+    uint32_t k = 0;
+    bool ok = true;
+    for (;;) {
+        const bool have = tile < ntiles;
+        uint64_t next = 0;
+        uint64_t e0 = 0;
+        uint32_t n = 0;
+        if (have) {
+            next = (uint64_t)gridDim.x + atomicAdd(&p.ws->next_tile, 1u);  // one claim ahead
+            if constexpr (LIST) {
+                while (t.tiles[jn + 1] <= tile) ++jn;
+                if (jn != j) {
+                    j = jn;
+                    gp = t.grads + (uint64_t)j * p.R;
+                    params = t.params[j];
+                    t0 = t.offs[j];
+                    bb = t.offs[j + 1] & ~7ull;
+                    tfirst = t.tiles[j];
+                }
+                e0 = t0 + (tile - tfirst) * kTile;
+            } else {
+                e0 = va + tile * kTile;
+            }
+            n = (uint32_t)((bb - e0) < (uint64_t)kTile ? (bb - e0) : (uint64_t)kTile);
+        }
+        const uint32_t stages = have ? C : 1u;  // past the last tile: one end marker
+        for (uint32_t c = 0; c < stages; ++c, ++k) {
+            const uint32_t st = k % D;
+            if (k >= D && !mbar_wait_bounded(&empty[st], ((k / D) - 1u) & 1u)) {
+                ok = false;
+                break;
+            }
+            if (!have) {
+                desc[st] = ChunkDesc{0ull, 0ull, nullptr, 0u, 0u};
+                mbar_arrive(&full[st]);
+            } else {
+                const uint32_t r0 = c * kChunkRanks;
+                const uint32_t rn = p.R - r0 < kChunkRanks ? p.R - r0 : kChunkRanks;
+                desc[st] = ChunkDesc{e0, t0, params, n, c};
+                chunk_issue<G>(io, gp, r0, rn, c + 1u == C, ring + st * Sh::kStage, &full[st], e0, e0 - t0, n);
+            }
+        }
+        if (!ok || !have) break;
+        tile = next;
+    }
+    if (!ok) {
+        // Do not leave while copies of this CTA may still land in its shared
+        // memory: wait (bounded) for the last chunk of every stage.
+        note_timeout();
+        for (uint32_t i = k > D ? k - D : 0u; i < k; ++i) (void)mbar_wait_bounded(&full[i % D], (i / D) & 1u);
+    }
+}
+
+// Adam on the four elements of a consumer thread after a tile's last chunk
+// (`st`: the stage's state part), and the stores: the arithmetic of
+// bulk_group after its reduction.
+template <class Pm, bool PUSH>
+__device__ __forceinline__ void chunk_update(const StepParams& p, const Scal& s, const double (&acc)[4],
+                                             const unsigned char* st, uint32_t q, uint64_t e, uint64_t le,
+                                             const StateIO& io, Pm* pp) {
+    const float4 w4 = *reinterpret_cast<const float4*>(st + q * 4u);
+    const float4 m4 = *reinterpret_cast<const float4*>(st + kTile * 4u + q * 4u);
+    const float4 v4 = *reinterpret_cast<const float4*>(st + 2u * kTile * 4u + q * 4u);
+    float w[4] = {w4.x, w4.y, w4.z, w4.w};
+    float m[4] = {m4.x, m4.y, m4.z, m4.w};
+    float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    float g[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        g[k] = (float)(acc[k] * s.inv_ws);
+        adam1(g[k], w[k], m[k], v[k], s);
+    }
+    __stcs(reinterpret_cast<float4*>(io.wo + e), make_float4(w[0], w[1], w[2], w[3]));
+    __stcs(reinterpret_cast<float4*>(io.mo + e), make_float4(m[0], m[1], m[2], m[3]));
+    __stcs(reinterpret_cast<float4*>(io.vo + e), make_float4(v[0], v[1], v[2], v[3]));
+    uint2 o;
+    o.x = pack2<Pm>(w[0], w[1]);
+    o.y = pack2<Pm>(w[2], w[3]);
+    __stcs(reinterpret_cast<uint2*>(pp + le), o);
+    if constexpr (PUSH)
+        for (uint32_t i = 0; i < p.npush; ++i) __stcs(reinterpret_cast<uint2*>(static_cast<Pm*>(p.push[i]) + le), o);
+    if (p.reduced != nullptr) __stcs(reinterpret_cast<float4*>(p.reduced + e), make_float4(g[0], g[1], g[2], g[3]));
+}
+
+// The consumer warps of the chunked kernel.
+template <class G, class Pm, bool PUSH>
+__device__ __forceinline__ void chunk_consume(const StepParams& p, uint64_t* full, uint64_t* empty,
+                                              const ChunkDesc* desc, const unsigned char* ring, bool& bad) {
+    using Sh = ChunkShape<G>;
+    constexpr uint32_t D = (uint32_t)Sh::kStages;
+    const StateIO io = state_io(p);
+    const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
+    const uint32_t C = (p.R + kChunkRanks - 1u) / kChunkRanks;
+    const uint32_t q = 4u * threadIdx.x;
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (uint32_t k = 0;; ++k) {
+        const uint32_t st = k % D;
+        if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
+            note_timeout();
+            break;
+        }
+        const ChunkDesc d = desc[st];
+        if (d.n == 0u) break;
+        const unsigned char* stage = ring + st * Sh::kStage;
+        if (d.chunk == 0u) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] = 0.0;
+        }
+        if (q < d.n) {
+            const uint32_t r0 = d.chunk * kChunkRanks;
+            const uint32_t rn = p.R - r0 < kChunkRanks ? p.R - r0 : kChunkRanks;
+            for (uint32_t r = 0; r < rn; ++r) {
+                const Raw4<G> raw = lds4<G>(stage + r * Sh::kGradSlice + q * sizeof(G));
+                if (p.check == 1) bad |= bad4(raw);
+                float f[4];
+                unpack4(raw, f);
+                const double c = p.wt[r0 + r];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] = fma(c, (double)f[i], acc[i]);
+            }
+            if (d.chunk + 1u == C)
+                chunk_update<Pm, PUSH>(p, s, acc, stage + kChunkRanks * Sh::kGradSlice, q, d.e0 + q,
+                                       d.e0 - d.toff + q, io, static_cast<Pm*>(d.params));
+        }
+        __syncwarp();
+        if ((threadIdx.x & 31u) == 0u) mbar_arrive(&empty[st]);
+    }
+}
+
+// Flat calls (PUSH as in step_bulk_kernel) and list calls over the whole
+// vector, any number of gradient buffers.
+template <class G, class Pm, bool LIST, bool PUSH = false>
+__global__ void __launch_bounds__(kBulkThreads, 1) step_chunked_kernel(const __grid_constant__ StepParams p) {
+    static_assert(!(LIST && PUSH), "parameter push is for flat calls");
+    using Sh = ChunkShape<G>;
+    constexpr int D = Sh::kStages;
+    constexpr uint32_t kConsumerWarps = kConsumers / 32;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = reinterpret_cast<uint64_t*>(smem + 64);
+    ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + 128);
+    unsigned char* ring = smem + kBarBytes + kGpBytes;
+    __shared__ const void* s_gp[LIST ? ZERO_MAX_RANKS : 1];  // a tensor's gradient bases (scalar pass)
+    __shared__ StepStart s_start;
+
+    const bool work = p.lo < p.hi;
+    if (threadIdx.x == 0) {
+        s_timed_out = 0u;
+        if (work) {
+            for (int i = 0; i < D; ++i) {
+                mbar_init(&full[i], 1u);
+                mbar_init(&empty[i], kConsumerWarps);
+            }
+            fence_mbar_init();
+        }
+    }
+    grid_dependency_wait();
+    allow_dependents();
+    bool skip = false;
+    if (p.check == 2) skip = *reinterpret_cast<volatile const unsigned*>(&p.ws->found) != 0u;
+    bool bad = false;
+    if (!skip && work) {
+        __syncthreads();
+        if (threadIdx.x == 0) s_start = StepStart{*p.ctrl, p.ws->found};
+        const uint64_t va = (p.lo + 7) & ~7ull, vb = p.hi & ~7ull;
+        if (threadIdx.x == kConsumers) {
+            chunk_produce<G, LIST>(p, va, vb, full, empty, desc, ring);
+        } else if (threadIdx.x < kConsumers) {
+            chunk_consume<G, Pm, PUSH>(p, full, empty, desc, ring, bad);
+        } else if (!LIST && blockIdx.x == gridDim.x - 1) {
+            const StateIO io = state_io(p);
+            const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
+            flat_ends<G, Pm, 0, PUSH>(p, s, io, threadIdx.x - kConsumers - 1u, bad);
+        }
+        if constexpr (LIST) {
+            // Ragged heads and tails, and tensors that cannot take the vector path.
+            __syncthreads();
+            uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
+            uint64_t b = a + p.chunk;
+            if (a < p.lo) a = p.lo;
+            if (b > p.hi) b = p.hi;
+            const StateIO io = state_io(p);
+            const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
+            if (a < b) list_scalar_whole<G, Pm, 0>(p, s, a, b, io, bad, s_gp);
         }
     } else if (threadIdx.x == 0) {
         s_start = StepStart{*p.ctrl, p.ws->found};

@@ -132,9 +132,6 @@ def _args(**over):
     (dict(push_params16=[A, None]), za.ZERO_EINVAL),
     (dict(push_params16=[A]), za.ZERO_EINVAL),               # pushes need an owner
     (dict(path=3), za.ZERO_EINVAL),                          # unknown kernel path
-    (dict(path=za.ZERO_PATH_STAGED, R=3, grads=[A] * 3), za.ZERO_EINVAL),   # no staged kernel for 3
-    (dict(path=za.ZERO_PATH_STAGED, R=16, grads=[A] * 16, grad_dtype=za.ZERO_F32), za.ZERO_EINVAL),  # 16 x fp32
-    (dict(path=za.ZERO_PATH_STAGED, n_grads=3), za.ZERO_EINVAL),
     (dict(n_grads=300), za.ZERO_ERANGE),
     (dict(n_grads=2, rank_weights=[1, -1]), za.ZERO_EINVAL),      # weights over the n_grads buffers
     (dict(grad_offset=4, owner=1), za.ZERO_EALIGN),
@@ -161,6 +158,20 @@ def test_list_step_rejects_flat_buffers_and_mismatched_list():
     with pytest.raises(za.ZeroError) as e:
         za.zero_step_fused_list(a, lst)
     assert e.value.status == za.ZERO_EINVAL
+
+
+def test_list_step_for_one_owner_has_no_staged_kernel_for_other_rank_counts():
+    """A flat or whole-list step takes a staged kernel for any R (the chunked
+    one where no instance is compiled for R); a list step for one owner has
+    no chunked kernel, so ZERO_PATH_STAGED needs R in 1, 2, 4, 8 (16 with
+    16-bit gradients)."""
+    for R, gdt in ((3, za.ZERO_BF16), (16, za.ZERO_F32)):
+        lst = za.zero_tensor_list(table=A, P=1000, T=3, R=R, grad_dtype=gdt, param_dtype=za.ZERO_BF16,
+                                  table_bytes=za.zero_list_table_bytes(3, R))
+        a = _args(grads=None, params16=None, R=R, grad_dtype=gdt, owner=1, path=za.ZERO_PATH_STAGED)
+        with pytest.raises(za.ZeroError) as e:
+            za.zero_step_fused_list(a, lst)
+        assert e.value.status == za.ZERO_EINVAL
 
 
 def test_gather_and_ctrl_argument_errors():
