@@ -433,7 +433,8 @@ def roofline_kernel(workload: str, world: int = 1) -> str:
     step = name + (" (flat)" if kind == "flat" else " (list)")
     gas = GAS.get(workload, 0)
     if gas:
-        acc = "accum_bulk_kernel" if staged else "accum_kernel"
+        chunk_pays = R >= 9 if gdt == "f32" else R >= 6      # the library's rule for a workspace call
+        acc = "accum_bulk_kernel" if staged else ("accum_chunked_kernel" if chunk_pays else "accum_kernel")
         return f"{gas} x {acc} + step_bulk_kernel (flat, R = 1 f32)"
     return step
 

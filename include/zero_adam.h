@@ -471,15 +471,16 @@ typedef struct zero_accum_args {
 } zero_accum_args;
 
 /* Launches one kernel; asynchronous on `stream`.  The staged kernel
- * (ZERO_PATH_STAGED above) hands its tiles out dynamically; here it needs a
- * workspace and ctrl and R = 1, 2, 4, 8 or (16-bit gradients) 16.  The
- * register kernel
- * streams through registers and touches neither workspace nor ctrl.  Both
- * give bitwise identical sums.  ZERO_PATH_AUTO takes the staged kernel
- * whenever it is possible (the faster one at nearly every size), else the
- * register kernel.  Errors:
+ * (ZERO_PATH_STAGED above: the instance compiled for R, else the ranks
+ * streamed eight at a time) hands its tiles out dynamically; here it needs a
+ * workspace and ctrl.  The register kernel streams through registers and
+ * touches neither workspace nor ctrl.  Both give bitwise identical sums.
+ * ZERO_PATH_AUTO takes the staged kernel when a workspace is given and the
+ * staged kernel is the faster one: an instance compiled for R, or the
+ * chunked kernel from R = 6 on (16-bit gradients) or R = 9 on (fp32), which
+ * pays a fixed cost per tile; else the register kernel.  Errors:
  * ZERO_EINVAL (also: exactly one of workspace and ctrl given; an unknown
- * path; ZERO_PATH_STAGED without a workspace or with another R),
+ * path; ZERO_PATH_STAGED without a workspace),
  * ZERO_EALIGN (accum, grads and workspace must be 16-byte aligned, ctrl
  * 8-byte aligned), ZERO_ERANGE (R > ZERO_MAX_RANKS, P > ZERO_MAX_ELEMENTS),
  * ZERO_EOVERFLOW, ZERO_ECUDA. */

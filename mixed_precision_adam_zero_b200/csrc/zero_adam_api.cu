@@ -202,9 +202,10 @@ const void* gather_fn(int32_t param_dtype) {
                                     : (const void*)gather_kernel<__half, LIST>;
 }
 
-// Accumulation: the bulk kernel for a compile-time rank count when the
-// caller gives a workspace, else the register kernel.  Measured on a B200
-// (R = 8 bf16, a window of one first and three continuing micro-batches):
+// Accumulation: when the caller gives a workspace, the bulk kernel compiled
+// for R or, for any other R, the chunked one; else the register kernel.
+// Measured on a B200 (R = 8 bf16, a window of one first and three continuing
+// micro-batches):
 // the staged kernel is 10 % faster at 4.2M elements, 4 % at 6.3M, equal at
 // 10.5M, 3 % faster at 12.6M and 7 % at 16.8M; only near 8.4M is the
 // register kernel ahead (4 %).
@@ -226,6 +227,8 @@ Kern accum_kern_rc(uint32_t R, bool bulk) {
                 break;
             default: break;
         }
+        // any other rank count: the ranks streamed eight at a time
+        return Kern{(const void*)accum_chunked_kernel<G>, AccumChunkShape<G>::kSmem, kBulkThreads};
     }
     switch (R) {
         case 1: return Kern{(const void*)accum_kernel<G, 1>, 0u, kThreads};
@@ -631,7 +634,14 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     if ((a->workspace == nullptr) != (a->ctrl == nullptr)) return ZERO_EINVAL;
     if (a->path != ZERO_PATH_AUTO && a->path != ZERO_PATH_REGISTER && a->path != ZERO_PATH_STAGED)
         return ZERO_EINVAL;
-    const bool can_stage = a->workspace != nullptr && has_staged(a->R, a->grad_dtype);
+    const bool can_stage = a->workspace != nullptr;  // a staged instance, or the chunked kernel
+    // AUTO takes the chunked kernel only where it measured faster than the
+    // register kernel on a B200: it pays a fixed cost per tile, so a tile has
+    // to carry enough gradient bytes (16-bit gradients from R = 6 on, fp32
+    // from R = 9 on; 67M elements: bf16 R = 3 0.72 vs 0.78 of the copy peak,
+    // R = 6 0.87 vs 0.75, R = 32 0.86 vs 0.70, fp32 R = 3 0.82 vs 0.94,
+    // R = 16 1.06 vs 1.01).
+    const bool chunk_pays = a->grad_dtype == ZERO_F32 ? a->R >= 9u : a->R >= 6u;
     if (a->path == ZERO_PATH_STAGED && !can_stage) return ZERO_EINVAL;
     if (!aligned16(a->workspace) || (reinterpret_cast<uintptr_t>(a->ctrl) & 7u) != 0) return ZERO_EALIGN;
     AccumParams ap;
@@ -669,7 +679,8 @@ int zero_accumulate_grads(const zero_accum_args* a, void* stream) {
     if (ap.lo >= ap.hi) return ZERO_OK;
     if (a->accum_offset > ap.lo) return ZERO_EINVAL;
     int err = ZERO_OK;
-    const bool staged = a->path == ZERO_PATH_STAGED || (a->path == ZERO_PATH_AUTO && can_stage);
+    const bool staged = a->path == ZERO_PATH_STAGED ||
+                        (a->path == ZERO_PATH_AUTO && can_stage && (has_staged(a->R, a->grad_dtype) || chunk_pays));
     const Kern k = accum_kern(a->grad_dtype, a->R, staged);
     const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;

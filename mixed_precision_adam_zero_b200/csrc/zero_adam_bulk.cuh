@@ -1083,6 +1083,166 @@ __global__ void __launch_bounds__(kBulkThreads, 1) accum_bulk_kernel(const __gri
     finish_accum(p);
 }
 
+// Accumulation for rank counts without a staged instance: the tiles of the
+// vector body as in accum_bulk_kernel, each passed through the ring as
+// ceil(R/8) stages of up to eight ranks' gradient slices, the last stage also
+// holding the accumulator slice when the window continues.  The float64
+// sums stay in registers across a tile's chunks, so the result is bitwise
+// accum_vec's.
+template <class G>
+using AccumChunkShape = AccumShape<G, (int)kChunkRanks>;
+
+template <class G>
+__global__ void __launch_bounds__(kBulkThreads, 1) accum_chunked_kernel(const __grid_constant__ AccumParams p) {
+    using Sh = AccumChunkShape<G>;
+    constexpr uint32_t D = (uint32_t)Sh::kStages;
+    constexpr uint32_t kConsumerWarps = kConsumers / 32;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = reinterpret_cast<uint64_t*>(smem + 64);
+    ChunkDesc* desc = reinterpret_cast<ChunkDesc*>(smem + 128);
+    unsigned char* ring = smem + kBarBytes + kGpBytes;
+    // the rank weights, read from shared memory (a parameter array indexed at
+    // run time would be a memory load on the critical path of every stage)
+    __shared__ double s_wt[ZERO_MAX_RANKS];
+    for (uint32_t r = threadIdx.x; r < p.R; r += kBulkThreads) s_wt[r] = p.wt[r];
+    if (threadIdx.x == 0) {
+        s_timed_out = 0u;
+        for (uint32_t i = 0; i < D; ++i) {
+            mbar_init(&full[i], 1u);
+            mbar_init(&empty[i], kConsumerWarps);
+        }
+        fence_mbar_init();
+    }
+    grid_dependency_wait();
+    allow_dependents();
+    __syncthreads();
+    const uint64_t va = (p.lo + 7) & ~7ull;
+    const uint64_t vb = p.hi & ~7ull;
+    const uint32_t C = (p.R + kChunkRanks - 1u) / kChunkRanks;
+    if (threadIdx.x == kConsumers) {
+        const G* gb1[kChunkRanks];  // R <= 8: the rank pointers, once
+#pragma unroll
+        for (uint32_t r = 0; r < kChunkRanks; ++r) gb1[r] = r < p.R ? static_cast<const G*>(p.grads[r]) : nullptr;
+        const uint64_t ntiles = flat_tile_count(va, vb);
+        uint64_t tile = blockIdx.x;
+        uint32_t k = 0;
+        bool ok = true;
+        for (;;) {
+            const bool have = tile < ntiles;
+            uint64_t next = 0, e0 = 0;
+            uint32_t n = 0;
+            if (have) {
+                next = (uint64_t)gridDim.x + atomicAdd(&p.ws->next_tile, 1u);  // one claim ahead
+                e0 = va + tile * kTile;
+                n = (uint32_t)((vb - e0) < (uint64_t)kTile ? (vb - e0) : (uint64_t)kTile);
+            }
+            const uint32_t stages = have ? C : 1u;  // past the last tile: one end marker
+            for (uint32_t c = 0; c < stages; ++c, ++k) {
+                const uint32_t st = k % D;
+                if (k >= D && !mbar_wait_bounded(&empty[st], ((k / D) - 1u) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                if (!have) {
+                    desc[st] = ChunkDesc{0ull, 0ull, nullptr, 0u, 0u};
+                    mbar_arrive(&full[st]);
+                } else {
+                    const uint32_t r0 = c * kChunkRanks;
+                    const uint32_t rn = p.R - r0 < kChunkRanks ? p.R - r0 : kChunkRanks;
+                    const bool load_acc = c + 1u == C && !p.first;
+                    desc[st] = ChunkDesc{e0, 0ull, nullptr, n, c};
+                    unsigned char* stage = ring + st * Sh::kStage;
+                    const uint32_t gbytes = n * (uint32_t)sizeof(G);
+                    mbar_expect_tx(&full[st], rn * gbytes + (load_acc ? n * 4u : 0u));
+                    if (C == 1u) {
+#pragma unroll
+                        for (uint32_t r = 0; r < kChunkRanks; ++r)
+                            if (r < rn) bulk_g2s(stage + r * Sh::kGradSlice, gb1[r] + e0, gbytes, &full[st]);
+                    } else {
+                        for (uint32_t r = 0; r < rn; ++r)
+                            bulk_g2s(stage + r * Sh::kGradSlice, static_cast<const G*>(p.grads[r0 + r]) + e0,
+                                     gbytes, &full[st]);
+                    }
+                    if (load_acc) bulk_g2s(stage + kChunkRanks * Sh::kGradSlice, p.acc + e0, n * 4u, &full[st]);
+                }
+            }
+            if (!ok || !have) break;
+            tile = next;
+        }
+        if (!ok) {
+            // Do not leave while copies of this CTA may still land in its
+            // shared memory: wait (bounded) for the last use of every stage.
+            note_timeout();
+            for (uint32_t i = k > D ? k - D : 0u; i < k; ++i) (void)mbar_wait_bounded(&full[i % D], (i / D) & 1u);
+        }
+    } else if (threadIdx.x < kConsumers) {
+        const uint32_t q = 4u * threadIdx.x;
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
+        double w1[kChunkRanks];  // R <= 8: the weights, once
+#pragma unroll
+        for (uint32_t r = 0; r < kChunkRanks; ++r) w1[r] = r < p.R ? s_wt[r] : 0.0;
+        for (uint32_t k = 0;; ++k) {
+            const uint32_t st = k % D;
+            if (!mbar_wait_bounded(&full[st], (k / D) & 1u)) {
+                note_timeout();
+                break;
+            }
+            const ChunkDesc d = desc[st];
+            if (d.n == 0u) break;
+            const unsigned char* stage = ring + st * Sh::kStage;
+            if (d.chunk == 0u) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] = 0.0;
+            }
+            if (q < d.n) {
+                const uint32_t r0 = d.chunk * kChunkRanks;
+                const uint32_t rn = p.R - r0 < kChunkRanks ? p.R - r0 : kChunkRanks;
+                // all of the chunk's loads first, then the sums in rank order
+                Raw4<G> raw[kChunkRanks];
+                double wc[kChunkRanks];
+#pragma unroll
+                for (uint32_t r = 0; r < kChunkRanks; ++r) {
+                    if (r < rn) {
+                        raw[r] = lds4<G>(stage + r * Sh::kGradSlice + q * sizeof(G));
+                        wc[r] = C == 1u ? w1[r] : s_wt[r0 + r];
+                    }
+                }
+#pragma unroll
+                for (uint32_t r = 0; r < kChunkRanks; ++r) {
+                    if (r < rn) {
+                        float f[4];
+                        unpack4(raw[r], f);
+                        const double c = wc[r];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc[i] = fma(c, (double)f[i], acc[i]);
+                    }
+                }
+                if (d.chunk + 1u == C) {
+                    float4 a4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (!p.first) a4 = *reinterpret_cast<const float4*>(stage + kChunkRanks * Sh::kGradSlice + q * 4u);
+                    const float prev[4] = {a4.x, a4.y, a4.z, a4.w};
+                    float out[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) out[i] = (float)((double)prev[i] + p.scale * (acc[i] * p.inv_wsum));
+                    __stcs(reinterpret_cast<float4*>(p.acc + d.e0 + q), make_float4(out[0], out[1], out[2], out[3]));
+                }
+            }
+            __syncwarp();
+            if ((threadIdx.x & 31u) == 0u) mbar_arrive(&empty[st]);
+        }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {
+        const GradPtrs<G, 0> gp(&p.grads[0]);
+        uint64_t ha = va > p.hi ? p.hi : va;
+        uint64_t tb = vb < ha ? ha : vb;
+        for (uint64_t e = p.lo + threadIdx.x; e < ha; e += kBulkThreads) accum_elem<G, 0>(p, gp, e);
+        for (uint64_t e = tb + threadIdx.x; e < p.hi; e += kBulkThreads) accum_elem<G, 0>(p, gp, e);
+    }
+    finish_accum(p);
+}
+
 // ------------------------------------------------------------ timeout health check
 
 // One thread waits on a barrier that nothing arrives at; the bounded wait

@@ -276,9 +276,6 @@ def test_pushes_need_an_owner():
     (dict(workspace=A, ctrl=A + 4), za.ZERO_EALIGN),
     (dict(path=3), za.ZERO_EINVAL),
     (dict(path=za.ZERO_PATH_STAGED), za.ZERO_EINVAL),                 # staged needs a workspace
-    (dict(R=3, grads=[A] * 3, workspace=A, ctrl=A, path=za.ZERO_PATH_STAGED), za.ZERO_EINVAL),
-    (dict(R=16, grads=[A] * 16, grad_dtype=za.ZERO_F32, workspace=A, ctrl=A, path=za.ZERO_PATH_STAGED),
-     za.ZERO_EINVAL),
     (dict(accum_offset=4, owner=1), za.ZERO_EALIGN),
     (dict(accum_offset=256, owner=1), za.ZERO_EINVAL),               # beyond owner 1's first element (250)
 ])
