@@ -158,6 +158,20 @@ def test_fp16_skip_list(two_set):
     _run_fp16(two_set, lst=True)
 
 
+@pytest.mark.parametrize("R", [3, 13])
+@pytest.mark.parametrize("two_set", [False, True])
+@pytest.mark.parametrize("lst", [False, True])
+def test_fp16_skip_with_chunked_rank_counts(R, two_set, lst):
+    """Rank counts without a compiled staged instance (the chunked kernel:
+    R = 3 is one chunk of ranks, R = 13 two): infs at steps 3 and 10 sit in
+    ranks 3 mod R and 10 mod R, so at R = 13 one lands in each chunk; the
+    in-pass flag (two-set) and the scan pass (in place) skip like the
+    oracle."""
+    z, st = _run_fp16(two_set, R=R, lst=lst, steps=11, bad_steps=(3, 10))
+    c = z.ctrl()
+    assert c.skipped == 2 and c.step == 9 and c.loss_scale == 16384.0
+
+
 def test_fp16_skip_with_loss_scale_growth():
     # growth every 2 applied steps (parity unpinned by the pages: checked
     # against the oracle's reading only)
