@@ -80,14 +80,25 @@ WORKLOADS = {
     "sweep256m": ("flat", 1 << 28, 8, "bf16", "bf16", False),
     "sweep1b": ("flat", 1 << 30, 8, "bf16", "bf16", False),
     "sweep3p2b": ("flat", LLAMA3B_P, 8, "bf16", "bf16", False),
+    # other rank counts: R = 16 (a compiled staged instance for 16-bit
+    # gradients) and counts the chunked kernel takes (ranks eight at a time)
+    "flat64m_r16": ("flat", 1 << 26, 16, "bf16", "bf16", False),
+    "flat64m_r3": ("flat", 1 << 26, 3, "bf16", "bf16", False),
+    "flat64m_r12": ("flat", 1 << 26, 12, "bf16", "bf16", False),
+    "flat64m_r32": ("flat", 1 << 26, 32, "bf16", "bf16", False),
+    "flat64m_r16_f32": ("flat", 1 << 26, 16, "f32", "bf16", False),
+    "llama3b_layer_r3": ("list", "llama3b_layer", 3, "bf16", "bf16", False),
 }
 GRAD_BYTES = {"bf16": 2, "f16": 2, "f32": 4}
 
 # Gradient-accumulation workloads: micro-batches per update.  Each micro-batch
 # of R rank gradients is reduced into an fp32 accumulation array, and the
 # update is one fused step (R = 1, fp32) over that array.
-GAS = {"flat16m_gas4": 4}
+GAS = {"flat16m_gas4": 4, "flat64m_r6_gas4": 4, "flat64m_r32_gas4": 4}
 WORKLOADS["flat16m_gas4"] = ("flat", 16_777_259, 8, "bf16", "bf16", False)
+# the chunked accumulation (rank counts without a compiled staged instance)
+WORKLOADS["flat64m_r6_gas4"] = ("flat", 1 << 26, 6, "bf16", "bf16", False)
+WORKLOADS["flat64m_r32_gas4"] = ("flat", 1 << 26, 32, "bf16", "bf16", False)
 # ZeRO-3 module gather: full padded 16-bit views of every GPT-2-medium tensor
 # from R = 4 rank shards (2 bytes read and 2 written per padded element).
 WORKLOADS["gpt2m_z3gather"] = ("z3gather", "gpt2m", 4, "bf16", "bf16", False)
