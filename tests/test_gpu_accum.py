@@ -98,8 +98,11 @@ def test_staged_and_register_kernels_agree_bitwise(gdt, R):
     assert not ws.any() and not ctrl.any()
 
 
-def test_staged_per_owner_equals_whole_bitwise():
-    P, R = 9 * 2048 + 77, 4
+@pytest.mark.parametrize("R", [4, 6, 13])
+def test_staged_per_owner_equals_whole_bitwise(R):
+    """Per-owner staged calls (compiled for R = 4; the chunked kernel for 6
+    and 13) against one register call over the whole vector."""
+    P = 9 * 2048 + 77
     g = _micro(P, R, torch.bfloat16, 90)
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     ctrl = torch.zeros(64, dtype=torch.uint8, device="cuda")
