@@ -19,6 +19,11 @@
 // that of step_kernel (adam1 and the float64 rank reduction), so the two
 // kernels give bitwise identical results.
 //
+// Instances are compiled for R = 1, 2, 4, 8 (and 16 with 16-bit gradients):
+// their R loads are unrolled into registers.  Any other R takes the chunked
+// kernels at the end of the file, which pass each tile through the ring in
+// stages of eight ranks.
+//
 // Waits on the stage barriers are bounded (by %globaltimer): a wait that
 // gives up marks the CTA as timed out, the CTA stops consuming, waits (again
 // bounded) for the copies it issued, and finishes normally; the grid's
