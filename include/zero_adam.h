@@ -139,8 +139,7 @@ typedef struct zero_ctrl {
  *                      instance is compiled for 1, 2, 4 and 8 gradient
  *                      buffers, and for 16 with 16-bit gradients; for any
  *                      other count the step streams each tile's ranks through
- *                      the stages eight at a time (flat calls and list calls
- *                      over the whole vector; not a list call for one owner);
+ *                      the stages eight at a time;
  *   ZERO_PATH_REGISTER every thread reads its gradients with plain 16-byte
  *                      global loads (ld.global) into registers; any count;
  *   ZERO_PATH_AUTO     the staged kernel wherever it can run (the faster one
@@ -370,8 +369,7 @@ int zero_selftest_wait_timeout(void *ctrl, void *stream);
  * kernel that, only if the step was skipped, re-casts the 16-bit parameters
  * from the untouched master set.
  * The step kernel is the one args->path selects; an unknown path is
- * ZERO_EINVAL, and so is ZERO_PATH_STAGED for a list call for one owner with
- * a gradient-buffer count other than 1, 2, 4, 8 or (16-bit gradients) 16.
+ * ZERO_EINVAL.
  * Errors: ZERO_EINVAL, ZERO_EALIGN, ZERO_ERANGE (R > ZERO_MAX_RANKS, or
  * P > ZERO_MAX_ELEMENTS), ZERO_EOVERFLOW (P*8 bytes overflow), ZERO_ECUDA. */
 int zero_step_fused(const zero_step_args *args, void *stream);

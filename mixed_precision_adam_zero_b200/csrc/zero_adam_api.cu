@@ -118,10 +118,10 @@ int launch(const void* fn, const Shape& sh, void* params, cudaStream_t st, unsig
 // ------------------------------------------------------------ kernel tables
 
 // Calls with a compiled rank count stage their tiles through shared memory
-// with bulk copies (step_bulk_kernel); flat calls and whole-list calls with
-// any other count stream each tile's ranks through the same kind of ring,
-// eight at a time (step_chunked_kernel); the register kernel takes the rest
-// and every call that asks for it.  PUSH: flat calls that also store the
+// with bulk copies (step_bulk_kernel); calls with any other count stream each
+// tile's ranks through the same kind of ring, eight at a time
+// (step_chunked_kernel); the register kernel takes every call that asks for
+// it.  PUSH: flat calls that also store the
 // 16-bit values into other replicas.
 enum class StepKind { Register, Staged, Chunked };
 
@@ -172,15 +172,13 @@ bool has_staged(uint32_t R, int32_t grad_dtype) {
 }
 
 // The step kernel for a path (ZERO_PATH_*): AUTO and STAGED take the staged
-// instance compiled for R, else (flat calls, whole-list calls) the chunked
-// kernel; a list call for one owner with another R, and REGISTER, take the
-// register kernel.
-Kern step_kern(bool list, bool whole, bool push, int32_t grad_dtype, int32_t param_dtype, uint32_t R,
-               uint32_t path) {
+// instance compiled for R, else the chunked kernel; REGISTER the register
+// kernel.
+Kern step_kern(bool list, bool push, int32_t grad_dtype, int32_t param_dtype, uint32_t R, uint32_t path) {
     StepKind kind = StepKind::Register;
     if (path != ZERO_PATH_REGISTER) {
         if (has_staged(R, grad_dtype)) kind = StepKind::Staged;
-        else if (!list || whole) kind = StepKind::Chunked;
+        else kind = StepKind::Chunked;
     }
     if (list) return step_kern_gd<true, false>(grad_dtype, param_dtype, R, kind);
     return push ? step_kern_gd<false, true>(grad_dtype, param_dtype, R, kind)
@@ -387,7 +385,7 @@ int run_step(const zero_step_args* a, StepParams* kp, cudaStream_t st) {
     } else {
         kp->check = check ? 1 : 0;
     }
-    const Kern k = step_kern(LIST, kp->whole != 0, kp->npush > 0, a->grad_dtype, a->param_dtype, kp->R, a->path);
+    const Kern k = step_kern(LIST, kp->npush > 0, a->grad_dtype, a->param_dtype, kp->R, a->path);
     const int ctas = resident_ctas(k.fn, &err, k.smem, k.threads);
     if (err) return err;
     const Shape sh = make_shape(lo, hi, ctas);
@@ -614,8 +612,6 @@ int zero_step_fused_list(const zero_step_args* a, const zero_tensor_list* l, voi
         return ZERO_EINVAL;  // multi-GPU fields: flat calls only
     if (a->P != l->P || a->R != l->R || a->grad_dtype != l->grad_dtype || a->param_dtype != l->param_dtype)
         return ZERO_EINVAL;
-    // A list call for one owner has no chunked kernel: STAGED needs a compiled R.
-    if (a->path == ZERO_PATH_STAGED && a->owner >= 0 && !has_staged(a->R, a->grad_dtype)) return ZERO_EINVAL;
     kp.tab = device_table(l);
     kp.whole = a->owner < 0 ? 1 : 0;
     return run_step<true>(a, &kp, static_cast<cudaStream_t>(stream));

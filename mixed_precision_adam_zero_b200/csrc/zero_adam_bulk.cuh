@@ -326,8 +326,9 @@ __device__ __forceinline__ void bulk_scalar_pass(const StepParams& p, const Scal
                     if (bb < ba) bb = ba;
                 }
                 if (ba > x || bb < sb) {
+                    const uint32_t nr = RC > 0 ? (uint32_t)RC : p.R;  // RC == 0: the chunked kernel, any R
                     __syncthreads();
-                    for (uint32_t r = threadIdx.x; r < RC; r += kBulkThreads) s_gp[r] = p.tab.grads[(uint64_t)j * RC + r];
+                    for (uint32_t r = threadIdx.x; r < nr; r += kBulkThreads) s_gp[r] = p.tab.grads[(uint64_t)j * nr + r];
                     __syncthreads();
                     const GradPtrs<G, RC> gp(s_gp);
                     Pm* pp = static_cast<Pm*>(p.tab.params[j]);
@@ -723,10 +724,10 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_bulk_kernel(const __grid
 // keeps their float64 sums in registers from the first chunk to the last, so
 // the ranks are added in the order 0..R-1 as in the other kernels (the
 // results are bitwise theirs); the last chunk applies Adam.  Flat calls and
-// list calls over the whole vector (a list call for one owner takes the
-// register kernel).  Tiles are handed out as in flat_dynamic and
-// list_dynamic: CTA b starts on tile b and claims the rest from the
-// workspace counter one tile ahead.
+// list calls over the whole vector hand their tiles out as flat_dynamic and
+// list_dynamic do (CTA b starts on tile b and claims the rest from the
+// workspace counter one tile ahead); a list call for one owner walks each
+// CTA's own range, as list_static does.
 constexpr uint32_t kChunkRanks = 8;
 static_assert(4 * kConsumers == kTile, "one 4-element group per consumer thread per tile");
 
@@ -834,6 +835,52 @@ __device__ __forceinline__ void chunk_produce(const StepParams& p, uint64_t va, 
     }
 }
 
+// The producer thread of the chunked kernel for a list call for one owner:
+// CTA b walks its own contiguous range [a, b) of the concatenation, tile by
+// tile through the vector bodies of its tensors (TileWalk), each tile taking
+// ceil(R/8) stages as above.
+template <class G>
+__device__ __forceinline__ void chunk_produce_static(const StepParams& p, uint64_t a, uint64_t b, uint64_t* full,
+                                                     uint64_t* empty, ChunkDesc* desc, unsigned char* ring) {
+    using Sh = ChunkShape<G>;
+    constexpr uint32_t D = (uint32_t)Sh::kStages;
+    const StateIO io = state_io(p);
+    const uint32_t C = (p.R + kChunkRanks - 1u) / kChunkRanks;
+    TileWalk<G, 1, true, false> pw;
+    pw.start(p, a, b);
+    uint32_t k = 0;
+    bool ok = true;
+    for (;;) {
+        uint64_t e0 = 0;
+        uint32_t n = 0;
+        const bool have = pw.next(p, e0, n);
+        // the walk has just moved past the tile's tensor: its index is j - 1
+        const void* const* gp = have ? p.tab.grads + (uint64_t)(pw.j - 1u) * p.R : nullptr;
+        const uint32_t stages = have ? C : 1u;  // past the last tile: one end marker
+        for (uint32_t c = 0; c < stages; ++c, ++k) {
+            const uint32_t st = k % D;
+            if (k >= D && !mbar_wait_bounded(&empty[st], ((k / D) - 1u) & 1u)) {
+                ok = false;
+                break;
+            }
+            if (!have) {
+                desc[st] = ChunkDesc{0ull, 0ull, nullptr, 0u, 0u};
+                mbar_arrive(&full[st]);
+            } else {
+                const uint32_t r0 = c * kChunkRanks;
+                const uint32_t rn = p.R - r0 < kChunkRanks ? p.R - r0 : kChunkRanks;
+                desc[st] = ChunkDesc{e0, pw.toff, pw.params, n, c};
+                chunk_issue<G>(io, gp, r0, rn, c + 1u == C, ring + st * Sh::kStage, &full[st], e0, e0 - pw.toff, n);
+            }
+        }
+        if (!ok || !have) break;
+    }
+    if (!ok) {
+        note_timeout();
+        for (uint32_t i = k > D ? k - D : 0u; i < k; ++i) (void)mbar_wait_bounded(&full[i % D], (i / D) & 1u);
+    }
+}
+
 // Adam on the four elements of a consumer thread after a tile's last chunk
 // (`st`: the stage's state part), and the stores: the arithmetic of
 // bulk_group after its reduction.
@@ -910,8 +957,8 @@ __device__ __forceinline__ void chunk_consume(const StepParams& p, uint64_t* ful
     }
 }
 
-// Flat calls (PUSH as in step_bulk_kernel) and list calls over the whole
-// vector, any number of gradient buffers.
+// Flat calls (PUSH as in step_bulk_kernel) and list calls, over the whole
+// vector or for one owner, any number of gradient buffers.
 template <class G, class Pm, bool LIST, bool PUSH = false>
 __global__ void __launch_bounds__(kBulkThreads, 1) step_chunked_kernel(const __grid_constant__ StepParams p) {
     static_assert(!(LIST && PUSH), "parameter push is for flat calls");
@@ -926,7 +973,11 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_chunked_kernel(const __g
     __shared__ const void* s_gp[LIST ? ZERO_MAX_RANKS : 1];  // a tensor's gradient bases (scalar pass)
     __shared__ StepStart s_start;
 
-    const bool work = p.lo < p.hi;
+    uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;  // this CTA's range (list calls)
+    uint64_t b = a + p.chunk;
+    if (a < p.lo) a = p.lo;
+    if (b > p.hi) b = p.hi;
+    const bool work = (LIST && !p.whole) ? a < b : p.lo < p.hi;
     if (threadIdx.x == 0) {
         s_timed_out = 0u;
         if (work) {
@@ -947,7 +998,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_chunked_kernel(const __g
         if (threadIdx.x == 0) s_start = StepStart{*p.ctrl, p.ws->found};
         const uint64_t va = (p.lo + 7) & ~7ull, vb = p.hi & ~7ull;
         if (threadIdx.x == kConsumers) {
-            chunk_produce<G, LIST>(p, va, vb, full, empty, desc, ring);
+            if (LIST && !p.whole) chunk_produce_static<G>(p, a, b, full, empty, desc, ring);
+            else chunk_produce<G, LIST>(p, va, vb, full, empty, desc, ring);
         } else if (threadIdx.x < kConsumers) {
             chunk_consume<G, Pm, PUSH>(p, full, empty, desc, ring, bad);
         } else if (!LIST && blockIdx.x == gridDim.x - 1) {
@@ -958,13 +1010,12 @@ __global__ void __launch_bounds__(kBulkThreads, 1) step_chunked_kernel(const __g
         if constexpr (LIST) {
             // Ragged heads and tails, and tensors that cannot take the vector path.
             __syncthreads();
-            uint64_t a = p.base + (uint64_t)blockIdx.x * p.chunk;
-            uint64_t b = a + p.chunk;
-            if (a < p.lo) a = p.lo;
-            if (b > p.hi) b = p.hi;
             const StateIO io = state_io(p);
             const Scal s = make_scal(p.h, p.ctrl->step + 1ull, p.ctrl->loss_scale, p.wsum);
-            if (a < b) list_scalar_whole<G, Pm, 0>(p, s, a, b, io, bad, s_gp);
+            if (a < b) {
+                if (p.whole) list_scalar_whole<G, Pm, 0>(p, s, a, b, io, bad, s_gp);
+                else bulk_scalar_pass<G, Pm, 0, true>(p, s, a, b, io, bad, s_gp);
+            }
         }
     } else if (threadIdx.x == 0) {
         s_start = StepStart{*p.ctrl, p.ws->found};

@@ -160,20 +160,6 @@ def test_list_step_rejects_flat_buffers_and_mismatched_list():
     assert e.value.status == za.ZERO_EINVAL
 
 
-def test_list_step_for_one_owner_has_no_staged_kernel_for_other_rank_counts():
-    """A flat or whole-list step takes a staged kernel for any R (the chunked
-    one where no instance is compiled for R); a list step for one owner has
-    no chunked kernel, so ZERO_PATH_STAGED needs R in 1, 2, 4, 8 (16 with
-    16-bit gradients)."""
-    for R, gdt in ((3, za.ZERO_BF16), (16, za.ZERO_F32)):
-        lst = za.zero_tensor_list(table=A, P=1000, T=3, R=R, grad_dtype=gdt, param_dtype=za.ZERO_BF16,
-                                  table_bytes=za.zero_list_table_bytes(3, R))
-        a = _args(grads=None, params16=None, R=R, grad_dtype=gdt, owner=1, path=za.ZERO_PATH_STAGED)
-        with pytest.raises(za.ZeroError) as e:
-            za.zero_step_fused_list(a, lst)
-        assert e.value.status == za.ZERO_EINVAL
-
-
 def test_gather_and_ctrl_argument_errors():
     for call, status in [
         (lambda: za.zero_gather_params(A, A, za.ZERO_F32, 10), za.ZERO_EINVAL),

@@ -56,13 +56,13 @@ def test_per_owner_calls_equal_one_all_owner_call_bitwise(P, R):
         assert za.zero_ctrl_read(c).step == 3
 
 
+@pytest.mark.parametrize("R", [4, 3, 13])
 @pytest.mark.parametrize("misalign", [False, True])
-def test_list_per_owner_calls_equal_one_whole_call_bitwise(misalign):
+def test_list_per_owner_calls_equal_one_whole_call_bitwise(misalign, R):
     """The same comparison for a tensor list: the whole-vector call hands out
     tiles dynamically, per-owner calls walk their slice statically; both must
-    give bitwise the same state."""
+    give bitwise the same state (R = 3, 13: the chunked kernel)."""
     numels = [1000, 37, 4096 * 3 + 5, 0, 2048, 9, 50_000]
-    R = 4
     def make():
         if not misalign:
             return ListZero(numels, R, "bf16", "bf16")
