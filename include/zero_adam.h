@@ -142,8 +142,9 @@ typedef struct zero_ctrl {
  *                      the stages eight at a time;
  *   ZERO_PATH_REGISTER every thread reads its gradients with plain 16-byte
  *                      global loads (ld.global) into registers; any count;
- *   ZERO_PATH_AUTO     the staged kernel wherever it can run (the faster one
- *                      at nearly every size), else the register kernel.
+ *   ZERO_PATH_AUTO     the step: the staged kernel (the faster one at
+ *                      nearly every size); the accumulation: see
+ *                      zero_accumulate_grads.
  * Both give bitwise identical results.  Across GPUs the gradient buffers are
  * other GPUs' memory mapped into this process: ZERO_PATH_REGISTER then reads
  * them with ordinary peer loads instead of bulk copies. */
@@ -328,9 +329,9 @@ int zero_workspace_init(void *workspace, void *stream);
 
 /* Overflow scan of one gradient buffer: the inf/NaN check of the step with
  * loss scaling (given at the top of this file; the pages describe no loss
- * scaling), taken ahead of a step with check_nonfinite = 2: sets the workspace's inf/NaN
- * word if any of grad[0, n) is inf or NaN, and otherwise leaves it as it
- * is, so several scans accumulate.  grad: device, 16-byte aligned, of
+ * scaling), taken ahead of a step with check_nonfinite = 2: sets the
+ * workspace's inf/NaN word if any of grad[0, n) is inf or NaN, and otherwise
+ * leaves it as it is, so several scans accumulate.  grad: device, 16-byte aligned, of
  * grad_dtype.  Asynchronous on `stream`.  Errors: ZERO_EINVAL, ZERO_EALIGN,
  * ZERO_EOVERFLOW, ZERO_ECUDA. */
 int zero_scan_nonfinite(const void *grad, int32_t grad_dtype, uint64_t n, void *workspace, void *stream);
@@ -343,8 +344,8 @@ int zero_scan_nonfinite(const void *grad, int32_t grad_dtype, uint64_t n, void *
  * update, as a two-set step with the overflow check on and growth_interval 1
  * whose wait gave up: device_error = 1 and last_skipped = 1, with step,
  * skipped, parity, loss_scale and growth_tracker unchanged.  It then exits
- * normally: no trap, no fault, the context stays usable.  Asynchronous on `stream`; read the
- * result with zero_ctrl_read.  Errors: ZERO_EINVAL (NULL ctrl), ZERO_EALIGN
+ * normally: no trap, no fault, the context stays usable.  Asynchronous on
+ * `stream`; read the result with zero_ctrl_read.  Errors: ZERO_EINVAL (NULL ctrl), ZERO_EALIGN
  * (ctrl not 8-byte aligned), ZERO_ECUDA. */
 int zero_selftest_wait_timeout(void *ctrl, void *stream);
 
@@ -358,9 +359,10 @@ int zero_selftest_wait_timeout(void *ctrl, void *stream);
  * updated-parameter all-gather).  The reduction runs over ranks 0..R-1 in
  * that order as float64 fused multiply-adds of w_r times the gradient (both
  * exact in float64), is scaled by 1/(sum(w)*S) and rounded once to float32;
- * results are bitwise reproducible run to run.  Sources: "Reduce first, then update the owned
- * slice" and "Communication volume isn't elapsed time" ("Deep dive:
- * DeepSpeed"); the AdamW/fp16 configuration of the "ZeRO" documentation page.
+ * results are bitwise reproducible run to run.  Sources: "Reduce first, then
+ * update the owned slice" and "Communication volume isn't elapsed time"
+ * ("Deep dive: DeepSpeed"); the AdamW/fp16 configuration of the "ZeRO"
+ * documentation page.
  *
  * Launches: one kernel, except (a) check on, in place, or check on with
  * owner >= 0: a scan kernel over all R gradients first (the skip decision
