@@ -324,6 +324,18 @@ int zero_ctrl_set(void *ctrl, const zero_ctrl *value, void *stream);
  * stream. */
 int zero_ctrl_read(const void *ctrl, zero_ctrl *out, void *stream);
 
+/* Lets kernels on the current device read and write memory of GPU
+ * `peer_device` (cudaDeviceEnablePeerAccess from the current device).  A
+ * step whose grads or push_params16 are another GPU's buffers mapped into
+ * this process needs it for every such GPU before its first launch: a
+ * buffer mapped by CUDA IPC with its owner's device current (as PyTorch
+ * maps a shared CUDA tensor) is not otherwise reachable from this device.
+ * ZERO_OK also when peer_device is the current device or access is already
+ * enabled.  Host call, synchronous.  Errors: ZERO_EINVAL (peer_device < 0, or
+ * the two GPUs cannot access each other), ZERO_ERANGE (no such device),
+ * ZERO_ECUDA. */
+int zero_enable_peer_access(int32_t peer_device);
+
 /* Zero a workspace of ZERO_WORKSPACE_BYTES (cudaMemsetAsync). */
 int zero_workspace_init(void *workspace, void *stream);
 

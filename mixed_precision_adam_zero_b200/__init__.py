@@ -46,7 +46,7 @@ EXPORTED = [
     "zero_ctrl_set", "zero_ctrl_read", "zero_workspace_init", "zero_step_fused",
     "zero_step_fused_list", "zero_list_table_build", "zero_gather_params",
     "zero_gather_params_list", "zero_step_fused_noalloc", "zero_accumulate_grads", "zero_selftest_wait_timeout",
-    "zero_scan_nonfinite",
+    "zero_scan_nonfinite", "zero_enable_peer_access",
     "zero_checkpoint_save", "zero_checkpoint_load", "zero_checkpoint_consolidate", "zero_checkpoint_error",
     "zero3_shard_bounds", "zero_parameter_storage", "zero3_gather_list_build", "zero3_gather",
 ]
@@ -146,6 +146,7 @@ def _lib() -> ctypes.CDLL:
         L.zero_ctrl_read.argtypes = [vp, ctypes.POINTER(zero_ctrl), vp]
         L.zero_workspace_init.argtypes = [vp, vp]
         L.zero_selftest_wait_timeout.argtypes = [vp, vp]
+        L.zero_enable_peer_access.argtypes = [i32]
         L.zero_scan_nonfinite.argtypes = [vp, i32, u64, vp, vp]
         L.zero_step_fused.argtypes = [ctypes.POINTER(zero_step_args), vp]
         L.zero_step_fused_noalloc.argtypes = [ctypes.POINTER(zero_step_args), vp]
@@ -244,6 +245,11 @@ def zero_ctrl_read(ctrl, stream=None) -> zero_ctrl:
     out = zero_ctrl()
     _check(_lib().zero_ctrl_read(_ptr(ctrl), ctypes.byref(out), _stream(stream)), "zero_ctrl_read")
     return out
+
+
+def zero_enable_peer_access(peer_device: int) -> None:
+    """Kernels on the current device may access GPU `peer_device`'s memory."""
+    _check(_lib().zero_enable_peer_access(int(peer_device)), "zero_enable_peer_access")
 
 
 def zero_workspace_init(workspace, stream=None) -> None:

@@ -575,6 +575,25 @@ int zero_selftest_wait_timeout(void* ctrl, void* stream) {
     return launch((const void*)wait_timeout_probe_kernel, sh, &c, static_cast<cudaStream_t>(stream), 0, 32);
 }
 
+int zero_enable_peer_access(int32_t peer_device) {
+    if (peer_device < 0) return ZERO_EINVAL;
+    int dev = 0, count = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaGetDeviceCount(&count);
+    if (e != cudaSuccess) return zadam_record_cuda(e);
+    if (peer_device >= count) return ZERO_ERANGE;
+    if (peer_device == dev) return ZERO_OK;
+    int can = 0;
+    if ((e = cudaDeviceCanAccessPeer(&can, dev, peer_device)) != cudaSuccess) return zadam_record_cuda(e);
+    if (!can) return ZERO_EINVAL;
+    e = cudaDeviceEnablePeerAccess(peer_device, 0);
+    if (e == cudaErrorPeerAccessAlreadyEnabled) {
+        (void)cudaGetLastError();  // not an error here: clear it from the thread's state
+        return ZERO_OK;
+    }
+    return e == cudaSuccess ? ZERO_OK : zadam_record_cuda(e);
+}
+
 int zero_workspace_init(void* workspace, void* stream) {
     if (workspace == nullptr) return ZERO_EINVAL;
     if (!aligned16(workspace)) return ZERO_EALIGN;

@@ -40,8 +40,8 @@ from torch.multiprocessing.reductions import reduce_tensor
 
 from . import (ZERO_F32, ZERO_WORKSPACE_FOUND_OFFSET, check_ctrl, make_accum_args, make_step_args, zero_accumulate_grads,
                zero_checkpoint_load, zero_checkpoint_save, zero_ctrl_bytes, zero_ctrl_init, zero_ctrl_read,
-               zero_gather_params, zero_partition_bounds, zero_scan_nonfinite, zero_step_fused,
-               zero_workspace_bytes, zero_workspace_init)
+               zero_enable_peer_access, zero_gather_params, zero_partition_bounds, zero_scan_nonfinite,
+               zero_step_fused, zero_workspace_bytes, zero_workspace_init)
 from .buffers import DTYPES
 
 
@@ -153,6 +153,12 @@ class Zero2Rank:
         # Peer views of every rank's gradient and 16-bit parameters.
         exchange = peers if peers is not None else exchange_peer_tensors
         self.peer_grads, self.peer_params16 = exchange([self.grad, self.params16], group)
+        # A shared CUDA tensor is mapped with its owner's device current, so
+        # this device reaches the peers' buffers only with peer access on.
+        with torch.cuda.device(self.device):
+            for t in self.peer_grads + self.peer_params16:
+                if t.device != self.device:
+                    zero_enable_peer_access(t.device.index)
         torch.cuda.synchronize(self.device)
         self._barrier()
 

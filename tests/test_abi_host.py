@@ -160,6 +160,12 @@ def test_list_step_rejects_flat_buffers_and_mismatched_list():
     assert e.value.status == za.ZERO_EINVAL
 
 
+def test_enable_peer_access_rejects_a_negative_device_before_any_cuda_call():
+    with pytest.raises(za.ZeroError) as e:
+        za.zero_enable_peer_access(-1)
+    assert e.value.status == za.ZERO_EINVAL
+
+
 def test_gather_and_ctrl_argument_errors():
     for call, status in [
         (lambda: za.zero_gather_params(A, A, za.ZERO_F32, 10), za.ZERO_EINVAL),

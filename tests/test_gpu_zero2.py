@@ -283,6 +283,16 @@ def test_emulated_accumulation_shares_the_skip_decision():
 
 # ---------------------------------------------------------------- two processes, one GPU, CUDA IPC
 
+def test_enable_peer_access_on_one_gpu():
+    """The current device needs no peer access to itself; a device that does
+    not exist is refused before any CUDA peer call."""
+    dev = torch.cuda.current_device()
+    za.zero_enable_peer_access(dev)
+    with pytest.raises(za.ZeroError) as e:
+        za.zero_enable_peer_access(torch.cuda.device_count())
+    assert e.value.status == za.ZERO_ERANGE
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
