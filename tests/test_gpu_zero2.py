@@ -111,7 +111,7 @@ def test_emulated_ranks_equal_the_single_call_bitwise(R, path):
     _run(P=200_003, R=R, path=path)
 
 
-@pytest.mark.parametrize("R", [4, 8])
+@pytest.mark.parametrize("R", [4, 8, 3, 5, 16])     # 3, 5 (and 16 with fp32): the chunked kernel
 @pytest.mark.parametrize("gdt,pdt", [("f32", "bf16"), ("bf16", "f16"), ("f16", "f16")])
 def test_emulated_ranks_dtypes_and_token_weights(gdt, pdt, R):
     _run(P=100_019, R=R, gdt=gdt, pdt=pdt, token=True)
