@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 
 # ------------------------------------------------------------ ownership
 
-@pytest.mark.parametrize("P,R", [(40_009, 8), (13, 4), (3, 8), (40_009, 3), (40_009, 13)])
+@pytest.mark.parametrize("P,R", [(40_009, 8), (13, 4), (3, 8), (40_009, 3), (40_009, 13), (7, 13), (40_009, 33)])
 def test_per_owner_calls_equal_one_all_owner_call_bitwise(P, R):
     """The pages' sharded/unsharded comparison on the device: R calls, each
     updating only owner r's slice with owner r's own control block, give
