@@ -17,7 +17,8 @@ HEADER = os.path.join(ROOT, "include", "zero_adam.h")
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    with open(HEADER) as f:
+        text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(zero3?_\w+)\s*\(", text)))
 
@@ -317,7 +318,8 @@ def test_parameter_storage_matches_the_oracle_and_the_pages():
 
 def test_header_constants_match_the_binding():
     import re
-    text = open(os.path.join(ROOT, "include", "zero_adam.h")).read()
+    with open(os.path.join(ROOT, "include", "zero_adam.h")) as f:
+        text = f.read()
     defines = {m.group(1): int(m.group(2)) for m in
                re.finditer(r"^#define (ZERO_[A-Z0-9_]+) \(?(-?\d+)\)?", text, flags=re.M)}
     assert len(defines) >= 17

@@ -53,7 +53,8 @@ MUTANTS = [
 
 
 def _build_mutant(tmp, i, old, new):
-    src = open(SRC).read()
+    with open(SRC) as f:
+        src = f.read()
     assert src.count(old) >= 1, old
     c = os.path.join(tmp, f"m{i}.c")
     with open(c, "w") as f:
