@@ -102,6 +102,11 @@ WORKLOADS["flat64m_r32_gas4"] = ("flat", 1 << 26, 32, "bf16", "bf16", False)
 # ZeRO-3 module gather: full padded 16-bit views of every GPT-2-medium tensor
 # from R = 4 rank shards (2 bytes read and 2 written per padded element).
 WORKLOADS["gpt2m_z3gather"] = ("z3gather", "gpt2m", 4, "bf16", "bf16", False)
+# ZeRO-3 optimizer step on one GPU: each of the R = 4 ranks steps over its own
+# padded shards of the GPT-2-medium tensors (a list of its shard pieces),
+# reading every rank's full gradient at the shard offsets; the R rank steps
+# together update every parameter once.
+WORKLOADS["gpt2m_z3step"] = ("z3step", "gpt2m", 4, "bf16", "bf16", False)
 # The ZeRO-2 step across GPUs, emulated on one GPU: R owner launches, each over
 # its own state slice, reading every rank's gradient slice and storing its
 # 16-bit results into all R replicas (the pushes land in this GPU's HBM).
@@ -155,7 +160,7 @@ def tensor_list(name: str):
 def workload_P(name: str, world: int = 1) -> int:
     """Parameters one step updates (the padded elements for the ZeRO-3 gather)."""
     kind, size, R, gdt, pdt, scaled = WORKLOADS[name]
-    if kind == "list":
+    if kind in ("list", "z3step"):
         return sum(n for _, n in tensor_list(size))
     if kind == "z3gather":
         return sum(R * -(-n // R) for _, n in tensor_list(size))
@@ -347,6 +352,37 @@ def build_workload(name: str, device, stream, world: int = 1) -> Bench:
         return Bench(P=R * sum(shard), call=lambda: zero3_gather(gl, stream), inputs=sbufs, output=fbuf,
                      launches=1, ctrl=lambda: None, keep=(table, full))
 
+    if kind == "z3step":
+        from mixed_precision_adam_zero_b200 import zero3_shard_bounds
+        numels = [n for _, n in tensor_list(size)]
+        T, P = len(numels), sum(numels)
+        gbufs = [torch.empty(P, dtype=gt, device=device) for _ in range(R)]
+        for r, g in enumerate(gbufs):
+            synth.fill_normal_(g, 1e-3, synth.seed_for(wl, synth.KIND_GRAD, r, 1))
+        full = [list(g.split(numels)) for g in gbufs]             # every rank's gradient, per tensor
+        w0 = synth.normal(P, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device)
+        offs = [0]
+        for n in numels:
+            offs.append(offs[-1] + n)
+        bounds = [[zero3_shard_bounds(n, R, r) for n in numels] for r in range(R)]
+        shard_buf = torch.empty(sum(b[2] for br in bounds for b in br), dtype=pt, device=device)
+        pieces = list(shard_buf.split([b[2] for br in bounds for b in br]))   # rank-major padded shards
+        ranks = []
+        for r in range(R):
+            sizes = [hi - lo for lo, hi, _ in bounds[r]]
+            params = [pieces[r * T + j][:sizes[j]] for j in range(T)]
+            grads = [[full[q][j][bounds[r][j][0]:bounds[r][j][1]] for j in range(T)] for q in range(R)]
+            z = ListZero(sizes, R, gdt, pdt, device=device, stream=stream, params16=params, grads=grads)
+            z.load_master(torch.cat([w0[offs[j] + lo:offs[j] + hi] for j, (lo, hi, _) in enumerate(bounds[r])]))
+            ranks.append(z)
+        rank_args = [z.step_args(hp=ADAMW) for z in ranks]
+
+        def call():
+            for z, a in zip(ranks, rank_args):
+                zero_step_fused_list(a, z.list, stream)
+        return Bench(P=P, call=call, inputs=gbufs, output=shard_buf, launches=R, ctrl=ranks[0].ctrl,
+                     keep=(ranks, rank_args, full, pieces))
+
     if kind == "zero2emu":
         from mixed_precision_adam_zero_b200.zero2 import rank_slice
         w0 = synth.normal(size, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device)
@@ -435,6 +471,8 @@ def roofline_kernel(workload: str, world: int = 1) -> str:
         return "z3_gather_kernel"
     if kind == "zero2emu":
         return f"{R} x step_bulk_kernel (flat, push): the owners of an emulated {R}-rank ZeRO-2 step"
+    if kind == "z3step":
+        return f"{R} x step_bulk_kernel (list): the ZeRO-3 ranks' steps over their shards"
     staged = R in (1, 2, 4, 8) or (R == 16 and gdt != "f32")
     name = "step_bulk_kernel" if staged else "step_chunked_kernel"   # flat and whole-list calls: always staged
     if kind == "zero2":
