@@ -107,6 +107,9 @@ WORKLOADS["gpt2m_z3gather"] = ("z3gather", "gpt2m", 4, "bf16", "bf16", False)
 # reading every rank's full gradient at the shard offsets; the R rank steps
 # together update every parameter once.
 WORKLOADS["gpt2m_z3step"] = ("z3step", "gpt2m", 4, "bf16", "bf16", False)
+# zero_gather_params alone: the round-to-nearest-even cast of 1.07B fp32
+# masters into the replicated bf16 buffer (4 bytes read, 2 written).
+WORKLOADS["gather1b"] = ("gather", 1 << 30, 1, "bf16", "bf16", False)
 # The ZeRO-2 step across GPUs, emulated on one GPU: R owner launches, each over
 # its own state slice, reading every rank's gradient slice and storing its
 # 16-bit results into all R replicas (the pushes land in this GPU's HBM).
@@ -180,6 +183,8 @@ def workload_bpp(name: str, world: int = 1) -> int:
     R = workload_R(name, world)
     if kind == "z3gather":
         return 4
+    if kind == "gather":
+        return 6
     if kind == "zero2emu":
         return zero2emu_bytes_per_param(R, gdt)
     if kind == "zero2":
@@ -352,6 +357,13 @@ def build_workload(name: str, device, stream, world: int = 1) -> Bench:
         return Bench(P=R * sum(shard), call=lambda: zero3_gather(gl, stream), inputs=sbufs, output=fbuf,
                      launches=1, ctrl=lambda: None, keep=(table, full))
 
+    if kind == "gather":
+        from mixed_precision_adam_zero_b200 import zero_gather_params
+        master = synth.normal(size, 0.02, synth.seed_for(wl, synth.KIND_MASTER), device=device)
+        p16 = torch.empty(size, dtype=pt, device=device)
+        return Bench(P=size, call=lambda: zero_gather_params(master, p16, pcode, size, stream), inputs=[master],
+                     output=p16, launches=1, ctrl=lambda: None, keep=(master,))
+
     if kind == "z3step":
         from mixed_precision_adam_zero_b200 import zero3_shard_bounds
         numels = [n for _, n in tensor_list(size)]
@@ -473,6 +485,8 @@ def roofline_kernel(workload: str, world: int = 1) -> str:
         return f"{R} x step_bulk_kernel (flat, push): the owners of an emulated {R}-rank ZeRO-2 step"
     if kind == "z3step":
         return f"{R} x step_bulk_kernel (list): the ZeRO-3 ranks' steps over their shards"
+    if kind == "gather":
+        return "gather_kernel (flat): zero_gather_params"
     staged = R in (1, 2, 4, 8) or (R == 16 and gdt != "f32")
     name = "step_bulk_kernel" if staged else "step_chunked_kernel"   # flat and whole-list calls: always staged
     if kind == "zero2":

@@ -26,7 +26,7 @@ def test_bytes_per_parameter_follow_the_formula():
 
 def test_every_workload_has_a_kernel_label_and_valid_fields():
     for name, (kind, size, R, gdt, pdt, scaled) in bench.WORKLOADS.items():
-        assert kind in ("flat", "list", "z3gather", "z3step", "zero2emu", "zero2"), name
+        assert kind in ("flat", "list", "z3gather", "z3step", "gather", "zero2emu", "zero2"), name
         assert (kind == "zero2" and R == 0) or 1 <= R <= 256, name
         assert gdt in bench.GRAD_BYTES and pdt in ("bf16", "f16"), name
         label = bench.roofline_kernel(name)
